@@ -1,0 +1,226 @@
+/*
+ * g4attn -- Gemma 4 decoder attention layer on NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libg4attn.so.  Every pointer argument is a plain pointer: "device"
+ * means memory the calling process allocated on the current CUDA device,
+ * "host" means ordinary process memory.  All tensors are dense row-major
+ * (last dimension contiguous).  The library never allocates, frees or
+ * synchronises device memory except where a function says so; the caller
+ * owns every buffer, the stream and the workspace.  Calls enqueue work on the
+ * given stream (a cudaStream_t passed as void*, NULL = the legacy default
+ * stream) and return without waiting.
+ *
+ * Page passages that define the operations (page title, section):
+ *  [K1] "Gemma 4" (Keras port docs), "What changed from Gemma 3":
+ *       plain-weight RMSNorm; zero-pad partial rope on partial_rotary_factor
+ *       of each head; K=V global MQA at global_head_dim 512; image tokens
+ *       attend bidirectionally within each image block on sliding layers,
+ *       global layers stay causal; a tail of layers reuses an earlier
+ *       layer's K/V.
+ *  [K2] "Gemma 4" (Keras port docs), "Gemma4Model" argument table:
+ *       num_heads, num_kv_heads, num_global_kv_heads, head_dim,
+ *       global_head_dim, k_eq_v, sliding_window, partial_rotary_factor,
+ *       num_kv_shared_layers.
+ *  [K3] "Gemma 4" (Keras port docs), "Gemma4ConditionalGenerate": decoding
+ *       is text-only over the per-layer KV cache.
+ *  [P1] "gemma4-pt-claude" README, "Supported Models": every variant uses
+ *       QK-norm and V-norm; "Attention Backend Notes": norms multiply by the
+ *       weight (x_normed * weight).
+ *  [P2] "gemma4-pt-claude" README, "KV Cache": the cache is sized for
+ *       prompt + new tokens and a write past its end is an error;
+ *       sliding-window layers may use a rolling cache of
+ *       max(window, prompt) slots; global layers keep the full context.
+ *  [V1] "Gemma 4" overview blog, "Sliding-window attention" and "Global
+ *       attention layers": a sliding query sees a window of recent keys, a
+ *       global query every earlier key.
+ *  [V2] "Gemma 4" overview blog, "Dual RoPE configurations": standard RoPE
+ *       on sliding layers, proportional/pruned RoPE on global layers, each
+ *       two-dimensional subspace rotated by the 2x2 rotation matrix.
+ *  [V3] "Gemma 4" overview blog, "Shared KV Cache": later layers reuse the
+ *       K/V of the most recent earlier layer of the same type and compute
+ *       only their own queries.
+ *
+ * Definitions used throughout (readings of the pages, stated once):
+ *  - RMSNorm over the d values of one head: x / sqrt(mean(x^2) + eps) * w,
+ *    with the weight vector w[d] used as it is (no 1 + w) and shared by all
+ *    heads of the layer; V-norm is the same without a weight  [K1][P1].
+ *  - RoPE at the 0-based token position p: pair k is (x[k], x[k + d/2]);
+ *    for k < R = rotary_fraction * d / 2 it is rotated by the angle
+ *    p * rope_theta^(-2k/d); the pairs k >= R pass through unchanged
+ *    (a zero-padded frequency vector)  [K1][V2].
+ *  - K=V (k_eq_v): K = RoPE(RMSNorm(k_raw) * w_k), V = RMSNorm(k_raw):
+ *    one raw projection feeds both  [K1].
+ *  - Query head h reads KV head h / (num_heads / num_kv_heads)  [K2].
+ *  - Keys a query at position i sees: global layer [0, i]; sliding layer the
+ *    `window` most recent positions [max(0, i - window + 1), i]; a sliding
+ *    query inside an image block [s, e) sees the union of its window and the
+ *    whole block, [min(max(0, i - window + 1), s), e - 1]  [K1][V1].
+ *    An image block is a maximal run of equal non-negative ids in
+ *    image_block_ids; -1 marks text.
+ *  - o_i = sum_j softmax_j(softmax_scale * q_i . k_j) v_j over those keys.
+ */
+#ifndef G4ATTN_H
+#define G4ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes.  Host-checkable errors return before anything is enqueued. */
+typedef enum {
+  G4ATTN_OK = 0,
+  G4ATTN_EINVAL = 1,          /* bad argument (NULL, shape, inconsistent desc) */
+  G4ATTN_EUNSUPPORTED = 2,    /* valid layer the library has no kernel for */
+  G4ATTN_ECACHE_OVERFLOW = 3, /* a write past the end of a non-rolling cache */
+  G4ATTN_ECUDA = 4,           /* a CUDA runtime call failed */
+  G4ATTN_EDEVICE = 5,         /* a kernel recorded an error (see status word) */
+  G4ATTN_EWORKSPACE = 6,      /* workspace NULL or smaller than required */
+  G4ATTN_ECACHE_EMPTY = 7     /* decode on a sequence whose cache holds nothing */
+} g4attn_status;
+
+enum { G4ATTN_SLIDING = 0, G4ATTN_GLOBAL = 1 };
+enum { G4ATTN_BF16 = 0, G4ATTN_FP32 = 1 };
+
+/* One attention layer [K2].  Sliding layers: window > 0, typically
+ * rotary_fraction 1.0 and rope_theta 1e4.  Global layers: window ignored,
+ * typically rotary_fraction 0.25 and rope_theta 1e6, k_eq_v on the K=V
+ * variants.  rotary_fraction * head_dim must be an even integer.
+ * softmax_scale multiplies q.k (1/sqrt(head_dim) or 1.0; the pages print
+ * both); rms_eps is added to mean(x^2) (the pages do not state it; 1e-6 is
+ * the usual value).  dtype is the element type of every raw input, weight,
+ * output and cache tensor of the call. */
+typedef struct {
+  int layer_type;        /* G4ATTN_SLIDING or G4ATTN_GLOBAL */
+  int window;            /* keys per sliding query, itself included */
+  float rotary_fraction; /* fraction of each head that is rotated */
+  double rope_theta;     /* RoPE base */
+  int k_eq_v;            /* 1: V derives from the K projection (v_raw NULL) */
+  int num_heads;         /* Hq, query heads */
+  int num_kv_heads;      /* Hkv, divides Hq */
+  int head_dim;          /* d: 64, 128, 256 or 512 */
+  float softmax_scale;
+  float rms_eps;
+  int dtype;             /* G4ATTN_BF16 or G4ATTN_FP32 */
+} g4attn_layer_desc;
+
+/* A per-layer KV cache [P2], caller-owned device memory.  K and V are stored
+ * separately, also on K=V layers, each [batch, num_kv_heads, capacity,
+ * head_dim] in `dtype`, holding post-prologue values (K after RMSNorm * w_k
+ * and RoPE, V after V-norm).  len[b] (device int32) counts the positions of
+ * sequence b written so far.  A rolling cache keeps position p at slot
+ * p % capacity and needs capacity >= window; it is only valid on sliding
+ * layers.  A non-rolling cache keeps position p at slot p and rejects
+ * p >= capacity. */
+typedef struct {
+  void *k;
+  void *v;
+  int32_t *len;
+  int capacity;
+  int rolling;
+  int batch;
+  int num_kv_heads;
+  int head_dim;
+  int dtype;
+} g4attn_cache;
+
+/* Bytes of device workspace g4attn_prefill needs for this layer and size.
+ * Returns 0 if the arguments are invalid. */
+size_t g4attn_prefill_workspace_size(const g4attn_layer_desc *desc, int B,
+                                     int T);
+
+/* Bytes of device workspace g4attn_decode needs for this layer and cache
+ * (batch, capacity).  Returns 0 if the arguments are invalid. */
+size_t g4attn_decode_workspace_size(const g4attn_layer_desc *desc,
+                                    const g4attn_cache *cache);
+
+/* Prefill of a whole prompt (positions 0..T-1) through one layer
+ * [K1][V1][V2]: prologue on Q, K, V, then masked softmax attention.
+ *
+ *  q_raw           device [B, T, num_heads, d]: query projection output.
+ *  k_raw           device [B, T, num_kv_heads, d], or NULL for a KV-shared
+ *                  layer [V3], which then reads its keys/values from `cache`
+ *                  (positions 0..T-1 must be present there) and writes none.
+ *  v_raw           device [B, T, num_kv_heads, d]; must be NULL with k_eq_v
+ *                  or with k_raw NULL, non-NULL otherwise.
+ *  q_norm_w        device [d]: QK-norm weight of the queries, used as is.
+ *  k_norm_w        device [d]: QK-norm weight of the keys (ignored if k_raw
+ *                  is NULL).
+ *  image_block_ids device int32 [B, T] or NULL: -1 text, a block is a maximal
+ *                  run of one non-negative id.  Ignored on global layers.
+ *  cache           NULL, or a cache of this layer: with k_raw the post-prologue
+ *                  K/V of positions 0..T-1 are written to it (a rolling cache
+ *                  keeps the last `capacity` of them) and len[b] is set to T;
+ *                  a non-rolling cache needs capacity >= T.
+ *  out             device [B, T, num_heads, d]: attention output.
+ *  workspace       device scratch of g4attn_prefill_workspace_size bytes,
+ *                  256-byte aligned; its contents are not preserved.
+ *  stream          cudaStream_t.
+ *
+ * Errors: G4ATTN_EINVAL for bad shapes, NULLs, head_dim not in
+ * {64,128,256,512}, num_heads % num_kv_heads != 0, window <= 0 on a sliding
+ * layer, rotary_fraction * d not an even integer, cache shape or dtype
+ * mismatch, a rolling cache on a global layer; G4ATTN_ECACHE_OVERFLOW for a
+ * non-rolling cache with capacity < T; G4ATTN_EWORKSPACE; G4ATTN_ECUDA if a
+ * launch fails.  Nothing is written when an error is returned. */
+int g4attn_prefill(const g4attn_layer_desc *desc, int B, int T,
+                   const void *q_raw, const void *k_raw, const void *v_raw,
+                   const void *q_norm_w, const void *k_norm_w,
+                   const int32_t *image_block_ids, g4attn_cache *cache,
+                   void *out, void *workspace, size_t ws_bytes, void *stream);
+
+/* Append one token per sequence to a layer's cache [P2][K3]: the key/value
+ * prologue of k_raw/v_raw (device [B, 1, num_kv_heads, d]; v_raw NULL with
+ * k_eq_v) at position p = len[b], written at slot p (rolling: p % capacity),
+ * then len[b] = p + 1.  k_norm_w is device [d].
+ * If p >= capacity on a non-rolling cache nothing is written for that
+ * sequence, len[b] is unchanged and the device status word records
+ * G4ATTN_ECACHE_OVERFLOW (read it with g4attn_get_device_status). */
+int g4attn_cache_append(const g4attn_layer_desc *desc, g4attn_cache *cache,
+                        const void *k_raw, const void *v_raw,
+                        const void *k_norm_w, void *stream);
+
+/* Single-token decode [K3][V1][V3]: for every sequence b the query of the
+ * token at position P = len[b] - 1 (the last one appended) attends over the
+ * keys of row P of a prefill -- [max(0, P - window + 1), P] on a sliding
+ * layer, [0, P] on a global one -- read from `cache`.  A KV-shared layer
+ * passes the cache of the layer it reads and skips the append.
+ *
+ *  q_raw     device [B, 1, num_heads, d];  q_norm_w device [d].
+ *  out       device [B, 1, num_heads, d].
+ *  workspace device scratch of g4attn_decode_workspace_size bytes (split-KV
+ *            partials), 256-byte aligned.
+ *
+ * The keys are split into fixed-size chunks; each chunk yields a partial
+ * softmax (max, sum, weighted values) and a combine kernel merges them.
+ * A sequence with len[b] == 0 gets a zero output and the device status word
+ * records G4ATTN_ECACHE_EMPTY. */
+int g4attn_decode(const g4attn_layer_desc *desc, const g4attn_cache *cache,
+                  const void *q_raw, const void *q_norm_w, void *out,
+                  void *workspace, size_t ws_bytes, void *stream);
+
+/* Waits for `stream`, then returns and clears the device status word of the
+ * current device: G4ATTN_OK, or the first error a kernel recorded since the
+ * last call.  Returns G4ATTN_ECUDA if the wait or the copy fails. */
+int g4attn_get_device_status(void *stream);
+
+/* Optional timing hook: the next g4attn_prefill or g4attn_decode call on any
+ * stream records start_event immediately before and stop_event immediately
+ * after its attention kernel (the dominant launch), on the call's stream, and
+ * then forgets both.  The events are cudaEvent_t handles owned by the caller.
+ * Passing NULLs cancels a pending request. */
+void g4attn_time_next_attention(void *start_event, void *stop_event);
+
+/* Number of kernel launches the library has enqueued since it was loaded. */
+uint64_t g4attn_launch_count(void);
+
+/* Static text for a status code. */
+const char *g4attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* G4ATTN_H */
