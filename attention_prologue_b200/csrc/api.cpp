@@ -1,0 +1,262 @@
+// C-ABI entry points of libg4attn.so (declared in include/g4attn.h): host-side
+// validation, workspace layout and kernel launches on the caller's stream.
+// Nothing here allocates device memory or waits for the device, except
+// g4attn_get_device_status.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <atomic>
+
+#include <cuda_runtime.h>
+
+#include "g4attn.h"
+#include "g4attn_internal.h"
+
+namespace g4 {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+static std::mutex g_time_mu;
+static cudaEvent_t g_time_ev0 = nullptr, g_time_ev1 = nullptr;
+
+// Take (and forget) a pending timing request.
+static void take_timing(cudaEvent_t* e0, cudaEvent_t* e1) {
+  std::lock_guard<std::mutex> lock(g_time_mu);
+  *e0 = g_time_ev0;
+  *e1 = g_time_ev1;
+  g_time_ev0 = g_time_ev1 = nullptr;
+}
+
+static size_t elem_size(int dtype) { return dtype == G4ATTN_FP32 ? 4 : 2; }
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Validate a layer descriptor and derive the kernels' view of it.
+static int make_cfg(const g4attn_layer_desc* d, LayerCfg* L) {
+  if (!d) return G4ATTN_EINVAL;
+  if (d->layer_type != G4ATTN_SLIDING && d->layer_type != G4ATTN_GLOBAL) return G4ATTN_EINVAL;
+  if (d->dtype != G4ATTN_BF16 && d->dtype != G4ATTN_FP32) return G4ATTN_EINVAL;
+  if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256 && d->head_dim != 512)
+    return G4ATTN_EINVAL;
+  if (d->num_heads < 1 || d->num_kv_heads < 1 || d->num_kv_heads > 32) return G4ATTN_EINVAL;
+  if (d->num_heads % d->num_kv_heads != 0) return G4ATTN_EINVAL;
+  if (d->layer_type == G4ATTN_SLIDING && d->window < 1) return G4ATTN_EINVAL;
+  if (!(d->rotary_fraction >= 0.f && d->rotary_fraction <= 1.f)) return G4ATTN_EINVAL;
+  const double rd = (double)d->rotary_fraction * d->head_dim;  // rotated dims, even integer
+  const long R2 = std::lround(rd);
+  if (std::fabs(rd - (double)R2) > 1e-6 || (R2 & 1)) return G4ATTN_EINVAL;
+  if (!(d->rope_theta > 0.0) || !std::isfinite(d->rope_theta)) return G4ATTN_EINVAL;
+  if (!std::isfinite(d->softmax_scale)) return G4ATTN_EINVAL;
+  if (!(d->rms_eps >= 0.f) || !std::isfinite(d->rms_eps)) return G4ATTN_EINVAL;
+  if (d->k_eq_v != 0 && d->k_eq_v != 1) return G4ATTN_EINVAL;
+  L->layer_type = d->layer_type;
+  L->window = d->layer_type == G4ATTN_SLIDING ? d->window : 0;
+  L->k_eq_v = d->k_eq_v;
+  L->Hq = d->num_heads;
+  L->Hkv = d->num_kv_heads;
+  L->d = d->head_dim;
+  L->dtype = d->dtype;
+  L->scale = d->softmax_scale;
+  L->eps = d->rms_eps;
+  std::memset(&L->rope, 0, sizeof(L->rope));
+  L->rope.rotated_pairs = (int)(R2 / 2);
+  for (int k = 0; k < L->rope.rotated_pairs; ++k)
+    L->rope.inv_freq[k] = std::pow(d->rope_theta, -2.0 * k / (double)d->head_dim);
+  return G4ATTN_OK;
+}
+
+static int check_cache(const LayerCfg& L, const g4attn_cache* c, int B) {
+  if (!c->k || !c->v || !c->len) return G4ATTN_EINVAL;
+  if (c->batch != B || c->num_kv_heads != L.Hkv || c->head_dim != L.d || c->dtype != L.dtype)
+    return G4ATTN_EINVAL;
+  if (c->capacity < 1 || (c->rolling != 0 && c->rolling != 1)) return G4ATTN_EINVAL;
+  if (c->rolling && (L.layer_type != G4ATTN_SLIDING || c->capacity < L.window))
+    return G4ATTN_EINVAL;
+  return G4ATTN_OK;
+}
+
+// Workspace of one prefill call.
+struct PrefillWs {
+  size_t q_hat, kv, intervals, total;  // byte offsets / sizes
+  bool need_kv;                        // keys go to scratch (no usable cache)
+};
+
+static PrefillWs prefill_ws(const LayerCfg& L, int B, int T, bool need_kv, bool intervals) {
+  PrefillWs w;
+  const size_t es = elem_size(L.dtype);
+  size_t off = 0;
+  w.q_hat = off;
+  off += align256((size_t)B * T * L.Hq * L.d * es);
+  w.kv = off;
+  if (need_kv) off += 2 * align256((size_t)B * T * L.Hkv * L.d * es);
+  w.intervals = off;
+  if (intervals) off += 2 * align256((size_t)B * T * sizeof(int32_t));
+  w.total = off;
+  w.need_kv = need_kv;
+  return w;
+}
+
+}  // namespace g4
+
+using namespace g4;
+
+extern "C" {
+
+size_t g4attn_prefill_workspace_size(const g4attn_layer_desc* desc, int B, int T) {
+  LayerCfg L;
+  if (make_cfg(desc, &L) != G4ATTN_OK || B < 0 || T < 0) return 0;
+  return prefill_ws(L, B, T, true, L.layer_type == G4ATTN_SLIDING).total;
+}
+
+size_t g4attn_decode_workspace_size(const g4attn_layer_desc* desc, const g4attn_cache* cache) {
+  LayerCfg L;
+  if (make_cfg(desc, &L) != G4ATTN_OK || !cache) return 0;
+  if (check_cache(L, cache, cache->batch) != G4ATTN_OK) return 0;
+  return align256(decode_partials_bytes(L, cache->batch, decode_plan(L, cache->capacity)));
+}
+
+int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_raw,
+                   const void* k_raw, const void* v_raw, const void* q_norm_w,
+                   const void* k_norm_w, const int32_t* image_block_ids, g4attn_cache* cache,
+                   void* out, void* workspace, size_t ws_bytes, void* stream) {
+  LayerCfg L;
+  int st = make_cfg(desc, &L);
+  if (st != G4ATTN_OK) return st;
+  if (B < 0 || T < 0) return G4ATTN_EINVAL;
+  if (!q_raw || !q_norm_w || !out) return G4ATTN_EINVAL;
+  const bool shared = k_raw == nullptr;  // KV-shared layer: keys come from the cache
+  if (shared) {
+    if (v_raw || !cache) return G4ATTN_EINVAL;
+  } else {
+    if (!k_norm_w) return G4ATTN_EINVAL;
+    if ((v_raw == nullptr) != (L.k_eq_v == 1)) return G4ATTN_EINVAL;
+  }
+  if (cache) {
+    if ((st = check_cache(L, cache, B)) != G4ATTN_OK) return st;
+    if (!cache->rolling && cache->capacity < T) return G4ATTN_ECACHE_OVERFLOW;
+    if (shared && cache->capacity < T) return G4ATTN_EINVAL;  // evicted keys cannot be read
+  }
+  if (B == 0 || T == 0) return G4ATTN_OK;
+
+  // attention reads keys from the cache when it holds positions 0..T-1 at
+  // slots 0..T-1, otherwise from scratch
+  const bool cache_is_src = cache && cache->capacity >= T;
+  const bool intervals = L.layer_type == G4ATTN_SLIDING && image_block_ids != nullptr;
+  PrefillWs w = prefill_ws(L, B, T, !cache_is_src, intervals);
+  if (!workspace || ws_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return G4ATTN_EWORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t es = elem_size(L.dtype);
+
+  KVSrc src;
+  if (cache_is_src) {
+    src = {cache->k, cache->v, cache->capacity};
+  } else {
+    char* kbuf = ws + w.kv;
+    char* vbuf = kbuf + align256((size_t)B * T * L.Hkv * L.d * es);
+    src = {kbuf, vbuf, T};
+  }
+  cudaError_t e = cudaSuccess;
+  if (!shared) {
+    KVDst d0{const_cast<void*>(src.k), const_cast<void*>(src.v), src.cap, 0, 0};
+    KVDst d1{nullptr, nullptr, 1, 0, 0};
+    if (cache && !cache_is_src)  // rolling cache smaller than the prompt: last `cap` positions
+      d1 = {cache->k, cache->v, cache->capacity, 1, T - cache->capacity};
+    e = launch_kv_prologue(L, B, T, k_raw, v_raw, k_norm_w, d0, d1, cache ? cache->len : nullptr,
+                           s);
+    if (e != cudaSuccess) return G4ATTN_ECUDA;
+  }
+  RowIntervals rows{nullptr, nullptr};
+  if (intervals) {
+    int32_t* lo = reinterpret_cast<int32_t*>(ws + w.intervals);
+    int32_t* hi = reinterpret_cast<int32_t*>(ws + w.intervals +
+                                             align256((size_t)B * T * sizeof(int32_t)));
+    if (launch_block_intervals(L, B, T, image_block_ids, lo, hi, s) != cudaSuccess)
+      return G4ATTN_ECUDA;
+    rows = {lo, hi};
+  }
+  void* q_hat = ws + w.q_hat;
+  if (launch_q_prologue(L, B, T, q_raw, q_norm_w, q_hat, s) != cudaSuccess) return G4ATTN_ECUDA;
+  cudaEvent_t ev0, ev1;
+  take_timing(&ev0, &ev1);
+  if (ev0) cudaEventRecord(ev0, s);
+  e = launch_attention_simt(L, B, T, q_hat, src, rows, out, s);
+  if (ev1) cudaEventRecord(ev1, s);
+  return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
+}
+
+int g4attn_cache_append(const g4attn_layer_desc* desc, g4attn_cache* cache, const void* k_raw,
+                        const void* v_raw, const void* k_norm_w, void* stream) {
+  LayerCfg L;
+  int st = make_cfg(desc, &L);
+  if (st != G4ATTN_OK) return st;
+  if (!cache || !k_raw || !k_norm_w) return G4ATTN_EINVAL;
+  if ((v_raw == nullptr) != (L.k_eq_v == 1)) return G4ATTN_EINVAL;
+  if ((st = check_cache(L, cache, cache->batch)) != G4ATTN_OK) return st;
+  if (cache->batch == 0) return G4ATTN_OK;
+  cudaError_t e = launch_append(L, cache->batch, k_raw, v_raw, k_norm_w, cache->k, cache->v,
+                                cache->len, cache->capacity, cache->rolling, status_ptr(),
+                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
+}
+
+int g4attn_decode(const g4attn_layer_desc* desc, const g4attn_cache* cache, const void* q_raw,
+                  const void* q_norm_w, void* out, void* workspace, size_t ws_bytes,
+                  void* stream) {
+  LayerCfg L;
+  int st = make_cfg(desc, &L);
+  if (st != G4ATTN_OK) return st;
+  if (!cache || !q_raw || !q_norm_w || !out) return G4ATTN_EINVAL;
+  if ((st = check_cache(L, cache, cache->batch)) != G4ATTN_OK) return st;
+  if (cache->batch == 0) return G4ATTN_OK;
+  const DecodePlan plan = decode_plan(L, cache->capacity);
+  const size_t need = decode_partials_bytes(L, cache->batch, plan);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return G4ATTN_EWORKSPACE;
+  cudaEvent_t ev0, ev1;
+  take_timing(&ev0, &ev1);
+  cudaError_t e = launch_decode(L, cache->batch, q_raw, q_norm_w, cache->k, cache->v, cache->len,
+                                cache->capacity, cache->rolling, plan,
+                                static_cast<float*>(workspace), out, status_ptr(),
+                                static_cast<cudaStream_t>(stream), ev0, ev1);
+  return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
+}
+
+int g4attn_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return G4ATTN_ECUDA;
+  int* p = status_ptr();
+  if (!p) return G4ATTN_ECUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return G4ATTN_ECUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(p, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
+      return G4ATTN_ECUDA;
+  }
+  return v;
+}
+
+void g4attn_time_next_attention(void* start_event, void* stop_event) {
+  std::lock_guard<std::mutex> lock(g_time_mu);
+  g_time_ev0 = static_cast<cudaEvent_t>(start_event);
+  g_time_ev1 = static_cast<cudaEvent_t>(stop_event);
+}
+
+uint64_t g4attn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* g4attn_status_string(int status) {
+  switch (status) {
+    case G4ATTN_OK: return "ok";
+    case G4ATTN_EINVAL: return "invalid argument";
+    case G4ATTN_EUNSUPPORTED: return "unsupported layer";
+    case G4ATTN_ECACHE_OVERFLOW: return "write past the end of a non-rolling KV cache";
+    case G4ATTN_ECUDA: return "CUDA runtime error";
+    case G4ATTN_EDEVICE: return "a kernel recorded an error";
+    case G4ATTN_EWORKSPACE: return "workspace missing, too small or not 256-byte aligned";
+    case G4ATTN_ECACHE_EMPTY: return "decode on a sequence with an empty cache";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,85 @@
+// Internal interface between the C-ABI layer (api.cpp) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace g4 {
+
+constexpr int kMaxHalf = 256;  // head_dim <= 512
+
+// RoPE of one layer: pair k (k < rotated_pairs) turns by pos * inv_freq[k];
+// inv_freq[k] = theta^(-2k/d) computed on the host in fp64.
+struct RopeParams {
+  double inv_freq[kMaxHalf];
+  int rotated_pairs;
+};
+
+// Validated copy of g4attn_layer_desc.
+struct LayerCfg {
+  int layer_type;  // 0 sliding, 1 global
+  int window;
+  int k_eq_v;
+  int Hq, Hkv, d;
+  int dtype;  // 0 bf16, 1 fp32
+  float scale, eps;
+  RopeParams rope;
+};
+
+// Where the key/value prologue writes: [B, Hkv, cap, d]; positions t >= first
+// go to slot (rolling ? t % cap : t).  k == nullptr: no destination.
+struct KVDst {
+  void* k;
+  void* v;
+  int cap;
+  int rolling;
+  int first;
+};
+
+// Keys of one attention source: [B, Hkv, cap, d], position t at slot t.
+struct KVSrc {
+  const void* k;
+  const void* v;
+  int cap;
+};
+
+// Per-row key interval [lo[b*T+i], hi[b*T+i]] (image blocks), or nullptr
+// when the interval follows from the layer type and window alone.
+struct RowIntervals {
+  const int32_t* lo;
+  const int32_t* hi;
+};
+
+cudaError_t launch_q_prologue(const LayerCfg& L, int B, int T, const void* q_raw, const void* wq,
+                              void* q_hat, cudaStream_t s);
+cudaError_t launch_kv_prologue(const LayerCfg& L, int B, int T, const void* k_raw,
+                               const void* v_raw, const void* wk, KVDst d0, KVDst d1,
+                               int32_t* len_out, cudaStream_t s);
+cudaError_t launch_block_intervals(const LayerCfg& L, int B, int T, const int32_t* ids,
+                                   int32_t* lo, int32_t* hi, cudaStream_t s);
+cudaError_t launch_attention_simt(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
+                                  RowIntervals rows, void* out, cudaStream_t s);
+cudaError_t launch_append(const LayerCfg& L, int B, const void* k_raw, const void* v_raw,
+                          const void* wk, void* cache_k, void* cache_v, int32_t* len, int cap,
+                          int rolling, int* status, cudaStream_t s);
+
+// Split-KV decode.  Partials: m, l [B, Hq, n_chunks] and o~ [B, Hq, n_chunks, d], fp32.
+struct DecodePlan {
+  int chunk;     // keys per chunk
+  int n_chunks;  // chunks per (sequence, head), upper bound
+};
+DecodePlan decode_plan(const LayerCfg& L, int cap);
+size_t decode_partials_bytes(const LayerCfg& L, int B, const DecodePlan& p);
+cudaError_t launch_decode(const LayerCfg& L, int B, const void* q_raw, const void* wq,
+                          const void* cache_k, const void* cache_v, const int32_t* len, int cap,
+                          int rolling, const DecodePlan& plan, float* partials, void* out,
+                          int* status, cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1);
+
+// Device status word of the current device (nullptr if it cannot be found).
+int* status_ptr();
+
+// Kernel launches counter (incremented by every launcher).
+void count_launch(int n = 1);
+
+}  // namespace g4

@@ -1,0 +1,190 @@
+// Prologue kernels of the Gemma 4 attention layer ("Gemma 4" Keras docs,
+// "What changed from Gemma 3": plain-weight RMSNorm, zero-pad partial rope,
+// K=V; "gemma4-pt-claude" README, "Supported Models": QK-norm and V-norm),
+// the per-row interval pre-pass of image blocks, and the cache append
+// ("gemma4-pt-claude" README, "KV Cache").
+//
+// Memory-bound: one warp per head vector, 16-byte accesses where the head
+// size allows, fp32 arithmetic, fp64 RoPE angle reduction.
+#include <mutex>
+
+#include "common.cuh"
+#include "g4attn.h"
+
+namespace g4 {
+
+__device__ int g_status;  // first error recorded by a kernel, 0 = none
+
+int* status_ptr() {
+  static std::mutex mu;
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+constexpr int kWarps = 8;  // warps per block of the per-vector kernels
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kWarps * 32)
+    q_prologue_kernel(const T* __restrict__ q_raw, const T* __restrict__ wq, T* __restrict__ q_hat,
+                      long n_vec, int T_, int Hq, const __grid_constant__ RopeParams rope,
+                      float eps) {
+  const long v = (long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (v >= n_vec) return;
+  const long t = (v / Hq) % T_;
+  float y0[D / 64], y1[D / 64];
+  prologue_vec<T, D>(q_raw + v * D, wq, t, &rope, eps, y0, y1);
+  store_vec<T, D>(q_hat + v * D, y0, y1);
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void put_kv(const KVDst& d, int Hkv, long b, int h, long t,
+                                       const float* k0, const float* k1, const float* v0,
+                                       const float* v1) {
+  if (!d.k || t < d.first) return;
+  const long slot = d.rolling ? t % d.cap : t;
+  const long off = (((long)b * Hkv + h) * d.cap + slot) * D;
+  store_vec<T, D>(static_cast<T*>(d.k) + off, k0, k1);
+  store_vec<T, D>(static_cast<T*>(d.v) + off, v0, v1);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kWarps * 32)
+    kv_prologue_kernel(const T* __restrict__ k_raw, const T* __restrict__ v_raw,
+                       const T* __restrict__ wk, int B, int T_, int Hkv, KVDst d0, KVDst d1,
+                       int32_t* __restrict__ len_out, const __grid_constant__ RopeParams rope,
+                       float eps) {
+  const long v = (long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const long n_vec = (long)B * T_ * Hkv;
+  if (v >= n_vec) return;
+  const int h = (int)(v % Hkv);
+  const long t = (v / Hkv) % T_;
+  const long b = v / ((long)Hkv * T_);
+  float k0[D / 64], k1[D / 64], u0[D / 64], u1[D / 64];
+  prologue_vec<T, D>(k_raw + v * D, wk, t, &rope, eps, k0, k1);
+  // V-norm: no weight, no rotation; with K=V it reads the key projection
+  prologue_vec<T, D>((v_raw ? v_raw : k_raw) + v * D, nullptr, t, nullptr, eps, u0, u1);
+  put_kv<T, D>(d0, Hkv, b, h, t, k0, k1, u0, u1);
+  put_kv<T, D>(d1, Hkv, b, h, t, k0, k1, u0, u1);
+  if (len_out && t == 0 && h == 0 && (threadIdx.x & 31) == 0) len_out[b] = T_;
+}
+
+// lo/hi of every row of a sliding layer with image blocks: the window
+// [max(0, i-w+1), i] united with the maximal run of equal non-negative ids
+// that contains i.
+__global__ void block_interval_kernel(const int32_t* __restrict__ ids, int B, int T_, int window,
+                                      int32_t* __restrict__ lo, int32_t* __restrict__ hi) {
+  const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long)B * T_) return;
+  const int i = (int)(idx % T_);
+  const int32_t* row = ids + (idx - i);
+  int a = i - window + 1;
+  if (a < 0) a = 0;
+  int e = i;
+  const int id = row[i];
+  if (id >= 0) {
+    int s = i;
+    while (s > 0 && row[s - 1] == id) --s;
+    while (e + 1 < T_ && row[e + 1] == id) ++e;
+    if (s < a) a = s;
+  }
+  lo[idx] = a;
+  hi[idx] = e;
+}
+
+// One token per sequence into the cache: CTA b, warp h = KV head.
+template <typename T, int D>
+__global__ void append_kernel(const T* __restrict__ k_raw, const T* __restrict__ v_raw,
+                              const T* __restrict__ wk, T* __restrict__ cache_k,
+                              T* __restrict__ cache_v, int32_t* __restrict__ len, int Hkv, int cap,
+                              int rolling, int* status, const __grid_constant__ RopeParams rope,
+                              float eps) {
+  const int b = blockIdx.x;
+  const int h = threadIdx.x >> 5;
+  const int pos = len[b];
+  if (!rolling && pos >= cap) {  // whole block takes this branch
+    if (threadIdx.x == 0) record_status(status, G4ATTN_ECACHE_OVERFLOW);
+    return;
+  }
+  const long slot = rolling ? pos % cap : pos;
+  const long src = ((long)b * Hkv + h) * D;
+  const long dst = (((long)b * Hkv + h) * cap + slot) * D;
+  float y0[D / 64], y1[D / 64];
+  prologue_vec<T, D>(k_raw + src, wk, pos, &rope, eps, y0, y1);
+  store_vec<T, D>(cache_k + dst, y0, y1);
+  prologue_vec<T, D>((v_raw ? v_raw : k_raw) + src, nullptr, pos, nullptr, eps, y0, y1);
+  store_vec<T, D>(cache_v + dst, y0, y1);
+  __syncthreads();  // every warp has read len[b]
+  if (threadIdx.x == 0) len[b] = pos + 1;
+}
+
+// ---------------------------------------------------------------------------
+
+template <typename F>
+static cudaError_t dispatch(const LayerCfg& L, F&& f) {
+  // f.template operator()<T, D>() for the layer's dtype and head size
+  switch (L.d) {
+    case 64: return L.dtype ? f.template operator()<float, 64>() : f.template operator()<__nv_bfloat16, 64>();
+    case 128: return L.dtype ? f.template operator()<float, 128>() : f.template operator()<__nv_bfloat16, 128>();
+    case 256: return L.dtype ? f.template operator()<float, 256>() : f.template operator()<__nv_bfloat16, 256>();
+    case 512: return L.dtype ? f.template operator()<float, 512>() : f.template operator()<__nv_bfloat16, 512>();
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_q_prologue(const LayerCfg& L, int B, int T, const void* q_raw, const void* wq,
+                              void* q_hat, cudaStream_t s) {
+  const long n_vec = (long)B * T * L.Hq;
+  const unsigned grid = (unsigned)((n_vec + kWarps - 1) / kWarps);
+  return dispatch(L, [&]<typename E, int D>() {
+    q_prologue_kernel<E, D><<<grid, kWarps * 32, 0, s>>>(
+        static_cast<const E*>(q_raw), static_cast<const E*>(wq), static_cast<E*>(q_hat), n_vec, T,
+        L.Hq, L.rope, L.eps);
+    count_launch();
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t launch_kv_prologue(const LayerCfg& L, int B, int T, const void* k_raw,
+                               const void* v_raw, const void* wk, KVDst d0, KVDst d1,
+                               int32_t* len_out, cudaStream_t s) {
+  const long n_vec = (long)B * T * L.Hkv;
+  const unsigned grid = (unsigned)((n_vec + kWarps - 1) / kWarps);
+  return dispatch(L, [&]<typename E, int D>() {
+    kv_prologue_kernel<E, D><<<grid, kWarps * 32, 0, s>>>(
+        static_cast<const E*>(k_raw), static_cast<const E*>(v_raw), static_cast<const E*>(wk), B,
+        T, L.Hkv, d0, d1, len_out, L.rope, L.eps);
+    count_launch();
+    return cudaGetLastError();
+  });
+}
+
+cudaError_t launch_block_intervals(const LayerCfg& L, int B, int T, const int32_t* ids,
+                                   int32_t* lo, int32_t* hi, cudaStream_t s) {
+  const long n = (long)B * T;
+  block_interval_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ids, B, T, L.window, lo, hi);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(const LayerCfg& L, int B, const void* k_raw, const void* v_raw,
+                          const void* wk, void* cache_k, void* cache_v, int32_t* len, int cap,
+                          int rolling, int* status, cudaStream_t s) {
+  return dispatch(L, [&]<typename E, int D>() {
+    append_kernel<E, D><<<B, 32 * L.Hkv, 0, s>>>(
+        static_cast<const E*>(k_raw), static_cast<const E*>(v_raw), static_cast<const E*>(wk),
+        static_cast<E*>(cache_k), static_cast<E*>(cache_v), len, L.Hkv, cap, rolling, status,
+        L.rope, L.eps);
+    count_launch();
+    return cudaGetLastError();
+  });
+}
+
+}  // namespace g4

@@ -1,0 +1,525 @@
+"""Benchmark of the Gemma 4 attention layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--no-decode] [--no-cpu-baseline]
+
+Headline: prefill attention TFLOP/s counting unmasked FLOPs only
+(4 * d * sum_i |I_i| * Hq * B; 2d for QK^T and 2d for PV per allowed pair) on
+the E2B-shaped sliding layer (B 1, T 8192, 8 query heads on 1 KV head, head
+dim 256, window 512), one g4attn_prefill call (prologue included) per step.
+The same JSON line carries the second half of the metric, decode KV-cache
+GB/s on the 26B-A4B-shaped step (64 sequences, cache lengths uniform in
+[4096, 131072]; a sliding layer on a 1024-slot rolling cache, a K=V global
+layer and a KV-shared layer reading it).
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream; L2 is flushed (a 256 MiB write) before every timed
+prefill step, outside the events; the decode step reads ~36 GB, far more than
+L2.  Barrier + synchronize on both sides; the maximum over ranks is reported.
+With N > 1 every rank runs its own instance (independent sequences, no
+collective on the data path): weak scaling.
+
+--impl reference times the float64 CPU oracle (the only other implementation
+of this layer) on the same workload and metric, on a bounded row sample.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from attention_prologue_b200 import g4attn as G  # noqa: E402
+from attention_prologue_b200 import workloads as W  # noqa: E402
+
+METRIC = "prefill attn TFLOP/s (unmasked) & decode KV-cache GB/s, % of B200 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work
+
+def allowed_pairs(w: W.PrefillWorkload, ids: torch.Tensor | None) -> int:
+    """sum over sequences and rows of |I_i| (keys each query sees)."""
+    L, T = w.layer, w.T
+    i = np.arange(T, dtype=np.int64)
+    if L.layer_type == W.GLOBAL:
+        return int(w.B * (i + 1).sum())
+    total = 0
+    for b in range(w.B):
+        lo = np.maximum(0, i - L.window + 1)
+        hi = i.copy()
+        if ids is not None:
+            row = ids[b].cpu().numpy()
+            t = 0
+            while t < T:
+                if row[t] < 0:
+                    t += 1
+                    continue
+                e = t
+                while e + 1 < T and row[e + 1] == row[t]:
+                    e += 1
+                lo[t:e + 1] = np.minimum(lo[t:e + 1], t)
+                hi[t:e + 1] = e
+                t = e + 1
+        total += int((hi - lo + 1).sum())
+    return total
+
+
+def prefill_flops(w: W.PrefillWorkload, ids) -> float:
+    return 4.0 * w.layer.head_dim * w.layer.num_heads * allowed_pairs(w, ids)
+
+
+def decode_bytes(L: W.LayerShape, lens, es=2) -> float:
+    """K and V bytes of the keys the new tokens attend to (P = len, after the
+    append) plus q, out and the appended K/V."""
+    n = np.asarray(lens, np.int64) + 1
+    if L.layer_type == W.SLIDING:
+        n = np.minimum(n, L.window)
+    kv = float(n.sum()) * L.num_kv_heads * L.head_dim * 2 * es
+    return kv + len(lens) * L.head_dim * es * (2 * L.num_heads + 2 * L.num_kv_heads)
+
+
+# ---------------------------------------------------------------------------
+# environment
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """SM clock and clock-event reasons sampled through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._index = index
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return None
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def visible_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            return int(vis.split(",")[local_rank])
+        except ValueError:
+            return local_rank
+    return local_rank
+
+
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def desc_of(L: W.LayerShape, dtype=torch.bfloat16) -> G.LayerDesc:
+    return G.make_desc(L.layer_type, L.num_heads, L.num_kv_heads, L.head_dim, window=L.window,
+                       rotary_fraction=L.rotary_fraction, rope_theta=L.rope_theta,
+                       k_eq_v=L.k_eq_v, softmax_scale=L.scale, rms_eps=L.rms_eps, dtype=dtype)
+
+
+def made_events(n):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in ev:  # torch creates the CUDA event on first record
+        e.record()
+    torch.cuda.synchronize()
+    return ev
+
+
+# ---------------------------------------------------------------------------
+# prefill
+
+def bench_prefill(args, dist: Dist, pk: dict):
+    w = W.E2B_SLIDING
+    dev = torch.device("cuda", dist.local)
+    inp = W.prefill_inputs(w, dev, seed=dist.rank)
+    d = desc_of(w.layer)
+    out = torch.empty_like(inp["q_raw"])
+    ws = torch.empty(G.g4attn_prefill_workspace_size(d, w.B, w.T), dtype=torch.uint8, device=dev)
+    flops = prefill_flops(w, inp["image_block_ids"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        G.g4attn_prefill(d, inp["q_raw"], inp["k_raw"], inp["v_raw"], inp["q_norm_w"],
+                         inp["k_norm_w"], inp["image_block_ids"], out=out, workspace=ws,
+                         stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    K = args.steps
+    s0, s1, a0, a1 = (made_events(K) for _ in range(4))
+    torch.cuda.synchronize()
+    dist.barrier()
+    launches0 = G.g4attn_launch_count()
+    with ClockSampler(visible_index(dist.local)) as clk:
+        torch.cuda.synchronize()
+        dist.barrier()
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            G.g4attn_time_next_attention(a0[i], a1[i])
+            s0[i].record(stream)
+            step()
+            s1[i].record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+    launches = G.g4attn_launch_count() - launches0
+    step_ms = [s0[i].elapsed_time(s1[i]) for i in range(K)]
+    attn_ms = [a0[i].elapsed_time(a1[i]) for i in range(K)]
+    total_ms = dist.max(sum(step_ms))
+    value = dist.world * flops * K / (total_ms * 1e-3) / 1e12
+    attn_avg = statistics.mean(attn_ms)
+    achieved = flops / (attn_avg * 1e-3) / 1e12
+    status = G.g4attn_get_device_status()
+    if status != G.G4ATTN_OK:
+        raise RuntimeError(f"device status after prefill: {G.g4attn_status_string(status)}")
+
+    # end to end: host (pinned) inputs -> device, prefill, output -> host
+    host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in inp.items()}
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dev_in = {k: (torch.empty_like(v) if v is not None else None) for k, v in inp.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = host_out.numel() * host_out.element_size()
+
+    def e2e_step():
+        for k, v in host.items():
+            if v is not None:
+                dev_in[k].copy_(v, non_blocking=True)
+        G.g4attn_prefill(d, dev_in["q_raw"], dev_in["k_raw"], dev_in["v_raw"], dev_in["q_norm_w"],
+                         dev_in["k_norm_w"], dev_in["image_block_ids"], out=out, workspace=ws,
+                         stream=stream)
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    e0, e1 = made_events(K), made_events(K)
+    torch.cuda.synchronize()
+    dist.barrier()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        e0[i].record(stream)
+        e2e_step()
+        e1[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = dist.max(sum(e0[i].elapsed_time(e1[i]) for i in range(K)))
+    e2e_value = dist.world * flops * K / (e2e_ms * 1e-3) / 1e12
+
+    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    res = dict(
+        value=value, ms_per_step=total_ms / K, flops=flops, launches=launches,
+        clocks=clk.summary(),
+        roofline={"bound": "tensor", "kernel": "attention (g4attn_prefill)", "achieved": achieved,
+                  "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                  "algorithmic_per_launch": flops, "avg_launch_ms": attn_avg},
+        e2e={"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+             "d2h_bytes_per_step": d2h},
+        inputs=inp, workload=w)
+    del flush, ws
+    return res
+
+
+# ---------------------------------------------------------------------------
+# decode
+
+def bench_decode(args, dist: Dist, pk: dict):
+    w = W.A4B_DECODE
+    dev = torch.device("cuda", dist.local)
+    lens = W.decode_lengths(w, seed=dist.rank)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + dist.rank)
+    S, Gl = w.sliding, w.global_
+    from dataclasses import replace
+    X = replace(Gl, softmax_scale=Gl.scale)  # KV-shared layer: own queries, G's cache
+    s_tok = W.decode_token_inputs(S, w.batch, g, dev, w.dtype)
+    g_tok = W.decode_token_inputs(Gl, w.batch, g, dev, w.dtype)
+    x_tok = W.decode_token_inputs(X, w.batch, g, dev, w.dtype, with_kv=False)
+    s_cache = G.KVCache.allocate(w.batch, S.num_kv_heads, w.sliding_capacity, S.head_dim,
+                                 rolling=True, device=dev)
+    g_cache = G.KVCache.allocate(w.batch, Gl.num_kv_heads, w.global_capacity, Gl.head_dim,
+                                 device=dev)
+    W.fill_cache(s_cache.k, s_cache.v, lens, True, g)
+    W.fill_cache(g_cache.k, g_cache.v, lens, False, g)
+    lens_dev = torch.as_tensor(lens, dtype=torch.int32, device=dev)
+    ds, dg, dx = desc_of(S), desc_of(Gl), desc_of(X)
+    outs = {k: torch.empty_like(t["q_raw"]) for k, t in (("s", s_tok), ("g", g_tok), ("x", x_tok))}
+    ws_s = torch.empty(G.g4attn_decode_workspace_size(ds, s_cache), dtype=torch.uint8, device=dev)
+    ws_g = torch.empty(G.g4attn_decode_workspace_size(dg, g_cache), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    nbytes = decode_bytes(S, lens) + decode_bytes(Gl, lens) + decode_bytes(X, lens)
+
+    def reset():
+        s_cache.len.copy_(lens_dev)
+        g_cache.len.copy_(lens_dev)
+
+    def step(ev=None):
+        G.g4attn_cache_append(ds, s_cache, s_tok["k_raw"], s_tok["v_raw"], s_tok["k_norm_w"], stream)
+        G.g4attn_decode(ds, s_cache, s_tok["q_raw"], s_tok["q_norm_w"], outs["s"], ws_s, stream)
+        G.g4attn_cache_append(dg, g_cache, g_tok["k_raw"], None, g_tok["k_norm_w"], stream)
+        if ev:
+            G.g4attn_time_next_attention(*ev)
+        G.g4attn_decode(dg, g_cache, g_tok["q_raw"], g_tok["q_norm_w"], outs["g"], ws_g, stream)
+        G.g4attn_decode(dx, g_cache, x_tok["q_raw"], x_tok["q_norm_w"], outs["x"], ws_g, stream)
+
+    for _ in range(args.warmup):
+        reset()
+        step()
+    K = args.steps
+    s0, s1, a0, a1 = (made_events(K) for _ in range(4))
+    torch.cuda.synchronize()
+    dist.barrier()
+    launches0 = G.g4attn_launch_count()
+    with ClockSampler(visible_index(dist.local)) as clk:
+        for i in range(K):
+            reset()
+            s0[i].record(stream)
+            step((a0[i], a1[i]))
+            s1[i].record(stream)
+        torch.cuda.synchronize()
+    dist.barrier()
+    launches = G.g4attn_launch_count() - launches0
+    total_ms = dist.max(sum(s0[i].elapsed_time(s1[i]) for i in range(K)))
+    status = G.g4attn_get_device_status()
+    if status != G.G4ATTN_OK:
+        raise RuntimeError(f"device status after decode: {G.g4attn_status_string(status)}")
+    g_ms = statistics.mean(a0[i].elapsed_time(a1[i]) for i in range(K))
+    g_split_bytes = decode_bytes(Gl, lens)
+    peak = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    achieved = g_split_bytes / (g_ms * 1e-3) / 1e9
+    res = {"metric": "decode KV-cache GB/s", "value": dist.world * nbytes * K / (total_ms * 1e-3) / 1e9,
+           "unit": "GB/s", "ms_per_step": total_ms / K, "bytes_per_step": nbytes,
+           "workload": w.name, "batch": w.batch, "len_range": [w.len_lo, w.len_hi],
+           "layers": ["sliding 16/8 d256 w1024 rolling 1024", "global K=V 16/2 d512",
+                      "KV-shared global 16/2 d512"],
+           "roofline": {"bound": "hbm", "kernel": "decode split-KV (global layer)",
+                        "achieved": achieved, "peak": peak, "unit": "GB/s",
+                        "frac": achieved / peak, "frac_of_8000": achieved / 8000.0,
+                        "traffic": None, "algorithmic_per_launch": g_split_bytes,
+                        "avg_launch_ms": g_ms},
+           "gpu_launches": launches, "clocks": clk.summary()}
+    del g_cache, s_cache
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and the reference arm)
+
+def oracle_sample(w: W.PrefillWorkload, inp: dict, stride: int, threads: int):
+    """Oracle on every `stride`-th query row (all heads, all sequences), plus
+    its key/value prologue charged pro rata.  Returns (TFLOP/s, seconds, rows)."""
+    import oracle
+    cpu = {k: (v.cpu() if v is not None else None) for k, v in inp.items()}
+    ol = oracle.Layer(layer_type=w.layer.layer_type, window=w.layer.window,
+                      rotary_fraction=w.layer.rotary_fraction, rope_theta=w.layer.rope_theta,
+                      k_eq_v=w.layer.k_eq_v, num_heads=w.layer.num_heads,
+                      num_kv_heads=w.layer.num_kv_heads, head_dim=w.layer.head_dim,
+                      softmax_scale=w.layer.scale, rms_eps=w.layer.rms_eps)
+    t0 = time.perf_counter()
+    kh, vh = oracle.prefill_kv(ol, cpu["k_raw"], cpu["v_raw"], cpu["k_norm_w"], threads)
+    t_kv = time.perf_counter() - t0
+    rows = list(range(0, w.T, stride))
+    ids = cpu["image_block_ids"]
+    t0 = time.perf_counter()
+    oracle.prefill_rows(ol, cpu["q_raw"], cpu["q_norm_w"], kh, vh,
+                        None if ids is None else ids.numpy(), rows, threads)
+    t_rows = time.perf_counter() - t0
+    i = np.asarray(rows, np.int64)
+    if w.layer.layer_type == W.GLOBAL:
+        pairs = w.B * (i + 1).sum()
+    else:
+        pairs = w.B * (i - np.maximum(0, i - w.layer.window + 1) + 1).sum()
+    flops = 4.0 * w.layer.head_dim * w.layer.num_heads * float(pairs)
+    secs = t_rows + t_kv * len(rows) / w.T
+    return flops / secs / 1e12, secs, len(rows)
+
+
+def pick_stride(w, inp, threads, target_s):
+    """Row stride whose sample takes about target_s seconds (calibrated)."""
+    probe = max(1, w.T // 64)
+    _, secs, _ = oracle_sample(w, inp, probe, threads)
+    per_row = secs / math.ceil(w.T / probe)
+    return max(1, int(math.ceil(w.T * per_row / target_s)))
+
+
+def cpu_baseline(w, inp, target_s=12.0):
+    import oracle
+    oracle.build()
+    threads = oracle.default_threads()
+    stride = pick_stride(w, inp, threads, target_s)
+    v, secs, n = oracle_sample(w, inp, stride, threads)
+    return {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{w.name}: every {stride}th query row ({n} rows x {w.layer.num_heads} heads, "
+                      f"{secs:.1f} s) plus the K/V prologue charged pro rata; float64 C, "
+                      f"{threads} threads"}
+
+
+def run_reference(args, dist: Dist):
+    if dist.rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    w = W.E2B_SLIDING
+    inp = W.prefill_inputs(w, "cpu", seed=0)
+    threads = oracle.default_threads()
+    per_step = min(10.0, 150.0 / max(1, args.steps + args.warmup))
+    stride = pick_stride(w, inp, threads, per_step)
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, stride, threads)
+    vals, secs = [], 0.0
+    for _ in range(args.steps):
+        v, s, n = oracle_sample(w, inp, stride, threads)
+        vals.append(v)
+        secs += s
+    value = float(np.mean(vals))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.T,
+                       "heads": [w.layer.num_heads, w.layer.num_kv_heads],
+                       "head_dim": w.layer.head_dim, "window": w.layer.window},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                             "sample": f"every {stride}th query row of {w.name}, all heads"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    dist = Dist() if args.impl == "ours" else None
+    if args.impl == "reference":
+        class _D:  # reference arm: CPU only, rank 0 prints
+            rank = int(os.environ.get("RANK", "0"))
+        return run_reference(args, _D())
+
+    torch.cuda.set_device(dist.local)
+    G.lib()  # fail loudly if the CUDA library is missing
+    pk, pk_src = peaks()
+    pre = bench_prefill(args, dist, pk)
+    dec = None if args.no_decode else bench_decode(args, dist, pk)
+    cpu = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(pre["workload"], pre["inputs"])
+    w = pre["workload"]
+    roof = dict(pre["roofline"])
+    roof["peak_source"] = f"{pk_src}: bf16_tflops (burst)"
+    if dec:
+        dec["roofline"]["peak_source"] = f"{pk_src}: hbm_gbs"
+    line = {"metric": METRIC, "value": pre["value"], "unit": "TFLOP/s", "n_gpus": dist.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": w.B * dist.world, "seq_len": w.T,
+                       "heads": [w.layer.num_heads, w.layer.num_kv_heads],
+                       "head_dim": w.layer.head_dim, "window": w.layer.window,
+                       "parallelism": f"replicas{dist.world}",
+                       "l2": "flushed (256 MiB write) before every timed prefill step",
+                       "unmasked_gflop_per_step": pre["flops"] / 1e9},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": pre["e2e"],
+            "gpu_launches": pre["launches"], "clocks": pre["clocks"], "decode": dec}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

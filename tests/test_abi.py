@@ -1,0 +1,165 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+include/g4attn.h declares, and rejects bad arguments before touching the GPU.
+No test here launches a kernel (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from attention_prologue_b200 import g4attn as G
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "g4attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(g4attn_\w+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_function():
+    lib = G.lib()
+    declared = header_functions()
+    assert set(declared) == set(G.EXPORTED)
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch):
+    monkeypatch.setattr(G, "_lib", None)
+    monkeypatch.setattr(G, "_LIB_PATH", "/nonexistent/libg4attn.so")
+    with pytest.raises(RuntimeError):
+        G.lib()
+
+
+def desc(**kw):
+    base = dict(layer_type=G.G4ATTN_SLIDING, num_heads=8, num_kv_heads=2, head_dim=256,
+                window=512)
+    base.update(kw)
+    return G.make_desc(base.pop("layer_type"), base.pop("num_heads"), base.pop("num_kv_heads"),
+                       base.pop("head_dim"), **base)
+
+
+def prefill_rc(d, B=1, T=16, k=FAKE, v=FAKE, ids=None, cache=None, ws=FAKE, ws_bytes=1 << 40):
+    return G.lib().g4attn_prefill(ctypes.byref(d), B, T, FAKE, k, v, FAKE, FAKE, ids,
+                                  ctypes.byref(cache) if cache is not None else None, FAKE, ws,
+                                  ws_bytes, None)
+
+
+def ccache(d, B=1, C=64, rolling=0, **kw):
+    c = G._CCache(FAKE, FAKE, FAKE, C, rolling, B, d.num_kv_heads, d.head_dim, d.dtype)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("bad", [
+    dict(head_dim=96), dict(head_dim=1024), dict(num_heads=6, num_kv_heads=4),
+    dict(num_kv_heads=0), dict(num_heads=64, num_kv_heads=64), dict(window=0),
+    dict(rotary_fraction=0.3), dict(rotary_fraction=1.5), dict(rope_theta=-1.0),
+    dict(rms_eps=-1.0), dict(softmax_scale=float("inf")), dict(layer_type=2),
+])
+def test_bad_descriptors_are_rejected(bad):
+    d = desc(**bad)
+    assert prefill_rc(d) == G.G4ATTN_EINVAL
+    assert G.lib().g4attn_prefill_workspace_size(ctypes.byref(d), 1, 16) == 0
+
+
+def test_bad_dtype_code_is_rejected():
+    d = desc()
+    d.dtype = 7
+    assert prefill_rc(d) == G.G4ATTN_EINVAL
+
+
+def test_k_eq_v_and_value_pointer_must_agree():
+    assert prefill_rc(desc(k_eq_v=True)) == G.G4ATTN_EINVAL  # v_raw given with K=V
+    assert prefill_rc(desc(k_eq_v=False), v=None) == G.G4ATTN_EINVAL  # v_raw missing
+    d = desc(layer_type=G.G4ATTN_GLOBAL, head_dim=512, rotary_fraction=0.25, k_eq_v=True)
+    assert prefill_rc(d, v=None, ws=None, ws_bytes=0) == G.G4ATTN_EWORKSPACE
+
+
+def test_kv_shared_prefill_needs_a_cache_holding_the_prompt():
+    d = desc()
+    assert prefill_rc(d, k=None, v=None) == G.G4ATTN_EINVAL  # no cache to read
+    assert prefill_rc(d, k=None, v=None, cache=ccache(d, C=8, rolling=0), T=16) == \
+        G.G4ATTN_ECACHE_OVERFLOW
+    dr = desc(window=8)
+    assert prefill_rc(dr, k=None, v=None, cache=ccache(dr, C=8, rolling=1), T=16) == \
+        G.G4ATTN_EINVAL
+
+
+def test_cache_checks():
+    d = desc()
+    assert prefill_rc(d, cache=ccache(d, C=8)) == G.G4ATTN_ECACHE_OVERFLOW  # T=16 > C
+    assert prefill_rc(d, cache=ccache(d, B=2)) == G.G4ATTN_EINVAL  # batch mismatch
+    assert prefill_rc(d, cache=ccache(d, head_dim=128)) == G.G4ATTN_EINVAL
+    assert prefill_rc(d, cache=ccache(d, num_kv_heads=1)) == G.G4ATTN_EINVAL
+    assert prefill_rc(d, cache=ccache(d, dtype=G.G4ATTN_FP32)) == G.G4ATTN_EINVAL
+    assert prefill_rc(d, cache=ccache(d, C=256, rolling=1)) == G.G4ATTN_EINVAL  # C < window
+    g = desc(layer_type=G.G4ATTN_GLOBAL, head_dim=512, rotary_fraction=0.25, k_eq_v=True)
+    assert prefill_rc(g, v=None, cache=ccache(g, C=1024, rolling=1)) == G.G4ATTN_EINVAL
+    c = ccache(d)
+    c.k = None
+    assert prefill_rc(d, cache=c) == G.G4ATTN_EINVAL
+
+
+def test_append_and_decode_validation():
+    lib = G.lib()
+    d = desc()
+    c = ccache(d, C=512)
+    assert lib.g4attn_cache_append(ctypes.byref(d), None, FAKE, FAKE, FAKE, None) == G.G4ATTN_EINVAL
+    assert lib.g4attn_cache_append(ctypes.byref(d), ctypes.byref(c), FAKE, None, FAKE, None) == \
+        G.G4ATTN_EINVAL
+    assert lib.g4attn_decode(ctypes.byref(d), ctypes.byref(c), FAKE, FAKE, FAKE, None, 0, None) == \
+        G.G4ATTN_EWORKSPACE
+    assert lib.g4attn_decode(ctypes.byref(d), ctypes.byref(c), None, FAKE, FAKE, FAKE, 1 << 30,
+                             None) == G.G4ATTN_EINVAL
+    # misaligned workspace
+    assert lib.g4attn_decode(ctypes.byref(d), ctypes.byref(c), FAKE, FAKE, FAKE,
+                             ctypes.c_void_p(0x10010), 1 << 30, None) == G.G4ATTN_EWORKSPACE
+
+
+def test_empty_inputs_are_a_no_op():
+    d = desc()
+    assert prefill_rc(d, B=0) == G.G4ATTN_OK
+    assert prefill_rc(d, T=0) == G.G4ATTN_OK
+    assert prefill_rc(d, B=-1) == G.G4ATTN_EINVAL
+
+
+def test_workspace_sizes():
+    d = desc(num_heads=8, num_kv_heads=1, head_dim=256, window=512)
+    B, T = 1, 8192
+    ws = G.lib().g4attn_prefill_workspace_size(ctypes.byref(d), B, T)
+    # q_hat + K/V scratch + two int32 interval arrays, 256-aligned pieces
+    assert ws == B * T * 8 * 256 * 2 + 2 * B * T * 1 * 256 * 2 + 2 * B * T * 4
+    c = ccache(d, B=64, C=1024, rolling=1)
+    dws = G.lib().g4attn_decode_workspace_size(ctypes.byref(d), ctypes.byref(c))
+    assert dws > 0 and dws % 256 == 0
+
+
+def test_status_strings():
+    for code in range(8):
+        assert G.g4attn_status_string(code) != "unknown status"
+    assert G.g4attn_status_string(99) == "unknown status"
+
+
+def test_cache_layout_reproduces_the_printed_kv_table():
+    """The cache stores K and V separately (also on K=V global layers), bf16,
+    [batch, kv_heads, capacity, head_dim]: the only layout that reproduces the
+    KV-cache table of the "gemma4-pt-claude" README."""
+    rows = [l.split() for l in open(os.path.join(ROOT, "tests", "golden", "kv_cache_table.txt"))
+            if l.strip() and not l.startswith("#")]
+    assert len(rows) == 2
+    for (model, layers, skv, hd, gkv, ghd, pattern, window, ctx, full, windowed) in rows:
+        layers, skv, hd, gkv, ghd, pattern, window, ctx = map(
+            int, (layers, skv, hd, gkv, ghd, pattern, window, ctx))
+        n_global = layers // pattern
+        n_sliding = layers - n_global
+        glob = n_global * G.cache_bytes(1, gkv, ctx, ghd, torch.bfloat16)
+        full_b = n_sliding * G.cache_bytes(1, skv, ctx, hd, torch.bfloat16) + glob
+        win_b = n_sliding * G.cache_bytes(1, skv, window, hd, torch.bfloat16) + glob
+        assert round(full_b / 1e9, 1) == float(full), model
+        assert round(win_b / 1e9, 1) == float(windowed), model

@@ -1,0 +1,149 @@
+"""GPU parity of g4attn_prefill (prologue + sliding / image-block / global
+attention) against the float64 oracle, element by element, on seeded inputs.
+
+Small cases run the whole output; the full-size workloads (the bench's launch
+configuration) are checked on sampled rows the oracle computes one by one."""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_prologue_b200 import g4attn as G
+from attention_prologue_b200 import workloads as W
+
+from helpers import (check, desc_of, gpu_prefill, oracle_layer, oracle_prefill, sample_rows)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def run_case(w, seed=0, rows=None, cache=None):
+    inp = W.prefill_inputs(w, DEV, seed)
+    out = gpu_prefill(w, inp, cache)
+    ref = oracle_prefill(w, inp, rows)
+    got = out if rows is None else out[:, rows]
+    return check(got, ref, w.dtype, w.name), inp, out
+
+
+# -- tiny fp32 configuration (both layers, both softmax scales) ---------------
+
+@pytest.mark.parametrize("w", [W.TINY_SLIDING, W.TINY_GLOBAL])
+@pytest.mark.parametrize("scale", [None, 1.0])
+def test_tiny_fp32(w, scale):
+    w = replace(w, layer=replace(w.layer, softmax_scale=scale))
+    run_case(w)
+
+
+# -- scaled-down bf16 shapes of each workload (several tiles + ragged tail) ---
+
+SMALL = [
+    W.scaled_down(W.E2B_SLIDING, T=1000),
+    W.scaled_down(W.E2B_SLIDING, T=300, B=2, window=64),
+    replace(W.scaled_down(W.G12B_SLIDING_MM, T=1200, B=2, num_heads=4, num_kv_heads=2,
+                          window=256), n_blocks=2),  # 280-token blocks > window 256
+    W.scaled_down(W.G31B_GLOBAL, T=700, num_heads=8, num_kv_heads=1),
+    W.scaled_down(W.G31B_GLOBAL, T=333, num_heads=4, num_kv_heads=2, k_eq_v=False),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_small_bf16(w):
+    run_case(w, seed=3)
+
+
+@pytest.mark.parametrize("hd", [64, 128])
+def test_other_head_dims(hd):
+    w = W.PrefillWorkload(f"hd{hd}", W.sliding(4, 2, hd, 40), 2, 150)
+    run_case(w, seed=5)
+    g = W.PrefillWorkload(f"g-hd{hd}", W.global_(4, 1, hd), 1, 150)
+    run_case(g, seed=6)
+
+
+# -- edge cases ---------------------------------------------------------------
+
+@pytest.mark.parametrize("T", [1, 2, 127, 129])
+def test_short_prompts(T):
+    run_case(W.PrefillWorkload(f"s{T}", W.sliding(8, 1, 256, 512), 1, T), seed=T)
+    run_case(W.PrefillWorkload(f"g{T}", W.global_(8, 1, 512), 1, T), seed=T)
+
+
+def test_blocks_at_the_edges_and_block_longer_than_window():
+    L = W.sliding(2, 1, 256, 32)
+    w = W.PrefillWorkload("edges", L, 2, 200)
+    inp = W.prefill_inputs(w, DEV, 11)
+    ids = torch.full((2, 200), -1, dtype=torch.int32)
+    ids[0, 0:50] = 0      # block at the start, longer than the window
+    ids[0, 120:200] = 1   # block at the end
+    ids[1, 60:61] = 4     # one-token block
+    ids[1, 61:100] = 5    # adjacent block with another id
+    inp["image_block_ids"] = ids.to(DEV)
+    out = gpu_prefill(w, inp)
+    check(out, oracle_prefill(w, inp), w.dtype, "edges")
+
+
+def test_global_layer_ignores_block_ids():
+    w = W.PrefillWorkload("g-ids", W.global_(4, 1, 512), 1, 300)
+    inp = W.prefill_inputs(w, DEV, 2)
+    a = gpu_prefill(w, inp)
+    inp["image_block_ids"] = torch.zeros(1, 300, dtype=torch.int32, device=DEV)
+    b = gpu_prefill(w, inp)
+    assert torch.equal(a, b)
+
+
+# -- cache writes, rolling cache, KV sharing ----------------------------------
+
+@pytest.mark.parametrize("rolling,cap", [(False, 700), (True, 512), (True, 600)])
+def test_cache_contents(rolling, cap):
+    """The post-prologue K/V written to the cache equal the oracle's k_hat,
+    v_hat (to bf16 rounding); a rolling cache smaller than the prompt keeps the
+    last `cap` positions at slot p % cap; len is set to T."""
+    w = W.PrefillWorkload("cache", W.sliding(8, 2, 256, 512), 2, 650)
+    inp = W.prefill_inputs(w, DEV, 4)
+    cache = G.KVCache.allocate(2, 2, cap, 256, rolling=rolling, device=DEV)
+    out = gpu_prefill(w, inp, cache)
+    check(out, oracle_prefill(w, inp), w.dtype, "out")
+    assert cache.len.tolist() == [650, 650]
+    kh, vh = oracle.prefill_kv(oracle_layer(w.layer), inp["k_raw"].cpu(), inp["v_raw"].cpu(),
+                               inp["k_norm_w"].cpu())
+    first = max(0, 650 - cap)
+    pos = np.arange(first, 650)
+    slots = pos % cap if rolling else pos
+    got_k = cache.k[:, :, slots].permute(0, 2, 1, 3)
+    got_v = cache.v[:, :, slots].permute(0, 2, 1, 3)
+    for got, ref in ((got_k, kh[:, pos]), (got_v, vh[:, pos])):
+        g = got.double().cpu().numpy()
+        assert np.max(np.abs(g - ref) / (np.abs(ref) + 1e-3)) < 2 ** -8 + 1e-6
+
+
+def test_kv_shared_prefill_reads_the_source_cache():
+    """A KV-shared layer passes k_raw = NULL and attends over the source
+    layer's cache with its own queries (overview blog, "Shared KV Cache")."""
+    src = W.PrefillWorkload("src", W.global_(8, 2, 512), 1, 400)
+    inp = W.prefill_inputs(src, DEV, 8)
+    cache = G.KVCache.allocate(1, 2, 512, 512, device=DEV)
+    gpu_prefill(src, inp, cache)
+    shared = W.PrefillWorkload("shared", replace(src.layer, softmax_scale=0.07), 1, 400)
+    sh = W.prefill_inputs(shared, DEV, 9)
+    d = desc_of(shared.layer, shared.dtype)
+    out = G.g4attn_prefill(d, sh["q_raw"], None, None, sh["q_norm_w"], None, cache=cache)
+    torch.cuda.synchronize()
+    ref = oracle.prefill(oracle_layer(shared.layer), sh["q_raw"].cpu(), inp["k_raw"].cpu(), None,
+                         sh["q_norm_w"].cpu(), inp["k_norm_w"].cpu())
+    check(out, ref, shared.dtype, "kv-shared")
+
+
+# -- full-size workloads, sampled rows ----------------------------------------
+
+@pytest.mark.parametrize("w,n", [(W.E2B_SLIDING, 96), (W.G12B_SLIDING_MM, 64),
+                                 (W.G31B_GLOBAL, 24)], ids=lambda x: getattr(x, "name", str(x)))
+def test_full_size_sampled(w, n):
+    rows = sample_rows(w.T, n)
+    if w.n_blocks:
+        ids = W.make_block_ids(w.B, w.T, w.n_blocks, w.block_len, 0)[0].numpy()
+        starts = [i for i in range(w.T) if ids[i] >= 0 and (i == 0 or ids[i - 1] != ids[i])]
+        for s in starts:  # rows at both ends of each image block of sequence 0
+            rows += [s, s + 1, s + w.block_len - 1, s + w.block_len]
+        rows = sorted(set(rows))
+    run_case(w, seed=0, rows=rows)
