@@ -223,6 +223,19 @@ int g4attn_decode(const g4attn_layer_desc* desc, const g4attn_cache* cache, cons
   return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
 }
 
+int g4attn_decode_noalloc(const g4attn_layer_desc* desc, const g4attn_cache* cache,
+                          const void* q_raw, const void* q_norm_w, void* out, void* stream) {
+  LayerCfg L;
+  int st = make_cfg(desc, &L);
+  if (st != G4ATTN_OK) return st;
+  if (!cache || !q_raw || !q_norm_w || !out) return G4ATTN_EINVAL;
+  if ((st = check_cache(L, cache, cache->batch)) != G4ATTN_OK) return st;
+  if (cache->batch == 0) return G4ATTN_OK;
+  return launch_decode_noalloc(L, cache->batch, q_raw, q_norm_w, cache->k, cache->v, cache->len,
+                               cache->capacity, cache->rolling, out, status_ptr(),
+                               static_cast<cudaStream_t>(stream));
+}
+
 int g4attn_get_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return G4ATTN_ECUDA;
   int* p = status_ptr();

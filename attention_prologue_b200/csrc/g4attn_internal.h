@@ -76,6 +76,12 @@ cudaError_t launch_decode(const LayerCfg& L, int B, const void* q_raw, const voi
                           int rolling, const DecodePlan& plan, float* partials, void* out,
                           int* status, cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1);
 
+// g4attn_decode with the split-KV partials in the library's fixed device
+// array instead of a workspace; returns a g4attn_status code.
+int launch_decode_noalloc(const LayerCfg& L, int B, const void* q_raw, const void* wq,
+                          const void* cache_k, const void* cache_v, const int32_t* len, int cap,
+                          int rolling, void* out, int* status, cudaStream_t s);
+
 // Device status word of the current device (nullptr if it cannot be found).
 int* status_ptr();
 

@@ -21,8 +21,9 @@ G4ATTN_SLIDING, G4ATTN_GLOBAL = 0, 1
 G4ATTN_BF16, G4ATTN_FP32 = 0, 1
 
 EXPORTED = ("g4attn_prefill_workspace_size", "g4attn_decode_workspace_size", "g4attn_prefill",
-            "g4attn_cache_append", "g4attn_decode", "g4attn_get_device_status",
-            "g4attn_time_next_attention", "g4attn_launch_count", "g4attn_status_string")
+            "g4attn_cache_append", "g4attn_decode", "g4attn_decode_noalloc",
+            "g4attn_get_device_status", "g4attn_time_next_attention", "g4attn_launch_count",
+            "g4attn_status_string")
 
 
 class G4AttnError(RuntimeError):
@@ -71,6 +72,8 @@ def lib() -> ctypes.CDLL:
         L.g4attn_cache_append.restype = I
         L.g4attn_decode.argtypes = [DP, CP, P, P, P, P, S, P]
         L.g4attn_decode.restype = I
+        L.g4attn_decode_noalloc.argtypes = [DP, CP, P, P, P, P]
+        L.g4attn_decode_noalloc.restype = I
         L.g4attn_get_device_status.argtypes = [P]
         L.g4attn_get_device_status.restype = I
         L.g4attn_time_next_attention.argtypes = [P, P]
@@ -226,6 +229,24 @@ def g4attn_decode(desc: LayerDesc, cache: KVCache, q_raw: torch.Tensor, q_norm_w
                              _ptr(q_norm_w, "q_norm_w", dev), _ptr(out, "out", dev),
                              _ptr(workspace, "workspace", dev), workspace.numel(), _stream(stream))
     _check(rc, "g4attn_decode")
+    return out
+
+
+def g4attn_decode_noalloc(desc: LayerDesc, cache: KVCache, q_raw: torch.Tensor,
+                          q_norm_w: torch.Tensor, out: torch.Tensor | None = None,
+                          stream=None) -> torch.Tensor:
+    """g4attn_decode without a workspace: the split-KV partials live in the
+    library's fixed 16 MiB device array (see g4attn_decode_noalloc in
+    g4attn.h).  For callers that cannot hand the library device memory per
+    call.  Calls that overlap on the GPU race on that array."""
+    cc = cache.c()
+    dev = cache.k.device
+    if out is None:
+        out = torch.empty_like(q_raw)
+    rc = lib().g4attn_decode_noalloc(ctypes.byref(desc), ctypes.byref(cc),
+                                     _ptr(q_raw, "q_raw", dev), _ptr(q_norm_w, "q_norm_w", dev),
+                                     _ptr(out, "out", dev), _stream(stream))
+    _check(rc, "g4attn_decode_noalloc")
     return out
 
 

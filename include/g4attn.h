@@ -201,6 +201,28 @@ int g4attn_decode(const g4attn_layer_desc *desc, const g4attn_cache *cache,
                   const void *q_raw, const void *q_norm_w, void *out,
                   void *workspace, size_t ws_bytes, void *stream);
 
+/* g4attn_decode without a workspace, for callers that cannot give the
+ * library device memory per call (for example a serving runtime that has
+ * handed all free device memory to its KV-cache pool, or a plugin host that
+ * exposes no allocator).  The pages have no counterpart: this is a property
+ * of the library, not of the layer.
+ *
+ * Same arguments, semantics and outputs as g4attn_decode, minus the
+ * workspace.  The split-KV partials go to a fixed 16 MiB array of device
+ * memory that the library holds on every GPU that loads it, until the process
+ * exits; this call allocates and frees nothing.  If the partials of one chunk
+ * per (sequence, query head) -- batch * num_heads * (head_dim + 2) * 4 bytes
+ * -- exceed 16 MiB the call returns G4ATTN_EWORKSPACE and enqueues nothing;
+ * when the usual number of chunks does not fit, the keys are split into fewer,
+ * longer chunks.  All calls on a device share the array: calls whose kernels
+ * may overlap on the GPU (other streams, other host threads) race on it and
+ * must be serialised by the caller.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress); make that first call before
+ * any stream capture. */
+int g4attn_decode_noalloc(const g4attn_layer_desc *desc, const g4attn_cache *cache,
+                          const void *q_raw, const void *q_norm_w, void *out,
+                          void *stream);
+
 /* Waits for `stream`, then returns and clears the device status word of the
  * current device: G4ATTN_OK, or the first error a kernel recorded since the
  * last call.  Returns G4ATTN_ECUDA if the wait or the copy fails. */
