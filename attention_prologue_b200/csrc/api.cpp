@@ -181,7 +181,9 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
   cudaEvent_t ev0, ev1;
   take_timing(&ev0, &ev1);
   if (ev0) cudaEventRecord(ev0, s);
-  e = launch_attention_simt(L, B, T, q_hat, src, rows, out, s);
+  e = attention_sm100_supported(L)
+          ? launch_attention_sm100(L, B, T, q_hat, src, rows, out, status_ptr(), s)
+          : launch_attention_simt(L, B, T, q_hat, src, rows, out, s);
   if (ev1) cudaEventRecord(ev1, s);
   return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
 }

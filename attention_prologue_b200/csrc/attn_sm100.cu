@@ -1,0 +1,436 @@
+// Prefill attention on the 5th-generation tensor cores (tcgen05, TMEM, TMA)
+// for head_dim 64 / 128 / 256: the sliding-window layers with image blocks
+// ("Gemma 4" overview blog, "Sliding-window attention"; "Gemma 4" Keras docs,
+// "What changed": bidirectional image blocks on sliding layers) and causal
+// global layers ("Global attention layers").
+//
+// One CTA computes 128 query rows of one query head:
+//   warp 0      TMA producer: Q tile once, then K/V tiles of 64 keys into a
+//               two-stage ring (128-byte swizzle, no multicast)
+//   warp 1      owns TMEM; one thread issues the MMAs:
+//                 S_j = Q K_j^T   (M 128, N 64, K = d; A, B K-major)
+//                 O  += P_j V_j   (M 128, N = d, K 64; P K-major, V MN-major)
+//   warps 4..7  softmax: thread r owns query row r (TMEM lane r); reads S_j,
+//               masks it with the row's key interval [lo, hi], writes
+//               P_j = exp2(S_j - m) as bf16 into swizzled shared memory, and
+//               at the end normalises O and stores it.
+// TMEM columns: S double buffer at 0 and 64, O at 128 (d columns).
+// Key tiles outside the union of the 128 rows' intervals are never loaded.
+//
+// The online softmax rescales O lazily: a row keeps the max it exponentiates
+// against until a new tile raises it by more than 8 (in log2 units), so P
+// stays below 2^8 and O is read and written back only on those rare tiles.
+//
+// Every mbarrier wait is bounded (sm100.cuh); on a timeout the CTA records
+// G4ATTN_EDEVICE, drains its in-flight copies and MMAs, frees TMEM and exits.
+#include <cuda.h>
+#include <mutex>
+
+#include "common.cuh"
+#include "g4attn.h"
+#include "sm100.cuh"
+
+namespace g4 {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int BM = 128;  // query rows per CTA
+constexpr int BN = 64;   // keys per tile
+constexpr int kStages = 2;
+constexpr int kThreads = 256;
+constexpr int kSoftmaxWarp0 = 4;
+
+template <int D>
+struct Layout {
+  static constexpr int kChunks = D / 64;                  // 64-element (128-byte) columns
+  static constexpr uint32_t kQChunk = BM * 128;           // bytes of one Q chunk
+  static constexpr uint32_t kKVChunk = BN * 128;          // bytes of one K or V chunk
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kK = kQ + kChunks * kQChunk;
+  static constexpr uint32_t kV = kK + kStages * kChunks * kKVChunk;
+  static constexpr uint32_t kP = kV + kStages * kChunks * kKVChunk;
+  static constexpr uint32_t kPBytes = BM * BN * 2;
+  static constexpr uint32_t kBars = kP + 2 * kPBytes;
+  static constexpr uint32_t kTotal = kBars + 256;       // barriers and scalars
+  static constexpr uint32_t kAlloc = kTotal + 1024;     // slack to align the base to 1024
+  static constexpr uint32_t kTmemCols = (128 + D) <= 256 ? 256 : 512;
+  static constexpr uint32_t kColO = 128;
+};
+
+struct Bars {  // offsets (in 8-byte words) of the mbarriers from Layout::kBars
+  enum {
+    q_full = 0,
+    kv_full = 1,   // [2]
+    kv_empty = 3,  // [2]
+    s_full = 5,    // [2]
+    p_full = 7,    // [2]
+    o_done = 9,
+    drain = 10,
+    count = 11
+  };
+};
+
+struct Scalars {  // ints after the barriers
+  uint32_t tmem_base;
+  int abort;
+  int klo, khi;
+};
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, RowIntervals rows,
+                      __nv_bfloat16* __restrict__ out, int T_, int Hq, int Hkv, int layer_type,
+                      int window, float scale_log2, int* status) {
+  using Ly = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t bars = base + Ly::kBars;
+  auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+  Scalars* sc = reinterpret_cast<Scalars*>(gbase + Ly::kBars + 8 * Bars::count);
+  volatile int* abort = &sc->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = gridDim.x - 1 - blockIdx.x;  // longest (latest) row tiles first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int r0 = tile * BM;
+  const int kvh = h / (Hq / Hkv);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(Bars::q_full), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(Bars::kv_full + s), 1);
+      mbar_init(bar(Bars::kv_empty + s), 1);
+      mbar_init(bar(Bars::s_full + s), 1);
+      mbar_init(bar(Bars::p_full + s), 4 * 32);
+    }
+    mbar_init(bar(Bars::o_done), 1);
+    mbar_init(bar(Bars::drain), 1);
+    sc->abort = 0;
+    sc->klo = 0x7fffffff;
+    sc->khi = -1;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  if (warp == 1) {
+    tmem_alloc(base + Ly::kBars + 8 * Bars::count, Ly::kTmemCols);
+    tmem_relinquish();
+  }
+  // row intervals of the softmax threads, reduced to the CTA's key range
+  int lo = 1, hi = 0;
+  const int r = threadIdx.x - kSoftmaxWarp0 * 32;  // row of a softmax thread
+  __syncthreads();
+  if (warp >= kSoftmaxWarp0) {
+    const int i = r0 + r;
+    if (i < T_) {
+      if (rows.lo) {
+        lo = rows.lo[(long)b * T_ + i];
+        hi = rows.hi[(long)b * T_ + i];
+      } else if (layer_type == 1) {
+        lo = 0;
+        hi = i;
+      } else {
+        lo = max(0, i - window + 1);
+        hi = i;
+      }
+      atomicMin(&sc->klo, lo);
+      atomicMax(&sc->khi, hi);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sc->tmem_base;
+  const int kt0 = sc->klo / BN;
+  const int n_tiles = sc->khi / BN - kt0 + 1;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(Bars::q_full), BM * D * 2);
+      for (int c = 0; c < Ly::kChunks; ++c)
+        tma_load_4d(base + Ly::kQ + c * Ly::kQChunk, &tm_q, bar(Bars::q_full), c * 64, h, r0, b);
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % kStages;
+        if (!mbar_wait(bar(Bars::kv_empty + s), ((j / kStages) & 1) ^ 1, abort)) break;
+        const int key0 = (kt0 + j) * BN;
+        mbar_arrive_expect_tx(bar(Bars::kv_full + s), 2 * BN * D * 2);
+        for (int c = 0; c < Ly::kChunks; ++c) {
+          const uint32_t off = (s * Ly::kChunks + c) * Ly::kKVChunk;
+          tma_load_3d(base + Ly::kK + off, &tm_k, bar(Bars::kv_full + s), c * 64, key0,
+                      b * Hkv + kvh);
+          tma_load_3d(base + Ly::kV + off, &tm_v, bar(Bars::kv_full + s), c * 64, key0,
+                      b * Hkv + kvh);
+        }
+        issued = j + 1;
+      }
+      if (*abort) {  // let the copies already issued land before the CTA exits
+        mbar_wait(bar(Bars::q_full), 0, nullptr);
+        for (int j = max(0, issued - kStages); j < issued; ++j)
+          mbar_wait(bar(Bars::kv_full + j % kStages), (j / kStages) & 1, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(BM, BN, 0, 0);
+      constexpr uint32_t idesc_o = idesc_bf16(BM, D, 0, 1);
+      auto issue_pv = [&](int j) {
+        const int s = j % kStages;
+        const uint32_t pbase = base + Ly::kP + (j & 1) * Ly::kPBytes;
+        const uint32_t vbase = base + Ly::kV + s * Ly::kChunks * Ly::kKVChunk;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t a = desc_sw128(pbase + kk * 32, 16, 1024);
+          const uint64_t bd = desc_sw128(vbase + kk * 16 * 128, Ly::kKVChunk, 1024);
+          mma_ss(tmem + Ly::kColO, a, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(bar(Bars::kv_empty + s));
+        mma_commit(bar(Bars::o_done));
+      };
+      bool ok = mbar_wait(bar(Bars::q_full), 0, abort);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kStages;
+        if (!(ok = mbar_wait(bar(Bars::kv_full + s), (j / kStages) & 1, abort))) break;
+        tc_fence_after();
+        const uint32_t kbase = base + Ly::kK + s * Ly::kChunks * Ly::kKVChunk;
+#pragma unroll
+        for (int kc = 0; kc < D / 16; ++kc) {
+          const int c = kc >> 2, sub = kc & 3;
+          const uint64_t a = desc_sw128(base + Ly::kQ + c * Ly::kQChunk + sub * 32, 16, 1024);
+          const uint64_t bd = desc_sw128(kbase + c * Ly::kKVChunk + sub * 32, 16, 1024);
+          mma_ss(tmem + (j & 1) * BN, a, bd, idesc_s, kc > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(Bars::s_full + (j & 1)));
+        if (j >= 1) {
+          if (!(ok = mbar_wait(bar(Bars::p_full + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort)))
+            break;
+          tc_fence_after();
+          issue_pv(j - 1);
+        }
+      }
+      if (ok && mbar_wait(bar(Bars::p_full + ((n_tiles - 1) & 1)), ((n_tiles - 1) >> 1) & 1,
+                          abort)) {
+        tc_fence_after();
+        issue_pv(n_tiles - 1);
+      }
+      if (*abort) {  // every MMA issued so far completes before TMEM is freed
+        mma_commit(bar(Bars::drain));
+        mbar_wait(bar(Bars::drain), 0, nullptr);
+      }
+    }
+  } else if (warp >= kSoftmaxWarp0) {
+    // ------------------------------------------------------------ softmax
+    const uint32_t lane_off = (uint32_t)((warp - kSoftmaxWarp0) * 32) << 16;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::s_full + (j & 1)), (j >> 1) & 1, abort));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[BN];
+      tmem_ld32(tmem + lane_off + (j & 1) * BN, sr);
+      tmem_ld32(tmem + lane_off + (j & 1) * BN + 32, sr + 32);
+      tmem_wait_ld();
+      const int key0 = (kt0 + j) * BN;
+      float x[BN];
+      float mt = -INFINITY;
+      const bool full = key0 >= lo && key0 + BN - 1 <= hi;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) {
+        float v = __uint_as_float(sr[c]) * scale_log2;
+        if (!full) v = (key0 + c >= lo && key0 + c <= hi) ? v : -INFINITY;
+        x[c] = v;
+        mt = fmaxf(mt, v);
+      }
+      // lazy rescale: only when the row max grows by more than 2^8
+      const bool first = m_used == -INFINITY;
+      const bool grow = !first && mt > m_used + 8.f;
+      if (__any_sync(0xffffffffu, grow)) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::o_done), (j - 1) & 1, abort));
+        if (!ok) break;
+        tc_fence_after();
+        const float alpha = grow ? exp2f(m_used - mt) : 1.f;
+        if (grow) {
+          l *= alpha;
+          m_used = mt;
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + Ly::kColO + c0, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st32(tmem + lane_off + Ly::kColO + c0, o);
+        }
+        tmem_wait_st();
+      }
+      if (first && mt != -INFINITY) m_used = mt;
+      // P = exp2(x - m_used) as bf16, written in the 128-byte-swizzled
+      // K-major layout: 16-byte chunk q of row r goes to chunk q ^ (r & 7)
+      const uint32_t prow = base + Ly::kP + (j & 1) * Ly::kPBytes + r * 128;
+      float rs = 0.f;
+#pragma unroll
+      for (int q = 0; q < BN / 8; ++q) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float p0 = m_used == -INFINITY ? 0.f : exp2f(x[8 * q + 2 * e] - m_used);
+          const float p1 = m_used == -INFINITY ? 0.f : exp2f(x[8 * q + 2 * e + 1] - m_used);
+          rs += p0 + p1;
+          __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
+          pk[e] = *reinterpret_cast<uint32_t*>(&bb);
+        }
+        const uint32_t dst = prow + ((q ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[0]),
+                     "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                     : "memory");
+      }
+      l += rs;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(Bars::p_full + (j & 1)));
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok)  // warp-uniform: the tcgen05 loads below are warp-collective
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::o_done), (n_tiles - 1) & 1, abort));
+    if (ok) {
+      tc_fence_after();
+      const int i = r0 + r;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = out + (((long)b * T_ + i) * Hq + h) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(tmem + lane_off + Ly::kColO + c0, o);
+        tmem_wait_ld();
+        if (i < T_) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            __nv_bfloat162 bb = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
+                                                      __uint_as_float(o[2 * e + 1]) * inv);
+            pk[e] = *reinterpret_cast<uint32_t*>(&bb);
+          }
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort) record_status(status, G4ATTN_EDEVICE);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Ly::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map with a 128-byte-swizzled box; dims[0] is the contiguous one.
+bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), gd, gs, bx, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
+                      RowIntervals rows, void* out, int* status, cudaStream_t s) {
+  CUtensorMap tq, tk, tv;
+  const uint64_t es = 2;
+  {  // q_hat [B, T, Hq, D]: dims (D, Hq, T, B)
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)L.Hq, (uint64_t)T, (uint64_t)B};
+    const uint64_t str[3] = {D * es, (uint64_t)L.Hq * D * es, (uint64_t)T * L.Hq * D * es};
+    const uint32_t box[4] = {64, 1, BM, 1};
+    if (!make_map(&tq, q_hat, 4, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {  // K, V [B * Hkv, cap, D]; only positions < T exist (rows past T read as 0)
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)T, (uint64_t)B * L.Hkv};
+    const uint64_t str[2] = {D * es, (uint64_t)kv.cap * D * es};
+    const uint32_t box[3] = {64, BN, 1};
+    if (!make_map(&tk, kv.k, 3, dims, str, box)) return cudaErrorInvalidValue;
+    if (!make_map(&tv, kv.v, 3, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  using Ly = Layout<D>;
+  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
+  if (e != cudaSuccess) return e;
+  const float scale_log2 = L.scale * 1.4426950408889634f;
+  dim3 grid((T + BM - 1) / BM, L.Hq, B);
+  attn_sm100_kernel<D><<<grid, kThreads, Ly::kAlloc, s>>>(
+      tq, tk, tv, rows, static_cast<__nv_bfloat16*>(out), T, L.Hq, L.Hkv, L.layer_type, L.window,
+      scale_log2, status);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attention_sm100_supported(const LayerCfg& L) {
+  return L.dtype == 0 && (L.d == 64 || L.d == 128 || L.d == 256);
+}
+
+cudaError_t launch_attention_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
+                                   RowIntervals rows, void* out, int* status, cudaStream_t s) {
+  switch (L.d) {
+    case 64: return run_sm100<64>(L, B, T, q_hat, kv, rows, out, status, s);
+    case 128: return run_sm100<128>(L, B, T, q_hat, kv, rows, out, status, s);
+    case 256: return run_sm100<256>(L, B, T, q_hat, kv, rows, out, status, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace g4

@@ -52,7 +52,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait for the phase of parity `parity` to complete.  Gives up after
 // `limit_ns` of wall time (or as soon as *abort is set by another thread of
 // the CTA), sets *abort and returns false: no wait in these kernels can spin
-// forever.
+// forever.  abort == nullptr: only the time limit applies (used to drain
+// in-flight work on the abort path).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns = 2000000000ull) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -60,9 +61,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 63) {
-      if (*abort) return false;
+      if (abort && *abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
-        *abort = 1;
+        if (abort) *abort = 1;
         return false;
       }
     }
