@@ -46,7 +46,7 @@ static int make_cfg(const g4attn_layer_desc* d, LayerCfg* L) {
   const long R2 = std::lround(rd);
   if (std::fabs(rd - (double)R2) > 1e-6 || (R2 & 1)) return G4ATTN_EINVAL;
   if (!(d->rope_theta > 0.0) || !std::isfinite(d->rope_theta)) return G4ATTN_EINVAL;
-  if (!std::isfinite(d->softmax_scale)) return G4ATTN_EINVAL;
+  if (!(d->softmax_scale > 0.f) || !std::isfinite(d->softmax_scale)) return G4ATTN_EINVAL;
   if (!(d->rms_eps >= 0.f) || !std::isfinite(d->rms_eps)) return G4ATTN_EINVAL;
   if (d->k_eq_v != 0 && d->k_eq_v != 1) return G4ATTN_EINVAL;
   L->layer_type = d->layer_type;
@@ -158,15 +158,16 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
     src = {kbuf, vbuf, T};
   }
   cudaError_t e = cudaSuccess;
+  KVDst d0{nullptr, nullptr, 1, 0, 0}, d1{nullptr, nullptr, 1, 0, 0};
   if (!shared) {
-    KVDst d0{const_cast<void*>(src.k), const_cast<void*>(src.v), src.cap, 0, 0};
-    KVDst d1{nullptr, nullptr, 1, 0, 0};
+    d0 = {const_cast<void*>(src.k), const_cast<void*>(src.v), src.cap, 0, 0};
     if (cache && !cache_is_src)  // rolling cache smaller than the prompt: last `cap` positions
       d1 = {cache->k, cache->v, cache->capacity, 1, T - cache->capacity};
-    e = launch_kv_prologue(L, B, T, k_raw, v_raw, k_norm_w, d0, d1, cache ? cache->len : nullptr,
-                           s);
-    if (e != cudaSuccess) return G4ATTN_ECUDA;
   }
+  void* q_hat = ws + w.q_hat;
+  e = launch_token_prologue(L, B, T, q_raw, q_norm_w, q_hat, shared ? nullptr : k_raw, v_raw,
+                            k_norm_w, d0, d1, (cache && !shared) ? cache->len : nullptr, s);
+  if (e != cudaSuccess) return G4ATTN_ECUDA;
   RowIntervals rows{nullptr, nullptr};
   if (intervals) {
     int32_t* lo = reinterpret_cast<int32_t*>(ws + w.intervals);
@@ -176,8 +177,6 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
       return G4ATTN_ECUDA;
     rows = {lo, hi};
   }
-  void* q_hat = ws + w.q_hat;
-  if (launch_q_prologue(L, B, T, q_raw, q_norm_w, q_hat, s) != cudaSuccess) return G4ATTN_ECUDA;
   cudaEvent_t ev0, ev1;
   take_timing(&ev0, &ev1);
   if (ev0) cudaEventRecord(ev0, s);

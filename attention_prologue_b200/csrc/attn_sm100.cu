@@ -5,8 +5,10 @@
 // global layers ("Global attention layers").
 //
 // One CTA computes 128 query rows of one query head:
-//   warp 0      TMA producer: Q tile once, then K/V tiles of 64 keys into a
-//               two-stage ring (128-byte swizzle, no multicast)
+//   warps 0, 2  TMA producers: Q tile once and K tiles (warp 0), V tiles
+//               (warp 2), 64 keys each, two-stage rings (128-byte swizzle,
+//               no multicast); a K slot is refilled as soon as S_j is done,
+//               a V slot as soon as PV_j is done
 //   warp 1      owns TMEM; one thread issues the MMAs:
 //                 S_j = Q K_j^T   (M 128, N 64, K = d; A, B K-major)
 //                 O  += P_j V_j   (M 128, N = d, K 64; P K-major, V MN-major)
@@ -62,13 +64,15 @@ struct Layout {
 struct Bars {  // offsets (in 8-byte words) of the mbarriers from Layout::kBars
   enum {
     q_full = 0,
-    kv_full = 1,   // [2]
-    kv_empty = 3,  // [2]
-    s_full = 5,    // [2]
-    p_full = 7,    // [2]
-    o_done = 9,
-    drain = 10,
-    count = 11
+    k_full = 1,    // [2]
+    k_empty = 3,   // [2]
+    v_full = 5,    // [2]
+    v_empty = 7,   // [2]
+    s_full = 9,    // [2]
+    p_full = 11,   // [2]
+    o_done = 13,
+    drain = 14,
+    count = 15
   };
 };
 
@@ -106,8 +110,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(Bars::q_full), 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(Bars::kv_full + s), 1);
-      mbar_init(bar(Bars::kv_empty + s), 1);
+      mbar_init(bar(Bars::k_full + s), 1);
+      mbar_init(bar(Bars::k_empty + s), 1);
+      mbar_init(bar(Bars::v_full + s), 1);
+      mbar_init(bar(Bars::v_empty + s), 1);
       mbar_init(bar(Bars::s_full + s), 1);
       mbar_init(bar(Bars::p_full + s), 4 * 32);
     }
@@ -155,31 +161,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kt0 = sc->klo / BN;
   const int n_tiles = sc->khi / BN - kt0 + 1;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ producers
+    // warp 0 loads Q and the K tiles, warp 2 the V tiles: each ring is
+    // refilled as soon as its own consumer (S_j for K, PV_j for V) is done.
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(Bars::q_full), BM * D * 2);
-      for (int c = 0; c < Ly::kChunks; ++c)
-        tma_load_4d(base + Ly::kQ + c * Ly::kQChunk, &tm_q, bar(Bars::q_full), c * 64, h, r0, b);
+      const bool is_k = warp == 0;
+      const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+      const uint32_t ring = base + (is_k ? Ly::kK : Ly::kV);
+      const int full = is_k ? Bars::k_full : Bars::v_full;
+      const int empty = is_k ? Bars::k_empty : Bars::v_empty;
+      if (is_k) {
+        mbar_arrive_expect_tx(bar(Bars::q_full), BM * D * 2);
+        for (int c = 0; c < Ly::kChunks; ++c)
+          tma_load_4d(base + Ly::kQ + c * Ly::kQChunk, &tm_q, bar(Bars::q_full), c * 64, h, r0,
+                      b);
+      }
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % kStages;
-        if (!mbar_wait(bar(Bars::kv_empty + s), ((j / kStages) & 1) ^ 1, abort)) break;
+        if (!mbar_wait(bar(empty + s), ((j / kStages) & 1) ^ 1, abort)) break;
         const int key0 = (kt0 + j) * BN;
-        mbar_arrive_expect_tx(bar(Bars::kv_full + s), 2 * BN * D * 2);
-        for (int c = 0; c < Ly::kChunks; ++c) {
-          const uint32_t off = (s * Ly::kChunks + c) * Ly::kKVChunk;
-          tma_load_3d(base + Ly::kK + off, &tm_k, bar(Bars::kv_full + s), c * 64, key0,
-                      b * Hkv + kvh);
-          tma_load_3d(base + Ly::kV + off, &tm_v, bar(Bars::kv_full + s), c * 64, key0,
-                      b * Hkv + kvh);
-        }
+        mbar_arrive_expect_tx(bar(full + s), BN * D * 2);
+        for (int c = 0; c < Ly::kChunks; ++c)
+          tma_load_3d(ring + (s * Ly::kChunks + c) * Ly::kKVChunk, tm, bar(full + s), c * 64,
+                      key0, b * Hkv + kvh);
         issued = j + 1;
       }
       if (*abort) {  // let the copies already issued land before the CTA exits
-        mbar_wait(bar(Bars::q_full), 0, nullptr);
+        if (is_k) mbar_wait(bar(Bars::q_full), 0, nullptr);
         for (int j = max(0, issued - kStages); j < issued; ++j)
-          mbar_wait(bar(Bars::kv_full + j % kStages), (j / kStages) & 1, nullptr);
+          mbar_wait(bar(full + j % kStages), (j / kStages) & 1, nullptr);
       }
     }
   } else if (warp == 1) {
@@ -197,13 +209,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = desc_sw128(vbase + kk * 16 * 128, Ly::kKVChunk, 1024);
           mma_ss(tmem + Ly::kColO, a, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(bar(Bars::kv_empty + s));
+        mma_commit(bar(Bars::v_empty + s));
         mma_commit(bar(Bars::o_done));
       };
       bool ok = mbar_wait(bar(Bars::q_full), 0, abort);
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kStages;
-        if (!(ok = mbar_wait(bar(Bars::kv_full + s), (j / kStages) & 1, abort))) break;
+        if (!(ok = mbar_wait(bar(Bars::k_full + s), (j / kStages) & 1, abort))) break;
         tc_fence_after();
         const uint32_t kbase = base + Ly::kK + s * Ly::kChunks * Ly::kKVChunk;
 #pragma unroll
@@ -214,15 +226,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + (j & 1) * BN, a, bd, idesc_s, kc > 0 ? 1u : 0u);
         }
         mma_commit(bar(Bars::s_full + (j & 1)));
+        mma_commit(bar(Bars::k_empty + s));
         if (j >= 1) {
           if (!(ok = mbar_wait(bar(Bars::p_full + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort)))
+            break;
+          if (!(ok = mbar_wait(bar(Bars::v_full + (j - 1) % kStages), ((j - 1) / kStages) & 1,
+                               abort)))
             break;
           tc_fence_after();
           issue_pv(j - 1);
         }
       }
       if (ok && mbar_wait(bar(Bars::p_full + ((n_tiles - 1) & 1)), ((n_tiles - 1) >> 1) & 1,
-                          abort)) {
+                          abort) &&
+          mbar_wait(bar(Bars::v_full + (n_tiles - 1) % kStages), ((n_tiles - 1) / kStages) & 1,
+                    abort)) {
         tc_fence_after();
         issue_pv(n_tiles - 1);
       }
@@ -247,14 +265,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int key0 = (kt0 + j) * BN;
       float x[BN];
       float mt = -INFINITY;
-      const bool full = key0 >= lo && key0 + BN - 1 <= hi;
+      if (key0 >= lo && key0 + BN - 1 <= hi) {  // interior tile: no mask
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        float v = __uint_as_float(sr[c]) * scale_log2;
-        if (!full) v = (key0 + c >= lo && key0 + c <= hi) ? v : -INFINITY;
-        x[c] = v;
-        mt = fmaxf(mt, v);
+        for (int c = 0; c < BN; ++c) {
+          x[c] = __uint_as_float(sr[c]);
+          mt = fmaxf(mt, x[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          x[c] = (key0 + c >= lo && key0 + c <= hi) ? __uint_as_float(sr[c]) : -INFINITY;
+          mt = fmaxf(mt, x[c]);
+        }
       }
+      mt *= scale_log2;  // scale > 0: the max of the scaled scores
       // lazy rescale: only when the row max grows by more than 2^8
       const bool first = m_used == -INFINITY;
       const bool grow = !first && mt > m_used + 8.f;
@@ -282,14 +306,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P = exp2(x - m_used) as bf16, written in the 128-byte-swizzled
       // K-major layout: 16-byte chunk q of row r goes to chunk q ^ (r & 7)
       const uint32_t prow = base + Ly::kP + (j & 1) * Ly::kPBytes + r * 128;
+      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;  // row with no key yet: P = 0
       float rs = 0.f;
 #pragma unroll
       for (int q = 0; q < BN / 8; ++q) {
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float p0 = m_used == -INFINITY ? 0.f : exp2f(x[8 * q + 2 * e] - m_used);
-          const float p1 = m_used == -INFINITY ? 0.f : exp2f(x[8 * q + 2 * e + 1] - m_used);
+          const float p0 = ex2_approx(fmaf(x[8 * q + 2 * e], scale_log2, neg_m));
+          const float p1 = ex2_approx(fmaf(x[8 * q + 2 * e + 1], scale_log2, neg_m));
           rs += p0 + p1;
           __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
           pk[e] = *reinterpret_cast<uint32_t*>(&bb);

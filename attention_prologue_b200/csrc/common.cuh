@@ -167,6 +167,63 @@ __device__ __forceinline__ void prologue_vec(const T* __restrict__ src, const T*
   }
 }
 
+// RoPE factors of one token for the pairs a lane holds (k = lane*E + e,
+// E = D/64): rot[e] = 0 marks a pass-through pair.
+template <int D>
+__device__ __forceinline__ void rope_factors(long pos, const RopeParams& rope, float* c, float* s,
+                                             bool* rot) {
+  constexpr int E = D / 64;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int k = lane * E + e;
+    rot[e] = k < rope.rotated_pairs;
+    c[e] = 1.f;
+    s[e] = 0.f;
+    if (rot[e]) rope_sincos(pos, rope.inv_freq[k], &s[e], &c[e]);
+  }
+}
+
+// RMSNorm (x * rsqrt(mean(x^2) + eps) * w) and optional RoPE of NH head
+// vectors of one token already loaded into registers (x0/x1: the two halves,
+// E = D/64 values per lane each), in place.  w0/w1 == nullptr: no weight.
+template <int D, int NH>
+__device__ __forceinline__ void norm_rope(float (*x0)[D / 64], float (*x1)[D / 64], const float* w0,
+                                          const float* w1, const float* c, const float* s,
+                                          const bool* rot, bool rope, float eps) {
+  constexpr int E = D / 64;
+  float ss[NH];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    ss[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) ss[h] += x0[h][e] * x0[h][e] + x1[h][e] * x1[h][e];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int h = 0; h < NH; ++h) ss[h] += __shfl_xor_sync(0xffffffffu, ss[h], o);
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    const float r = rsqrtf(ss[h] / (float)D + eps);
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      float a = x0[h][e] * r, b = x1[h][e] * r;
+      if (w0) {
+        a *= w0[e];
+        b *= w1[e];
+      }
+      if (rope && rot[e]) {
+        const float a2 = a * c[e] - b * s[e];
+        b = a * s[e] + b * c[e];
+        a = a2;
+      }
+      x0[h][e] = a;
+      x1[h][e] = b;
+    }
+  }
+}
+
 template <typename T, int D>
 __device__ __forceinline__ void store_vec(T* __restrict__ dst, const float* y0, const float* y1) {
   constexpr int E = D / 64;

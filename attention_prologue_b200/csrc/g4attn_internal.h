@@ -51,11 +51,12 @@ struct RowIntervals {
   const int32_t* hi;
 };
 
-cudaError_t launch_q_prologue(const LayerCfg& L, int B, int T, const void* q_raw, const void* wq,
-                              void* q_hat, cudaStream_t s);
-cudaError_t launch_kv_prologue(const LayerCfg& L, int B, int T, const void* k_raw,
-                               const void* v_raw, const void* wk, KVDst d0, KVDst d1,
-                               int32_t* len_out, cudaStream_t s);
+// Q, K and V prologue of a prompt in one launch (one warp per token);
+// k_raw == nullptr: queries only (KV-shared layer).
+cudaError_t launch_token_prologue(const LayerCfg& L, int B, int T, const void* q_raw,
+                                  const void* wq, void* q_hat, const void* k_raw,
+                                  const void* v_raw, const void* wk, KVDst d0, KVDst d1,
+                                  int32_t* len_out, cudaStream_t s);
 cudaError_t launch_block_intervals(const LayerCfg& L, int B, int T, const int32_t* ids,
                                    int32_t* lo, int32_t* hi, cudaStream_t s);
 cudaError_t launch_attention_simt(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,

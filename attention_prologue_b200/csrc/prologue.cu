@@ -4,8 +4,9 @@
 // the per-row interval pre-pass of image blocks, and the cache append
 // ("gemma4-pt-claude" README, "KV Cache").
 //
-// Memory-bound: one warp per head vector, 16-byte accesses where the head
-// size allows, fp32 arithmetic, fp64 RoPE angle reduction.
+// Memory-bound: one warp per token (prompt) or per KV head (append), 16-byte
+// accesses where the head size allows, fp32 arithmetic, fp64 RoPE angle
+// reduction computed once per token and shared by all of its heads.
 #include <mutex>
 
 #include "common.cuh"
@@ -32,19 +33,6 @@ int* status_ptr() {
 constexpr int kWarps = 8;  // warps per block of the per-vector kernels
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kWarps * 32)
-    q_prologue_kernel(const T* __restrict__ q_raw, const T* __restrict__ wq, T* __restrict__ q_hat,
-                      long n_vec, int T_, int Hq, const __grid_constant__ RopeParams rope,
-                      float eps) {
-  const long v = (long)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  if (v >= n_vec) return;
-  const long t = (v / Hq) % T_;
-  float y0[D / 64], y1[D / 64];
-  prologue_vec<T, D>(q_raw + v * D, wq, t, &rope, eps, y0, y1);
-  store_vec<T, D>(q_hat + v * D, y0, y1);
-}
-
-template <typename T, int D>
 __device__ __forceinline__ void put_kv(const KVDst& d, int Hkv, long b, int h, long t,
                                        const float* k0, const float* k1, const float* v0,
                                        const float* v1) {
@@ -55,25 +43,60 @@ __device__ __forceinline__ void put_kv(const KVDst& d, int Hkv, long b, int h, l
   store_vec<T, D>(static_cast<T*>(d.v) + off, v0, v1);
 }
 
+// Prologue of a whole prompt, one warp per token: the RoPE factors of the
+// token (position t) are computed once and applied to its Hq query heads and
+// Hkv key heads; the value heads are normalised without weight or rotation
+// (from the key projection with K=V).  Heads are processed NB at a time with
+// all their loads issued first.  k_raw == nullptr: queries only.
 template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32)
-    kv_prologue_kernel(const T* __restrict__ k_raw, const T* __restrict__ v_raw,
-                       const T* __restrict__ wk, int B, int T_, int Hkv, KVDst d0, KVDst d1,
-                       int32_t* __restrict__ len_out, const __grid_constant__ RopeParams rope,
-                       float eps) {
-  const long v = (long)blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const long n_vec = (long)B * T_ * Hkv;
-  if (v >= n_vec) return;
-  const int h = (int)(v % Hkv);
-  const long t = (v / Hkv) % T_;
-  const long b = v / ((long)Hkv * T_);
-  float k0[D / 64], k1[D / 64], u0[D / 64], u1[D / 64];
-  prologue_vec<T, D>(k_raw + v * D, wk, t, &rope, eps, k0, k1);
-  // V-norm: no weight, no rotation; with K=V it reads the key projection
-  prologue_vec<T, D>((v_raw ? v_raw : k_raw) + v * D, nullptr, t, nullptr, eps, u0, u1);
-  put_kv<T, D>(d0, Hkv, b, h, t, k0, k1, u0, u1);
-  put_kv<T, D>(d1, Hkv, b, h, t, k0, k1, u0, u1);
-  if (len_out && t == 0 && h == 0 && (threadIdx.x & 31) == 0) len_out[b] = T_;
+    token_prologue_kernel(const T* __restrict__ q_raw, const T* __restrict__ wq,
+                          T* __restrict__ q_hat, const T* __restrict__ k_raw,
+                          const T* __restrict__ v_raw, const T* __restrict__ wk, int B, int T_,
+                          int Hq, int Hkv, KVDst d0, KVDst d1, int32_t* __restrict__ len_out,
+                          const __grid_constant__ RopeParams rope, float eps) {
+  constexpr int E = D / 64, NB = 4;
+  const long tok = (long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (tok >= (long)B * T_) return;
+  const int lane = threadIdx.x & 31;
+  const long t = tok % T_, b = tok / T_;
+  float c[E], s[E];
+  bool rot[E];
+  rope_factors<D>(t, rope, c, s, rot);
+  float w0[E], w1[E];
+  Vec<T, E>::load(wq + lane * E, w0);
+  Vec<T, E>::load(wq + D / 2 + lane * E, w1);
+  for (int h0 = 0; h0 < Hq; h0 += NB) {
+    float x0[NB][E], x1[NB][E];
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      const int h = min(h0 + j, Hq - 1);  // tail: recompute the last head, store once
+      const T* src = q_raw + (tok * Hq + h) * D;
+      Vec<T, E>::load(src + lane * E, x0[j]);
+      Vec<T, E>::load(src + D / 2 + lane * E, x1[j]);
+    }
+    norm_rope<D, NB>(x0, x1, w0, w1, c, s, rot, true, eps);
+#pragma unroll
+    for (int j = 0; j < NB; ++j)
+      if (h0 + j < Hq) store_vec<T, D>(q_hat + (tok * Hq + h0 + j) * D, x0[j], x1[j]);
+  }
+  if (!k_raw) return;
+  Vec<T, E>::load(wk + lane * E, w0);
+  Vec<T, E>::load(wk + D / 2 + lane * E, w1);
+  const T* vsrc = v_raw ? v_raw : k_raw;
+  for (int h = 0; h < Hkv; ++h) {
+    float x0[2][E], x1[2][E];
+    const long off = (tok * Hkv + h) * D;
+    Vec<T, E>::load(k_raw + off + lane * E, x0[0]);
+    Vec<T, E>::load(k_raw + off + D / 2 + lane * E, x1[0]);
+    Vec<T, E>::load(vsrc + off + lane * E, x0[1]);
+    Vec<T, E>::load(vsrc + off + D / 2 + lane * E, x1[1]);
+    norm_rope<D, 1>(x0, x1, w0, w1, c, s, rot, true, eps);
+    norm_rope<D, 1>(x0 + 1, x1 + 1, nullptr, nullptr, c, s, rot, false, eps);
+    put_kv<T, D>(d0, Hkv, b, h, t, x0[0], x1[0], x0[1], x1[1]);
+    put_kv<T, D>(d1, Hkv, b, h, t, x0[0], x1[0], x0[1], x1[1]);
+  }
+  if (len_out && t == 0 && lane == 0) len_out[b] = T_;
 }
 
 // lo/hi of every row of a sliding layer with image blocks: the window
@@ -139,28 +162,17 @@ static cudaError_t dispatch(const LayerCfg& L, F&& f) {
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_q_prologue(const LayerCfg& L, int B, int T, const void* q_raw, const void* wq,
-                              void* q_hat, cudaStream_t s) {
-  const long n_vec = (long)B * T * L.Hq;
-  const unsigned grid = (unsigned)((n_vec + kWarps - 1) / kWarps);
+cudaError_t launch_token_prologue(const LayerCfg& L, int B, int T, const void* q_raw,
+                                  const void* wq, void* q_hat, const void* k_raw,
+                                  const void* v_raw, const void* wk, KVDst d0, KVDst d1,
+                                  int32_t* len_out, cudaStream_t s) {
+  const long n_tok = (long)B * T;
+  const unsigned grid = (unsigned)((n_tok + kWarps - 1) / kWarps);
   return dispatch(L, [&]<typename E, int D>() {
-    q_prologue_kernel<E, D><<<grid, kWarps * 32, 0, s>>>(
-        static_cast<const E*>(q_raw), static_cast<const E*>(wq), static_cast<E*>(q_hat), n_vec, T,
-        L.Hq, L.rope, L.eps);
-    count_launch();
-    return cudaGetLastError();
-  });
-}
-
-cudaError_t launch_kv_prologue(const LayerCfg& L, int B, int T, const void* k_raw,
-                               const void* v_raw, const void* wk, KVDst d0, KVDst d1,
-                               int32_t* len_out, cudaStream_t s) {
-  const long n_vec = (long)B * T * L.Hkv;
-  const unsigned grid = (unsigned)((n_vec + kWarps - 1) / kWarps);
-  return dispatch(L, [&]<typename E, int D>() {
-    kv_prologue_kernel<E, D><<<grid, kWarps * 32, 0, s>>>(
+    token_prologue_kernel<E, D><<<grid, kWarps * 32, 0, s>>>(
+        static_cast<const E*>(q_raw), static_cast<const E*>(wq), static_cast<E*>(q_hat),
         static_cast<const E*>(k_raw), static_cast<const E*>(v_raw), static_cast<const E*>(wk), B,
-        T, L.Hkv, d0, d1, len_out, L.rope, L.eps);
+        T, L.Hq, L.Hkv, d0, d1, len_out, L.rope, L.eps);
     count_launch();
     return cudaGetLastError();
   });

@@ -177,6 +177,14 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 2^x with the hardware approximation (MUFU.EX2; subnormal results flush to
+// zero, 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------- descriptors
 
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: version 1

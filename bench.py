@@ -1,7 +1,8 @@
 """Benchmark of the Gemma 4 attention layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--no-decode] [--no-cpu-baseline]
+                    [--workload NAME] [--no-decode] [--decode-only] [--decode-batch B]
+                    [--no-e2e] [--no-cpu-baseline]
 
 Headline: prefill attention TFLOP/s counting unmasked FLOPs only
 (4 * d * sum_i |I_i| * Hq * B; 2d for QK^T and 2d for PV per allowed pair) on
@@ -214,7 +215,7 @@ def made_events(n):
 # prefill
 
 def bench_prefill(args, dist: Dist, pk: dict):
-    w = W.E2B_SLIDING
+    w = W.PREFILL_WORKLOADS[args.workload]
     dev = torch.device("cuda", dist.local)
     inp = W.prefill_inputs(w, dev, seed=dist.rank)
     d = desc_of(w.layer)
@@ -258,6 +259,17 @@ def bench_prefill(args, dist: Dist, pk: dict):
     if status != G.G4ATTN_OK:
         raise RuntimeError(f"device status after prefill: {G.g4attn_status_string(status)}")
 
+    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    res = dict(
+        value=value, ms_per_step=total_ms / K, flops=flops, launches=launches,
+        clocks=clk.summary(),
+        roofline={"bound": "tensor", "kernel": "attention (g4attn_prefill)", "achieved": achieved,
+                  "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                  "algorithmic_per_launch": flops, "avg_launch_ms": attn_avg},
+        e2e=None, inputs=inp, workload=w)
+    if args.no_e2e:
+        return res
+
     # end to end: host (pinned) inputs -> device, prefill, output -> host
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in inp.items()}
     host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -287,17 +299,8 @@ def bench_prefill(args, dist: Dist, pk: dict):
     torch.cuda.synchronize()
     e2e_ms = dist.max(sum(e0[i].elapsed_time(e1[i]) for i in range(K)))
     e2e_value = dist.world * flops * K / (e2e_ms * 1e-3) / 1e12
-
-    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    res = dict(
-        value=value, ms_per_step=total_ms / K, flops=flops, launches=launches,
-        clocks=clk.summary(),
-        roofline={"bound": "tensor", "kernel": "attention (g4attn_prefill)", "achieved": achieved,
-                  "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                  "algorithmic_per_launch": flops, "avg_launch_ms": attn_avg},
-        e2e={"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-             "d2h_bytes_per_step": d2h},
-        inputs=inp, workload=w)
+    res["e2e"] = {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                  "d2h_bytes_per_step": d2h}
     del flush, ws
     return res
 
@@ -306,13 +309,13 @@ def bench_prefill(args, dist: Dist, pk: dict):
 # decode
 
 def bench_decode(args, dist: Dist, pk: dict):
-    w = W.A4B_DECODE
+    from dataclasses import replace
+    w = W.A4B_DECODE if not args.decode_batch else replace(W.A4B_DECODE, batch=args.decode_batch)
     dev = torch.device("cuda", dist.local)
     lens = W.decode_lengths(w, seed=dist.rank)
     g = torch.Generator(device=dev)
     g.manual_seed(1000 + dist.rank)
     S, Gl = w.sliding, w.global_
-    from dataclasses import replace
     X = replace(Gl, softmax_scale=Gl.scale)  # KV-shared layer: own queries, G's cache
     s_tok = W.decode_token_inputs(S, w.batch, g, dev, w.dtype)
     g_tok = W.decode_token_inputs(Gl, w.batch, g, dev, w.dtype)
@@ -371,7 +374,7 @@ def bench_decode(args, dist: Dist, pk: dict):
     achieved = g_split_bytes / (g_ms * 1e-3) / 1e9
     res = {"metric": "decode KV-cache GB/s", "value": dist.world * nbytes * K / (total_ms * 1e-3) / 1e9,
            "unit": "GB/s", "ms_per_step": total_ms / K, "bytes_per_step": nbytes,
-           "workload": w.name, "batch": w.batch, "len_range": [w.len_lo, w.len_hi],
+           "workload": w.name if w.batch == 64 else f"{w.name}-b{w.batch}", "batch": w.batch, "len_range": [w.len_lo, w.len_hi],
            "layers": ["sliding 16/8 d256 w1024 rolling 1024", "global K=V 16/2 d512",
                       "KV-shared global 16/2 d512"],
            "roofline": {"bound": "hbm", "kernel": "decode split-KV (global layer)",
@@ -478,7 +481,13 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=W.E2B_SLIDING.name,
+                    choices=[n for n in W.PREFILL_WORKLOADS if not n.startswith("tiny")])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="sequences of the decode step (default: the workload's 64)")
+    ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -493,6 +502,20 @@ def main(argv=None):
     torch.cuda.set_device(dist.local)
     G.lib()  # fail loudly if the CUDA library is missing
     pk, pk_src = peaks()
+    if args.decode_only:
+        dec = bench_decode(args, dist, pk)
+        dec["roofline"]["peak_source"] = f"{pk_src}: hbm_gbs"
+        if dist.rank == 0:
+            line = {"metric": METRIC, "value": dec["value"], "unit": "GB/s", "n_gpus": dist.world,
+                    "steps": args.steps, "warmup": args.warmup,
+                    "ms_per_step": dec["ms_per_step"], "higher_is_better": True,
+                    "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                    "config": {"workload": dec["workload"], "global_batch": dec["batch"] * dist.world},
+                    "roofline": dec["roofline"], "cpu_baseline": None, "e2e": None,
+                    "gpu_launches": dec["gpu_launches"], "clocks": dec["clocks"], "decode": dec}
+            print(json.dumps(line), flush=True)
+        dist.close()
+        return 0
     pre = bench_prefill(args, dist, pk)
     dec = None if args.no_decode else bench_decode(args, dist, pk)
     cpu = None

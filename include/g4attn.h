@@ -88,8 +88,8 @@ enum { G4ATTN_BF16 = 0, G4ATTN_FP32 = 1 };
  * rotary_fraction 1.0 and rope_theta 1e4.  Global layers: window ignored,
  * typically rotary_fraction 0.25 and rope_theta 1e6, k_eq_v on the K=V
  * variants.  rotary_fraction * head_dim must be an even integer.
- * softmax_scale multiplies q.k (1/sqrt(head_dim) or 1.0; the pages print
- * both); rms_eps is added to mean(x^2) (the pages do not state it; 1e-6 is
+ * softmax_scale (> 0) multiplies q.k (1/sqrt(head_dim) or 1.0; the pages
+ * print both); rms_eps is added to mean(x^2) (the pages do not state it; 1e-6 is
  * the usual value).  dtype is the element type of every raw input, weight,
  * output and cache tensor of the call. */
 typedef struct {

@@ -60,7 +60,8 @@ def ccache(d, B=1, C=64, rolling=0, **kw):
     dict(head_dim=96), dict(head_dim=1024), dict(num_heads=6, num_kv_heads=4),
     dict(num_kv_heads=0), dict(num_heads=64, num_kv_heads=64), dict(window=0),
     dict(rotary_fraction=0.3), dict(rotary_fraction=1.5), dict(rope_theta=-1.0),
-    dict(rms_eps=-1.0), dict(softmax_scale=float("inf")), dict(layer_type=2),
+    dict(rms_eps=-1.0), dict(softmax_scale=float("inf")), dict(softmax_scale=0.0),
+    dict(softmax_scale=-0.5), dict(layer_type=2),
 ])
 def test_bad_descriptors_are_rejected(bad):
     d = desc(**bad)
