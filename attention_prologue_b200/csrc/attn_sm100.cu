@@ -4,14 +4,16 @@
 // "What changed": bidirectional image blocks on sliding layers) and causal
 // global layers ("Global attention layers").
 //
-// One CTA computes 128 query rows of one query head:
+// One CTA computes 128 query rows: gp query heads that share one KV head
+// (GQA) x 128/gp consecutive positions, row r = (position r / gp, head
+// r % gp), so a tile spans fewer positions and meets fewer masked keys:
 //   warps 0, 2  TMA producers: Q tile once and K tiles (warp 0), V tiles
 //               (warp 2), 64 keys each, two-stage rings (128-byte swizzle,
 //               no multicast); a K slot is refilled as soon as S_j is done,
 //               a V slot as soon as PV_j is done
 //   warp 1      owns TMEM; one thread issues the MMAs:
-//                 S_j = Q K_j^T   (M 128, N 64, K = d; A, B K-major)
-//                 O  += P_j V_j   (M 128, N = d, K 64; P K-major, V MN-major)
+//                 S_j = Q K_j^T   (M 128, N 64, K = d; A, B K-major in smem)
+//                 O  += P_j V_j   (M 128, N = d, K 64; P from TMEM, V MN-major)
 //   warps 4..7  softmax: thread r owns query row r (TMEM lane r); reads S_j,
 //               masks it with the row's key interval [lo, hi], writes
 //               P_j = exp2(S_j - m) as bf16 into swizzled shared memory, and
@@ -40,23 +42,24 @@ namespace {
 
 constexpr int BM = 128;  // query rows per CTA
 constexpr int BN = 64;   // keys per tile
-constexpr int kStages = 2;
+constexpr int kStagesV = 2;
 constexpr int kThreads = 256;
 constexpr int kSoftmaxWarp0 = 4;
 
-template <int D>
+// D: head dims this CTA handles (the whole head, or half of it when kPair).
+template <int D, bool kPair>
 struct Layout {
+  static constexpr int kStagesK = kPair ? 2 : 3;          // K is needed one S before V
   static constexpr int kChunks = D / 64;                  // 64-element (128-byte) columns
   static constexpr uint32_t kQChunk = BM * 128;           // bytes of one Q chunk
   static constexpr uint32_t kKVChunk = BN * 128;          // bytes of one K or V chunk
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + kChunks * kQChunk;
-  static constexpr uint32_t kV = kK + kStages * kChunks * kKVChunk;
-  static constexpr uint32_t kP = kV + kStages * kChunks * kKVChunk;
-  static constexpr uint32_t kPBytes = BM * BN * 2;
-  static constexpr uint32_t kBars = kP + 2 * kPBytes;
-  static constexpr uint32_t kTotal = kBars + 256;       // barriers and scalars
-  static constexpr uint32_t kAlloc = kTotal + 1024;     // slack to align the base to 1024
+  static constexpr uint32_t kV = kK + kStagesK * kChunks * kKVChunk;
+  static constexpr uint32_t kX = kV + kStagesV * kChunks * kKVChunk;  // partial-S inbox
+  static constexpr uint32_t kBars = kX + (kPair ? BM * BN * 4 : 0);
+  static constexpr uint32_t kAlloc = kBars + 256;  // + barriers and scalars
+  static_assert(kAlloc <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
   static constexpr uint32_t kTmemCols = (128 + D) <= 256 ? 256 : 512;
   static constexpr uint32_t kColO = 128;
 };
@@ -64,15 +67,18 @@ struct Layout {
 struct Bars {  // offsets (in 8-byte words) of the mbarriers from Layout::kBars
   enum {
     q_full = 0,
-    k_full = 1,    // [2]
-    k_empty = 3,   // [2]
-    v_full = 5,    // [2]
-    v_empty = 7,   // [2]
-    s_full = 9,    // [2]
-    p_full = 11,   // [2]
-    o_done = 13,
-    drain = 14,
-    count = 15
+    k_full = 1,    // [3]
+    k_empty = 4,   // [3]
+    v_full = 7,    // [2]
+    v_empty = 9,   // [2]
+    s_full = 11,   // [2]
+    p_full = 13,   // [2]
+    o_done = 15,   // one phase per PV (rescale waits: always within one phase)
+    drain = 16,
+    o_last = 17,   // single phase: the last PV (the epilogue may lag several PVs)
+    rx_full = 18,  // pair: the peer's partial S of this tile is in the inbox
+    tx_ok = 19,    // pair: the peer has read what this CTA sent it
+    count = 20
   };
 };
 
@@ -84,34 +90,46 @@ struct Scalars {  // ints after the barriers
 
 }  // namespace
 
-template <int D>
+template <int D, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, RowIntervals rows,
                       __nv_bfloat16* __restrict__ out, int T_, int Hq, int Hkv, int layer_type,
-                      int window, float scale_log2, int* status) {
-  using Ly = Layout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* gbase = smem_raw + (base - raw);
+                      int window, float scale_log2, int gp_log2, int* status) {
+  using Ly = Layout<D, kPair>;
+  constexpr int kStagesK = Ly::kStagesK;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the 128-byte-swizzle atoms assume a 1024-byte aligned base
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) record_status(status, G4ATTN_EDEVICE);
+    return;
+  }
+  const uint32_t base = smem_u32(smem_raw);
+  uint8_t* gbase = smem_raw;
   const uint32_t bars = base + Ly::kBars;
   auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
   Scalars* sc = reinterpret_cast<Scalars*>(gbase + Ly::kBars + 8 * Bars::count);
   volatile int* abort = &sc->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = gridDim.x - 1 - blockIdx.x;  // longest (latest) row tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int r0 = tile * BM;
-  const int kvh = h / (Hq / Hkv);
+  // kPair: the two CTAs of a cluster share the rows and split the head dims
+  const uint32_t rank = kPair ? cluster_rank() : 0u;
+  const int dcol0 = (int)rank * D;  // first head dim of this CTA
+  const int n_rt = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int tile = n_rt - 1 - (kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x);  // latest first
+  const int b = blockIdx.z;
+  const int h0 = blockIdx.y << gp_log2;    // first query head of the tile
+  const int p0 = tile * (BM >> gp_log2);   // first position of the tile
+  const int kvh = h0 / (Hq / Hkv);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(Bars::q_full), 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesK; ++s) {
       mbar_init(bar(Bars::k_full + s), 1);
       mbar_init(bar(Bars::k_empty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(bar(Bars::v_full + s), 1);
       mbar_init(bar(Bars::v_empty + s), 1);
       mbar_init(bar(Bars::s_full + s), 1);
@@ -119,6 +137,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(Bars::o_done), 1);
     mbar_init(bar(Bars::drain), 1);
+    mbar_init(bar(Bars::o_last), 1);
+    mbar_init(bar(Bars::rx_full), 4 * 32);
+    mbar_init(bar(Bars::tx_ok), 4 * 32);
     sc->abort = 0;
     sc->klo = 0x7fffffff;
     sc->khi = -1;
@@ -137,8 +158,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   int lo = 1, hi = 0;
   const int r = threadIdx.x - kSoftmaxWarp0 * 32;  // row of a softmax thread
   __syncthreads();
+  const int i = p0 + (r >> gp_log2);             // position of a softmax thread's row
+  const int hrow = h0 + (r & ((1 << gp_log2) - 1));  // and its query head
   if (warp >= kSoftmaxWarp0) {
-    const int i = r0 + r;
     if (i < T_) {
       if (rows.lo) {
         lo = rows.lo[(long)b * T_ + i];
@@ -157,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if constexpr (kPair) cluster_sync_all();  // the peer's barriers exist before any remote use
   const uint32_t tmem = sc->tmem_base;
   const int kt0 = sc->klo / BN;
   const int n_tiles = sc->khi / BN - kt0 + 1;
@@ -171,27 +194,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ring = base + (is_k ? Ly::kK : Ly::kV);
       const int full = is_k ? Bars::k_full : Bars::v_full;
       const int empty = is_k ? Bars::k_empty : Bars::v_empty;
+      const int nst = is_k ? kStagesK : kStagesV;
       if (is_k) {
         mbar_arrive_expect_tx(bar(Bars::q_full), BM * D * 2);
         for (int c = 0; c < Ly::kChunks; ++c)
-          tma_load_4d(base + Ly::kQ + c * Ly::kQChunk, &tm_q, bar(Bars::q_full), c * 64, h, r0,
-                      b);
+          tma_load_4d(base + Ly::kQ + c * Ly::kQChunk, &tm_q, bar(Bars::q_full), dcol0 + c * 64,
+                      h0, p0, b);
       }
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % kStages;
-        if (!mbar_wait(bar(empty + s), ((j / kStages) & 1) ^ 1, abort)) break;
+        const int s = j % nst;
+        if (!mbar_wait(bar(empty + s), ((j / nst) & 1) ^ 1, abort)) break;
         const int key0 = (kt0 + j) * BN;
         mbar_arrive_expect_tx(bar(full + s), BN * D * 2);
         for (int c = 0; c < Ly::kChunks; ++c)
-          tma_load_3d(ring + (s * Ly::kChunks + c) * Ly::kKVChunk, tm, bar(full + s), c * 64,
-                      key0, b * Hkv + kvh);
+          tma_load_3d(ring + (s * Ly::kChunks + c) * Ly::kKVChunk, tm, bar(full + s),
+                      dcol0 + c * 64, key0, b * Hkv + kvh);
         issued = j + 1;
       }
       if (*abort) {  // let the copies already issued land before the CTA exits
         if (is_k) mbar_wait(bar(Bars::q_full), 0, nullptr);
-        for (int j = max(0, issued - kStages); j < issued; ++j)
-          mbar_wait(bar(full + j % kStages), (j / kStages) & 1, nullptr);
+        for (int j = max(0, issued - nst); j < issued; ++j)
+          mbar_wait(bar(full + j % nst), (j / nst) & 1, nullptr);
       }
     }
   } else if (warp == 1) {
@@ -200,22 +224,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_s = idesc_bf16(BM, BN, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16(BM, D, 0, 1);
       auto issue_pv = [&](int j) {
-        const int s = j % kStages;
-        const uint32_t pbase = base + Ly::kP + (j & 1) * Ly::kPBytes;
+        const int s = j % kStagesV;
         const uint32_t vbase = base + Ly::kV + s * Ly::kChunks * Ly::kKVChunk;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = desc_sw128(pbase + kk * 32, 16, 1024);
+          // A = P_j in TMEM: row m in lane m, 16 keys = 8 packed columns per step
           const uint64_t bd = desc_sw128(vbase + kk * 16 * 128, Ly::kKVChunk, 1024);
-          mma_ss(tmem + Ly::kColO, a, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + Ly::kColO, tmem + (j & 1) * BN + kk * 8, bd, idesc_o,
+                 (j > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(bar(Bars::v_empty + s));
         mma_commit(bar(Bars::o_done));
       };
       bool ok = mbar_wait(bar(Bars::q_full), 0, abort);
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kStages;
-        if (!(ok = mbar_wait(bar(Bars::k_full + s), (j / kStages) & 1, abort))) break;
+        const int s = j % kStagesK;
+        if (!(ok = mbar_wait(bar(Bars::k_full + s), (j / kStagesK) & 1, abort))) break;
         tc_fence_after();
         const uint32_t kbase = base + Ly::kK + s * Ly::kChunks * Ly::kKVChunk;
 #pragma unroll
@@ -230,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= 1) {
           if (!(ok = mbar_wait(bar(Bars::p_full + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort)))
             break;
-          if (!(ok = mbar_wait(bar(Bars::v_full + (j - 1) % kStages), ((j - 1) / kStages) & 1,
+          if (!(ok = mbar_wait(bar(Bars::v_full + (j - 1) % kStagesV), ((j - 1) / kStagesV) & 1,
                                abort)))
             break;
           tc_fence_after();
@@ -239,10 +263,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ok && mbar_wait(bar(Bars::p_full + ((n_tiles - 1) & 1)), ((n_tiles - 1) >> 1) & 1,
                           abort) &&
-          mbar_wait(bar(Bars::v_full + (n_tiles - 1) % kStages), ((n_tiles - 1) / kStages) & 1,
-                    abort)) {
+          mbar_wait(bar(Bars::v_full + (n_tiles - 1) % kStagesV),
+                    ((n_tiles - 1) / kStagesV) & 1, abort)) {
         tc_fence_after();
         issue_pv(n_tiles - 1);
+        mma_commit(bar(Bars::o_last));
       }
       if (*abort) {  // every MMA issued so far completes before TMEM is freed
         mma_commit(bar(Bars::drain));
@@ -262,6 +287,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tmem + lane_off + (j & 1) * BN, sr);
       tmem_ld32(tmem + lane_off + (j & 1) * BN + 32, sr + 32);
       tmem_wait_ld();
+      if constexpr (kPair) {
+        // S = this CTA's partial (its half of the head dims) + the peer's.
+        // Send ours into the peer's inbox row r (16-byte slot q at q ^ (r & 15)),
+        // then read the peer's from our inbox; both CTAs add the same two fp32
+        // values, so both softmaxes see bit-identical scores.
+        if (j > 0) {  // the peer has read the previous tile's partial
+          ok = __all_sync(0xffffffffu, mbar_wait_cluster(bar(Bars::tx_ok), (j - 1) & 1, abort));
+          if (!ok) break;
+        }
+        const uint32_t inbox_row = base + Ly::kX + r * (BN * 4);
+#pragma unroll
+        for (int q = 0; q < BN / 4; ++q) {
+          const uint32_t dst = map_peer(inbox_row + ((q ^ (r & 15)) << 4), rank ^ 1u);
+          st_cluster_v4(dst, __uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1]),
+                        __uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3]));
+        }
+        mbar_arrive_remote(map_peer(bar(Bars::rx_full), rank ^ 1u));
+        ok = __all_sync(0xffffffffu, mbar_wait_cluster(bar(Bars::rx_full), j & 1, abort));
+        if (!ok) break;
+        const float4* inbox = reinterpret_cast<const float4*>(gbase + Ly::kX + r * (BN * 4));
+#pragma unroll
+        for (int q = 0; q < BN / 4; ++q) {
+          const float4 v = inbox[q ^ (r & 15)];
+          sr[4 * q] = __float_as_uint(__uint_as_float(sr[4 * q]) + v.x);
+          sr[4 * q + 1] = __float_as_uint(__uint_as_float(sr[4 * q + 1]) + v.y);
+          sr[4 * q + 2] = __float_as_uint(__uint_as_float(sr[4 * q + 2]) + v.z);
+          sr[4 * q + 3] = __float_as_uint(__uint_as_float(sr[4 * q + 3]) + v.w);
+        }
+        mbar_arrive_remote(map_peer(bar(Bars::tx_ok), rank ^ 1u));
+      }
       const int key0 = (kt0 + j) * BN;
       float x[BN];
       float mt = -INFINITY;
@@ -303,40 +358,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
       }
       if (first && mt != -INFINITY) m_used = mt;
-      // P = exp2(x - m_used) as bf16, written in the 128-byte-swizzled
-      // K-major layout: 16-byte chunk q of row r goes to chunk q ^ (r & 7)
-      const uint32_t prow = base + Ly::kP + (j & 1) * Ly::kPBytes + r * 128;
+      // P = exp2(x - m_used) as packed bf16 pairs, stored over the first 32
+      // columns of this tile's S buffer (the PV MMA reads A from TMEM; the
+      // next S MMA into this buffer is issued after that PV)
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;  // row with no key yet: P = 0
       float rs = 0.f;
+      uint32_t pk[BN / 2];
 #pragma unroll
-      for (int q = 0; q < BN / 8; ++q) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = ex2_approx(fmaf(x[8 * q + 2 * e], scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(x[8 * q + 2 * e + 1], scale_log2, neg_m));
-          rs += p0 + p1;
-          __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
-          pk[e] = *reinterpret_cast<uint32_t*>(&bb);
-        }
-        const uint32_t dst = prow + ((q ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[0]),
-                     "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
-                     : "memory");
+      for (int e = 0; e < BN / 2; ++e) {
+        const float p0 = ex2_approx(fmaf(x[2 * e], scale_log2, neg_m));
+        const float p1 = ex2_approx(fmaf(x[2 * e + 1], scale_log2, neg_m));
+        rs += p0 + p1;
+        __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
+        pk[e] = *reinterpret_cast<uint32_t*>(&bb);
       }
+      tmem_st32(tmem + lane_off + (j & 1) * BN, pk);
+      tmem_wait_st();
       l += rs;
-      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(Bars::p_full + (j & 1)));
     }
     // ------------------------------------------------------------ epilogue
     if (ok)  // warp-uniform: the tcgen05 loads below are warp-collective
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::o_done), (n_tiles - 1) & 1, abort));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::o_last), 0, abort));
     if (ok) {
       tc_fence_after();
-      const int i = r0 + r;
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = out + (((long)b * T_ + i) * Hq + h) * D;
+      __nv_bfloat16* dst = out + (((long)b * T_ + i) * Hq + hrow) * (kPair ? 2 * D : D) + dcol0;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -359,6 +407,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  if constexpr (kPair) {
+    // the peer's last access to this CTA is its read receipt for the last
+    // tile: wait for it (bounded) before the CTA's shared memory goes away
+    if (warp >= kSoftmaxWarp0 && n_tiles > 0)
+      mbar_wait_cluster(bar(Bars::tx_ok), (n_tiles - 1) & 1, nullptr);
+  }
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort) record_status(status, G4ATTN_EDEVICE);
@@ -411,33 +465,60 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
          CUDA_SUCCESS;
 }
 
-template <int D>
+// Query heads packed per tile: the largest power of two <= 8 dividing
+// Hq / Hkv (every head of a tile reads the same KV head).
+int pack_log2(const LayerCfg& L) {
+  const int g = L.Hq / L.Hkv;
+  int lg = 0;
+  while (lg < 3 && g % (2 << lg) == 0) ++lg;
+  return lg;
+}
+
+template <int D, bool kPair>
 cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
                       RowIntervals rows, void* out, int* status, cudaStream_t s) {
+  static_assert(!kPair || D == 256, "pairs split head_dim 512");
   CUtensorMap tq, tk, tv;
+  const int gp_log2 = pack_log2(L);
+  constexpr int DF = kPair ? 2 * D : D;  // full head dim
   const uint64_t es = 2;
   {  // q_hat [B, T, Hq, D]: dims (D, Hq, T, B)
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)L.Hq, (uint64_t)T, (uint64_t)B};
-    const uint64_t str[3] = {D * es, (uint64_t)L.Hq * D * es, (uint64_t)T * L.Hq * D * es};
-    const uint32_t box[4] = {64, 1, BM, 1};
+    const uint64_t dims[4] = {(uint64_t)DF, (uint64_t)L.Hq, (uint64_t)T, (uint64_t)B};
+    const uint64_t str[3] = {DF * es, (uint64_t)L.Hq * DF * es, (uint64_t)T * L.Hq * DF * es};
+    const uint32_t box[4] = {64, (uint32_t)(1 << gp_log2), (uint32_t)(BM >> gp_log2), 1};
     if (!make_map(&tq, q_hat, 4, dims, str, box)) return cudaErrorInvalidValue;
   }
   {  // K, V [B * Hkv, cap, D]; only positions < T exist (rows past T read as 0)
-    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)T, (uint64_t)B * L.Hkv};
-    const uint64_t str[2] = {D * es, (uint64_t)kv.cap * D * es};
+    const uint64_t dims[3] = {(uint64_t)DF, (uint64_t)T, (uint64_t)B * L.Hkv};
+    const uint64_t str[2] = {DF * es, (uint64_t)kv.cap * DF * es};
     const uint32_t box[3] = {64, BN, 1};
     if (!make_map(&tk, kv.k, 3, dims, str, box)) return cudaErrorInvalidValue;
     if (!make_map(&tv, kv.v, 3, dims, str, box)) return cudaErrorInvalidValue;
   }
-  using Ly = Layout<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D>,
+  using Ly = Layout<D, kPair>;
+  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D, kPair>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
   if (e != cudaSuccess) return e;
   const float scale_log2 = L.scale * 1.4426950408889634f;
-  dim3 grid((T + BM - 1) / BM, L.Hq, B);
-  attn_sm100_kernel<D><<<grid, kThreads, Ly::kAlloc, s>>>(
-      tq, tk, tv, rows, static_cast<__nv_bfloat16*>(out), T, L.Hq, L.Hkv, L.layer_type, L.window,
-      scale_log2, status);
+  const int bp = BM >> gp_log2;  // positions per tile
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((T + bp - 1) / bp * (kPair ? 2 : 1), L.Hq >> gp_log2, B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Ly::kAlloc;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  if (kPair) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  e = cudaLaunchKernelEx(&cfg, attn_sm100_kernel<D, kPair>, tq, tk, tv, rows,
+                         static_cast<__nv_bfloat16*>(out), T, L.Hq, L.Hkv, L.layer_type, L.window,
+                         scale_log2, gp_log2, status);
+  if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();
 }
@@ -445,15 +526,16 @@ cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc 
 }  // namespace
 
 bool attention_sm100_supported(const LayerCfg& L) {
-  return L.dtype == 0 && (L.d == 64 || L.d == 128 || L.d == 256);
+  return L.dtype == 0 && (L.d == 64 || L.d == 128 || L.d == 256 || L.d == 512);
 }
 
 cudaError_t launch_attention_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
                                    RowIntervals rows, void* out, int* status, cudaStream_t s) {
   switch (L.d) {
-    case 64: return run_sm100<64>(L, B, T, q_hat, kv, rows, out, status, s);
-    case 128: return run_sm100<128>(L, B, T, q_hat, kv, rows, out, status, s);
-    case 256: return run_sm100<256>(L, B, T, q_hat, kv, rows, out, status, s);
+    case 64: return run_sm100<64, false>(L, B, T, q_hat, kv, rows, out, status, s);
+    case 128: return run_sm100<128, false>(L, B, T, q_hat, kv, rows, out, status, s);
+    case 256: return run_sm100<256, false>(L, B, T, q_hat, kv, rows, out, status, s);
+    case 512: return run_sm100<256, true>(L, B, T, q_hat, kv, rows, out, status, s);
   }
   return cudaErrorInvalidValue;
 }

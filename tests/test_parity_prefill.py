@@ -147,3 +147,15 @@ def test_full_size_sampled(w, n):
             rows += [s, s + 1, s + w.block_len - 1, s + w.block_len]
         rows = sorted(set(rows))
     run_case(w, seed=0, rows=rows)
+
+
+@pytest.mark.parametrize("T", [17, 65, 100, 127, 129, 200])
+def test_few_tile_prompts_repeated(T):
+    """Prompts of one to four key tiles, run several times: the epilogue must
+    wait for the last PV product even when the softmax finishes early."""
+    for L in (W.sliding(8, 1, 256, 512), W.global_(8, 2, 256), W.sliding(4, 2, 128, 64)):
+        w = W.PrefillWorkload(f"rep{T}", L, 2, T)
+        inp = W.prefill_inputs(w, DEV, T)
+        ref = oracle_prefill(w, inp)
+        for _ in range(4):
+            check(gpu_prefill(w, inp), ref, w.dtype, f"{w.name} d{L.head_dim}")
