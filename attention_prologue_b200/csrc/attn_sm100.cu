@@ -446,9 +446,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // bf16 tensor map with a 128-byte-swizzled box; dims[0] is the contiguous one.
-bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box) {
+bool make_bf16_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+                   const uint64_t* strides_bytes, const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gd[5], gs[4];
@@ -463,6 +465,13 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
+}
+
+namespace {
+
+bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+  return make_bf16_map(m, ptr, rank, dims, strides_bytes, box);
 }
 
 // Query heads packed per tile: the largest power of two <= 8 dividing

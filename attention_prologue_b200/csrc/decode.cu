@@ -5,7 +5,9 @@
 // layer's cache and computes only its queries).
 //
 // Split-KV: the keys of sequence b, [lo, P] with P = len[b] - 1, are cut into
-// fixed-size chunks; CTA (chunk, KV head, sequence) computes for the query
+// fixed-size chunks on a grid aligned to 16 positions (chunk c covers
+// [base + c*chunk, base + (c+1)*chunk) with base = lo rounded down to a
+// multiple of 16, clipped to [lo, P]); CTA (chunk, KV head, sequence) computes for the query
 // heads of that KV head the partial softmax of the chunk
 //   m = max_j s_j,  l = sum_j e^{s_j - m},  o~ = sum_j e^{s_j - m} v_j,
 // and the combine kernel merges the chunks with
@@ -22,8 +24,8 @@ constexpr int kDecHeads = 4;  // query heads handled per pass over the chunk
 DecodePlan decode_plan(const LayerCfg& L, int cap) {
   DecodePlan p;
   const long span = L.layer_type == 0 ? (long)(L.window < cap ? L.window : cap) : (long)cap;
-  p.chunk = span <= 4096 ? 256 : 2048;
-  p.n_chunks = (int)((span + p.chunk - 1) / p.chunk);
+  p.chunk = span <= 4096 ? 256 : 2048;  // a multiple of 16
+  p.n_chunks = (int)((span + 15 + p.chunk - 1) / p.chunk);  // the aligned grid adds <= 15
   return p;
 }
 
@@ -59,9 +61,10 @@ __global__ void __launch_bounds__(kDecWarps * 32)
   }
   const int P = L - 1;
   const int lo = decode_lo(P, layer_type, window);
-  const int k_begin = lo + c * chunk;
-  if (k_begin > P) return;
-  const int k_end = min(P + 1, k_begin + chunk);
+  const int c0 = (lo & ~15) + c * chunk;
+  if (c0 > P) return;
+  const int k_begin = max(lo, c0);
+  const int k_end = min(P + 1, c0 + chunk);
   const long kv_base = ((long)b * Hkv + kvh) * cap;
 
   for (int hg = 0; hg < g; hg += kDecHeads) {
@@ -158,7 +161,7 @@ __global__ void __launch_bounds__(128)
     return;
   }
   const int P = L - 1;
-  const int n = P - decode_lo(P, layer_type, window) + 1;
+  const int n = P + 1 - (decode_lo(P, layer_type, window) & ~15);
   const int cnt = (n + chunk - 1) / chunk;
   const long base = ((long)b * Hq + h) * nc;
   float M = -INFINITY;
@@ -183,13 +186,19 @@ static cudaError_t run_decode(const LayerCfg& L, int B, const void* q_raw, const
   float* part_o = partials + 2 * (size_t)B * L.Hq * plan.n_chunks;
   dim3 grid(plan.n_chunks, L.Hkv, B);
   if (ev0) cudaEventRecord(ev0, s);
-  decode_split_kernel<T, D><<<grid, kDecWarps * 32, 0, s>>>(
-      static_cast<const T*>(q_raw), static_cast<const T*>(wq), static_cast<const T*>(cache_k),
-      static_cast<const T*>(cache_v), len, cap, rolling, L.Hq, L.Hkv, L.layer_type, L.window,
-      L.scale, L.eps, plan.chunk, plan.n_chunks, part_ml, part_o, status, L.rope);
-  count_launch();
+  cudaError_t e;
+  if (decode_mma_supported(L, cap, rolling)) {
+    e = launch_decode_mma(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, plan, part_ml,
+                          part_o, status, s);
+  } else {
+    decode_split_kernel<T, D><<<grid, kDecWarps * 32, 0, s>>>(
+        static_cast<const T*>(q_raw), static_cast<const T*>(wq), static_cast<const T*>(cache_k),
+        static_cast<const T*>(cache_v), len, cap, rolling, L.Hq, L.Hkv, L.layer_type, L.window,
+        L.scale, L.eps, plan.chunk, plan.n_chunks, part_ml, part_o, status, L.rope);
+    count_launch();
+    e = cudaGetLastError();
+  }
   if (ev1) cudaEventRecord(ev1, s);
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_combine_kernel<T, D><<<dim3(L.Hq, B), 128, 0, s>>>(part_ml, part_o, len, L.Hq,
                                                             L.layer_type, L.window, plan.chunk,

@@ -1,0 +1,362 @@
+// Split-KV decode on tensor cores for bf16 caches ("Gemma 4" Keras docs,
+// "Gemma4ConditionalGenerate": decoding over the per-layer KV cache;
+// "Gemma 4" overview blog, "Shared KV Cache").
+//
+// The query heads of one KV head (g <= 8; grouped-query attention) form the
+// N = 8 side of m16n8k16 MMAs, so every cache byte is read once per KV head
+// and the arithmetic stays far below the tensor pipe's rate: the kernel is an
+// HBM stream.
+//
+// CTA = (chunk of positions, KV head, sequence), 5 warps:
+//   warp 4     TMA producer: 16-key K and V tiles (128-byte swizzled boxes of
+//              64 dims) into a ring of NS stages (128-192 KB in flight)
+//   warps 0-3  take tiles round-robin (tile i: warp i % 4, stage i % NS with
+//              NS a multiple of 4, so every stage has one consumer); per tile:
+//                S^T = K Q^T            (16 keys x 8 heads, ldmatrix + mma)
+//                online softmax per head (the thread's two heads are the same
+//                in S^T and in its O^T accumulators: no shuffles for O)
+//                O^T += V^T P^T         (ldmatrix.trans for V^T, movmatrix
+//                                        turns P into the B operand)
+// At the end the 4 warps' partial softmaxes are merged in shared memory and
+// the chunk's (m, l, o~) are written for the combine kernel (decode.cu).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "g4attn.h"
+#include "sm100.cuh"
+
+namespace g4 {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kConsumers = 4;
+constexpr int kThreadsDm = (kConsumers + 1) * 32;
+constexpr int kKeys = 16;  // keys per tile
+
+template <int D>
+struct DmLayout {
+  static constexpr int kBoxes = D / 64;
+  static constexpr uint32_t kBox = kKeys * 128;            // 16 keys x 64 dims, 2 KB
+  static constexpr uint32_t kTile = kBoxes * kBox;         // K (or V) of one tile
+  static constexpr uint32_t kStage = 2 * kTile;            // K then V
+  // Stage count: a multiple of the consumer count, so stage s is only ever
+  // consumed by warp s % 4 and that warp waits its phases in order (a parity
+  // wait is only meaningful when the previous phase is known to be complete).
+  static constexpr int kFit = (192 * 1024) / kStage > 16 ? 16 : (192 * 1024) / kStage;
+  static constexpr int kStages = kFit - kFit % kConsumers;
+  static_assert(kStages >= kConsumers, "at least one stage per consumer");
+  static constexpr uint32_t kQ = kStages * kStage;         // q_hat [8][D] bf16
+  static constexpr uint32_t kBars = kQ + 8 * D * 2;        // full[NS], empty[NS]
+  static constexpr uint32_t kAlloc = kBars + 2 * kStages * 8 + 64;
+  static_assert(kConsumers * 8 * D * 4 + kConsumers * 8 * 8 <= kQ, "merge buffer fits");
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+// D (16x8, fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Byte offset of (key, dim) inside a K or V tile: box dim/64, row key, the
+// 16-byte chunk of the dim swizzled by the row (128-byte swizzle).
+__device__ __forceinline__ uint32_t tile_off(int key, int dim) {
+  return (uint32_t)((dim >> 6) * (kKeys * 128) + key * 128 + ((((dim & 63) >> 3) ^ (key & 7)) << 4));
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kThreadsDm, 1)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __restrict__ wq,
+                      const int32_t* __restrict__ len, int cap, int rolling, int Hq, int Hkv,
+                      int layer_type, int window, float scale_log2, float eps, int chunk, int nc,
+                      float* __restrict__ part_ml, float* __restrict__ part_o, int* status,
+                      const __grid_constant__ RopeParams rope) {
+  using Ly = DmLayout<D>;
+  constexpr int NS = Ly::kStages;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if (smem_u32(smem) & 1023u) {  // the swizzled boxes assume a 1024-byte aligned base
+    if (threadIdx.x == 0) record_status(status, G4ATTN_EDEVICE);
+    return;
+  }
+  const uint32_t base = smem_u32(smem);
+  const uint32_t bars = base + Ly::kBars;
+  __shared__ int s_abort;
+  volatile int* abort = &s_abort;
+
+  const int c = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = Hq / Hkv;
+  const int L = len[b];
+  if (L <= 0 || (!rolling && L > cap)) {  // nothing to read / len past the end: no access
+    if (c == 0 && kvh == 0 && threadIdx.x == 0)
+      record_status(status, L <= 0 ? G4ATTN_ECACHE_EMPTY : G4ATTN_ECACHE_OVERFLOW);
+    return;
+  }
+  const int P = L - 1;
+  const int lo = layer_type == 0 ? max(0, P - window + 1) : 0;
+  const int c0 = (lo & ~15) + c * chunk;  // chunk start, 16-aligned
+  if (c0 > P) return;
+  const int c1 = min(P + 1, c0 + chunk);
+  const int t0 = c0 >> 4;
+  const int n_t = ((c1 - 1) >> 4) - t0 + 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bars + 8 * s, 1);             // full: producer's expect_tx
+      mbar_init(bars + 8 * (NS + s), 1);      // empty: the consuming warp
+    }
+    s_abort = 0;
+    fence_barrier_init();
+  }
+  // query prologue (RMSNorm * w_q, RoPE at P) of the g heads into q_hat; rows g..7 zero
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem + Ly::kQ);
+  if (warp < kConsumers) {
+    for (int hh = warp; hh < 8; hh += kConsumers) {
+      if (hh < g) {
+        float y0[D / 64], y1[D / 64];
+        prologue_vec<__nv_bfloat16, D>(q_raw + ((long)b * Hq + kvh * g + hh) * D, wq, P, &rope,
+                                       eps, y0, y1);
+        store_vec<__nv_bfloat16, D>(qs + hh * D, y0, y1);
+      } else {
+        for (int k = lane; k < D; k += 32) qs[hh * D + k] = __float2bfloat16_rn(0.f);
+      }
+    }
+  }
+  __syncthreads();
+
+  float acc[D / 16][4];  // O^T of this thread: dims 16mt + lane/4 (+8) x heads hA, hB
+#pragma unroll
+  for (int mt = 0; mt < D / 16; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+  float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;  // heads hA = 2(lane%4), hB = hA+1
+
+  if (warp == kConsumers) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      int issued = 0;
+      for (int i = 0; i < n_t; ++i) {
+        const int s = i % NS;
+        if (!mbar_wait(bars + 8 * (NS + s), ((i / NS) & 1) ^ 1, abort)) break;
+        const int pos = (t0 + i) * kKeys;
+        const int slot = rolling ? pos % cap : pos;  // rolling caches: cap % 16 == 0
+        const uint32_t st = base + s * Ly::kStage;
+        mbar_arrive_expect_tx(bars + 8 * s, Ly::kStage);
+#pragma unroll
+        for (int bx = 0; bx < Ly::kBoxes; ++bx) {
+          tma_load_3d(st + bx * Ly::kBox, &tm_k, bars + 8 * s, bx * 64, slot, b * Hkv + kvh);
+          tma_load_3d(st + Ly::kTile + bx * Ly::kBox, &tm_v, bars + 8 * s, bx * 64, slot,
+                      b * Hkv + kvh);
+        }
+        issued = i + 1;
+      }
+      if (*abort)  // let the copies already issued land before the CTA exits
+        for (int i = max(0, issued - NS); i < issued; ++i)
+          mbar_wait(bars + 8 * (i % NS), (i / NS) & 1, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    // B operand of S^T = K Q^T for every 16-dim step: q_hat[head = lane/4][dims]
+    uint32_t qb[D / 16][2];
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const __nv_bfloat16* qr = qs + (lane >> 2) * D + kk * 16 + (lane & 3) * 2;
+      qb[kk][0] = *reinterpret_cast<const uint32_t*>(qr);
+      qb[kk][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
+    }
+    for (int i = warp; i < n_t; i += kConsumers) {
+      const int s = i % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * s, (i / NS) & 1, abort))) break;
+      const uint32_t kb = base + s * Ly::kStage, vb = kb + Ly::kTile;
+      const int pos0 = (t0 + i) * kKeys;
+      if (pos0 + kKeys - 1 > P) {  // last tile: zero V rows past P (never written)
+        const int first = P - pos0 + 1;
+        uint8_t* vrow = smem + s * Ly::kStage + Ly::kTile;
+        for (int e = lane; e < (kKeys - first) * Ly::kBoxes * 8; e += 32) {
+          const int rr = first + e / (Ly::kBoxes * 8), rest = e % (Ly::kBoxes * 8);
+          *reinterpret_cast<uint4*>(vrow + (rest >> 3) * Ly::kBox + rr * 128 + (rest & 7) * 16) =
+              make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();  // a later TMA refill of this stage comes after these writes
+        __syncwarp();
+      }
+      // S^T (16 keys x 8 heads)
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int mi = lane >> 3;
+        const int key = (lane & 7) + (mi & 1) * 8;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          uint32_t a[4];
+          ldsm_x4(kb + tile_off(key, kk * 16 + (mi >> 1) * 8), a);
+          mma16816(sc, a, qb[kk][0], qb[kk][1]);
+        }
+      }
+      // masked scores in log2 units: rows = keys pos0 + lane/4 (+8), cols = heads
+      const int kA = pos0 + (lane >> 2), kB = kA + 8;
+      const bool vA = kA >= lo && kA <= P, vB = kB >= lo && kB <= P;
+      const float x0 = vA ? sc[0] * scale_log2 : -INFINITY;  // (kA, head hA)
+      const float x1 = vA ? sc[1] * scale_log2 : -INFINITY;  // (kA, head hB)
+      const float x2 = vB ? sc[2] * scale_log2 : -INFINITY;  // (kB, head hA)
+      const float x3 = vB ? sc[3] * scale_log2 : -INFINITY;  // (kB, head hB)
+      float tA = fmaxf(x0, x2), tB = fmaxf(x1, x3);
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        tA = fmaxf(tA, __shfl_xor_sync(0xffffffffu, tA, o));
+        tB = fmaxf(tB, __shfl_xor_sync(0xffffffffu, tB, o));
+      }
+      const float nA = fmaxf(mA, tA), nB = fmaxf(mB, tB);
+      const float ngA = nA == -INFINITY ? 0.f : -nA, ngB = nB == -INFINITY ? 0.f : -nB;
+      const float cA = ex2_approx(mA + ngA), cB = ex2_approx(mB + ngB);  // 0 while m = -inf
+      const float p0 = ex2_approx(x0 + ngA), p2 = ex2_approx(x2 + ngA);
+      const float p1 = ex2_approx(x1 + ngB), p3 = ex2_approx(x3 + ngB);
+      float sA = p0 + p2, sB = p1 + p3;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        sA += __shfl_xor_sync(0xffffffffu, sA, o);
+        sB += __shfl_xor_sync(0xffffffffu, sB, o);
+      }
+      lA = lA * cA + sA;
+      lB = lB * cB + sB;
+      mA = nA;
+      mB = nB;
+      // P^T as the B operand: transpose the (keys x heads) 8x8 blocks
+      const uint32_t pb0 = movm_t(pack_bf16(p0, p1));
+      const uint32_t pb1 = movm_t(pack_bf16(p2, p3));
+      {
+        const int mi = lane >> 3;
+        const int key = (lane & 7) + (mi >> 1) * 8;
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+          acc[mt][0] *= cA;
+          acc[mt][1] *= cB;
+          acc[mt][2] *= cA;
+          acc[mt][3] *= cB;
+          uint32_t a[4];
+          ldsm_x4_t(vb + tile_off(key, mt * 16 + (mi & 1) * 8), a);
+          mma16816(acc[mt], a, pb0, pb1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars + 8 * (NS + s));
+    }
+  }
+  __syncthreads();  // every tile consumed: no copy is in flight, the ring can be reused
+  if (*abort) {
+    if (threadIdx.x == 0) record_status(status, G4ATTN_EDEVICE);
+    return;
+  }
+  // merge the 4 warps' partial softmaxes (each relative to its own maxima)
+  float* red = reinterpret_cast<float*>(smem);                           // [4][8][D]
+  float* rml = reinterpret_cast<float*>(smem + kConsumers * 8 * D * 4);  // [4][8][m, l]
+  if (warp < kConsumers) {
+    const int hA = 2 * (lane & 3), hB = hA + 1, dr = lane >> 2;
+    float* ra = red + (warp * 8 + hA) * D;
+    float* rb = red + (warp * 8 + hB) * D;
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+      ra[mt * 16 + dr] = acc[mt][0];
+      rb[mt * 16 + dr] = acc[mt][1];
+      ra[mt * 16 + dr + 8] = acc[mt][2];
+      rb[mt * 16 + dr + 8] = acc[mt][3];
+    }
+    if (lane < 4) {
+      rml[(warp * 8 + hA) * 2] = mA;
+      rml[(warp * 8 + hA) * 2 + 1] = lA;
+      rml[(warp * 8 + hB) * 2] = mB;
+      rml[(warp * 8 + hB) * 2 + 1] = lB;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < g * D; e += blockDim.x) {
+    const int h = e / D, dim = e - h * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, rml[(w * 8 + h) * 2]);
+    float den = 0.f, o = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumers; ++w) {
+      const float mw = rml[(w * 8 + h) * 2];
+      const float a = mw == -INFINITY ? 0.f : ex2_approx(mw - M);
+      den += a * rml[(w * 8 + h) * 2 + 1];
+      o += a * red[(w * 8 + h) * D + dim];
+    }
+    const long pidx = ((long)b * Hq + kvh * g + h) * nc + c;
+    part_o[pidx * D + dim] = o;
+    if (dim == 0) {  // the combine kernel works in natural-log units
+      part_ml[2 * pidx] = M * 0.69314718055994531f;
+      part_ml[2 * pidx + 1] = den;
+    }
+  }
+}
+
+bool decode_mma_supported(const LayerCfg& L, int cap, int rolling) {
+  return L.dtype == 0 && L.Hq / L.Hkv <= 8 && (!rolling || cap % kKeys == 0);
+}
+
+template <int D>
+static cudaError_t run_mma(const LayerCfg& L, int B, const void* q_raw, const void* wq,
+                           const void* cache_k, const void* cache_v, const int32_t* len, int cap,
+                           int rolling, const DecodePlan& plan, float* part_ml, float* part_o,
+                           int* status, cudaStream_t s) {
+  using Ly = DmLayout<D>;
+  CUtensorMap tk, tv;
+  const uint64_t dims[3] = {(uint64_t)D, (uint64_t)cap, (uint64_t)B * L.Hkv};
+  const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)cap * D * 2};
+  const uint32_t box[3] = {64, kKeys, 1};
+  if (!make_bf16_map(&tk, cache_k, 3, dims, str, box)) return cudaErrorInvalidValue;
+  if (!make_bf16_map(&tv, cache_v, 3, dims, str, box)) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
+  if (e != cudaSuccess) return e;
+  dim3 grid(plan.n_chunks, L.Hkv, B);
+  decode_mma_kernel<D><<<grid, kThreadsDm, Ly::kAlloc, s>>>(
+      tk, tv, static_cast<const __nv_bfloat16*>(q_raw), static_cast<const __nv_bfloat16*>(wq), len,
+      cap, rolling, L.Hq, L.Hkv, L.layer_type, L.window, L.scale * 1.4426950408889634f, L.eps,
+      plan.chunk, plan.n_chunks, part_ml, part_o, status, L.rope);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_mma(const LayerCfg& L, int B, const void* q_raw, const void* wq,
+                              const void* cache_k, const void* cache_v, const int32_t* len,
+                              int cap, int rolling, const DecodePlan& plan, float* part_ml,
+                              float* part_o, int* status, cudaStream_t s) {
+  switch (L.d) {
+    case 64: return run_mma<64>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, plan, part_ml, part_o, status, s);
+    case 128: return run_mma<128>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, plan, part_ml, part_o, status, s);
+    case 256: return run_mma<256>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, plan, part_ml, part_o, status, s);
+    case 512: return run_mma<512>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, plan, part_ml, part_o, status, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace g4

@@ -47,10 +47,10 @@ int launch_decode_noalloc(const LayerCfg& L, int B, const void* q_raw, const voi
   const size_t max_chunks = kDecodeScratchBytes / per_chunk;
   if (max_chunks == 0) return G4ATTN_EWORKSPACE;  // one chunk's partials exceed the array
   if ((size_t)plan.n_chunks > max_chunks) {
-    // fewer, longer chunks covering at least the same key span
+    // fewer, longer chunks (still multiples of 16) covering at least the same span
     const long span = (long)plan.chunk * plan.n_chunks;
     plan.n_chunks = (int)max_chunks;
-    plan.chunk = (int)((span + plan.n_chunks - 1) / plan.n_chunks);
+    plan.chunk = (int)(((span + plan.n_chunks - 1) / plan.n_chunks + 15) & ~15L);
   }
   float* scratch = decode_scratch_ptr();
   if (!scratch) return G4ATTN_ECUDA;

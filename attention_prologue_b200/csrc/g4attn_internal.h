@@ -81,11 +81,28 @@ cudaError_t launch_decode(const LayerCfg& L, int B, const void* q_raw, const voi
                           int rolling, const DecodePlan& plan, float* partials, void* out,
                           int* status, cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1);
 
+// Tensor-core split kernel of g4attn_decode (bf16, <= 8 query heads per KV
+// head, rolling caches with capacity % 16 == 0); writes the same partials
+// as the CUDA-core split kernel.
+bool decode_mma_supported(const LayerCfg& L, int cap, int rolling);
+cudaError_t launch_decode_mma(const LayerCfg& L, int B, const void* q_raw, const void* wq,
+                              const void* cache_k, const void* cache_v, const int32_t* len,
+                              int cap, int rolling, const DecodePlan& plan, float* part_ml,
+                              float* part_o, int* status, cudaStream_t s);
+
 // g4attn_decode with the split-KV partials in the library's fixed device
 // array instead of a workspace; returns a g4attn_status code.
 int launch_decode_noalloc(const LayerCfg& L, int B, const void* q_raw, const void* wq,
                           const void* cache_k, const void* cache_v, const int32_t* len, int cap,
                           int rolling, void* out, int* status, cudaStream_t s);
+
+// Tensor map of a bf16 tensor with a 128-byte-swizzled box (dims[0]
+// contiguous, strides in bytes for dims 1..rank-1); false on failure.
+}  // namespace g4
+struct CUtensorMap_st;
+namespace g4 {
+bool make_bf16_map(CUtensorMap_st* m, const void* ptr, int rank, const uint64_t* dims,
+                   const uint64_t* strides_bytes, const uint32_t* box);
 
 // Device status word of the current device (nullptr if it cannot be found).
 int* status_ptr();

@@ -174,3 +174,20 @@ def test_full_size_decode_step_sampled():
     check(x_out[seqs, 0], oracle_decode(X, sub(x_tok), g_k, g_v, n_max, False, lens[seqs],
                                         src_tok=sub(g_tok), src_layer=Gl), torch.bfloat16,
           "kv-shared")
+
+
+def test_long_chunks_repeated():
+    """Caches longer than 4096 positions are split into 2048-key chunks
+    (128 tiles per CTA, many laps of the K/V ring); run several times."""
+    L = W.global_(16, 2, 512)
+    lens = [4097, 6000, 8190, 5000, 7777, 4500, 8100, 6543]
+    tok, cache = make_layer_state(L, len(lens), 8192, False, lens, seed=21)
+    ck, cv = cache.k.cpu(), cache.v.cpu()
+    d = desc_of(L, torch.bfloat16)
+    G.g4attn_cache_append(d, cache, tok["k_raw"], None, tok["k_norm_w"])
+    ref = oracle_decode(L, tok, ck, cv, 8192, False, lens)
+    for _ in range(3):
+        out = G.g4attn_decode(d, cache, tok["q_raw"], tok["q_norm_w"])
+        torch.cuda.synchronize()
+        assert G.g4attn_get_device_status() == G.G4ATTN_OK
+        check(out[:, 0], ref, torch.bfloat16, "long chunks")
