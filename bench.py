@@ -95,6 +95,32 @@ def decode_bytes(L: W.LayerShape, lens, es=2) -> float:
 # ---------------------------------------------------------------------------
 # environment
 
+def profiled_traffic(profile: str, workload: str, bench_workload: str):
+    """DRAM bytes per launch of a kernel from a committed ncu summary, or None
+    if the summary is for another workload or the kernel source has changed
+    since the counters were taken (its sha256 is recorded in the summary)."""
+    if workload != bench_workload:
+        return None
+    path = os.path.join(ROOT, "profiles", profile)
+    if not os.path.exists(path):
+        return None
+    import hashlib
+    fields = {}
+    for line in open(path):
+        if line.startswith(("kernel source:", "source_sha256:")):
+            k, v = line.split(":", 1)
+            fields[k] = v.strip()
+        elif line.startswith("| traffic_bytes_per_launch |"):
+            fields["traffic"] = line.split("|")[2].strip()
+    src = os.path.join(ROOT, fields.get("kernel source:", "").strip() or fields.get("kernel source", ""))
+    if "traffic" not in fields or not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != fields.get("source_sha256"):
+            return None
+    return float(fields["traffic"])
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -216,6 +242,8 @@ def made_events(n):
 
 def bench_prefill(args, dist: Dist, pk: dict):
     w = W.PREFILL_WORKLOADS[args.workload]
+    if args.seq_len:  # a shorter prompt of the same layer (profiling runs)
+        w = W.scaled_down(w, T=args.seq_len)
     dev = torch.device("cuda", dist.local)
     inp = W.prefill_inputs(w, dev, seed=dist.rank)
     d = desc_of(w.layer)
@@ -234,6 +262,19 @@ def bench_prefill(args, dist: Dist, pk: dict):
         step()
     K = args.steps
     s0, s1, a0, a1 = (made_events(K) for _ in range(4))
+    # One step as a CUDA graph (the library's launches of one g4attn_prefill
+    # call), replayed K times: no host launch gaps inside the timed steps.
+    graph = None
+    if not args.no_graph:
+        torch.cuda.synchronize()
+        n0 = G.g4attn_launch_count()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            G.g4attn_prefill(d, inp["q_raw"], inp["k_raw"], inp["v_raw"], inp["q_norm_w"],
+                             inp["k_norm_w"], inp["image_block_ids"], out=out, workspace=ws)
+        per_step_launches = G.g4attn_launch_count() - n0
+        for _ in range(args.warmup):
+            graph.replay()
     torch.cuda.synchronize()
     dist.barrier()
     launches0 = G.g4attn_launch_count()
@@ -242,14 +283,24 @@ def bench_prefill(args, dist: Dist, pk: dict):
         dist.barrier()
         for i in range(K):
             flush.fill_(i & 0xFF)
-            G.g4attn_time_next_attention(a0[i], a1[i])
             s0[i].record(stream)
-            step()
+            if graph is None:
+                step()
+            else:
+                graph.replay()
             s1[i].record(stream)
         torch.cuda.synchronize()
         dist.barrier()
-    launches = G.g4attn_launch_count() - launches0
+    launches = (G.g4attn_launch_count() - launches0 if graph is None
+                else per_step_launches * K)
     step_ms = [s0[i].elapsed_time(s1[i]) for i in range(K)]
+    # the dominant kernel alone: the library records a0/a1 around its
+    # attention launch on the call's stream (eager calls, same L2 flushing)
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        G.g4attn_time_next_attention(a0[i], a1[i])
+        step()
+    torch.cuda.synchronize()
     attn_ms = [a0[i].elapsed_time(a1[i]) for i in range(K)]
     total_ms = dist.max(sum(step_ms))
     value = dist.world * flops * K / (total_ms * 1e-3) / 1e12
@@ -264,9 +315,11 @@ def bench_prefill(args, dist: Dist, pk: dict):
         value=value, ms_per_step=total_ms / K, flops=flops, launches=launches,
         clocks=clk.summary(),
         roofline={"bound": "tensor", "kernel": "attention (g4attn_prefill)", "achieved": achieved,
-                  "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                  "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                  "traffic": profiled_traffic("attn_sm100_e2b_sliding.md", w.name,
+                                              W.E2B_SLIDING.name),
                   "algorithmic_per_launch": flops, "avg_launch_ms": attn_avg},
-        e2e=None, inputs=inp, workload=w)
+        e2e=None, inputs=inp, workload=w, graph=graph is not None)
     if args.no_e2e:
         return res
 
@@ -483,11 +536,14 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=W.E2B_SLIDING.name,
                     choices=[n for n in W.PREFILL_WORKLOADS if not n.startswith("tiny")])
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override the prefill workload's prompt length (profiling runs)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="sequences of the decode step (default: the workload's 64)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager calls, not a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -535,6 +591,8 @@ def main(argv=None):
                        "head_dim": w.layer.head_dim, "window": w.layer.window,
                        "parallelism": f"replicas{dist.world}",
                        "l2": "flushed (256 MiB write) before every timed prefill step",
+                       "step": "one g4attn_prefill call replayed as a CUDA graph" if pre["graph"]
+                               else "one g4attn_prefill call (eager)",
                        "unmasked_gflop_per_step": pre["flops"] / 1e9},
             "roofline": roof, "cpu_baseline": cpu, "e2e": pre["e2e"],
             "gpu_launches": pre["launches"], "clocks": pre["clocks"], "decode": dec}
