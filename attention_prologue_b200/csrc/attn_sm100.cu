@@ -1,5 +1,5 @@
 // Prefill attention on the 5th-generation tensor cores (tcgen05, TMEM, TMA)
-// for head_dim 64 / 128 / 256: the sliding-window layers with image blocks
+// for head_dim 64 / 128 / 256 (512 lives in attn_pair.cu): the sliding-window layers with image blocks
 // ("Gemma 4" overview blog, "Sliding-window attention"; "Gemma 4" Keras docs,
 // "What changed": bidirectional image blocks on sliding layers) and causal
 // global layers ("Global attention layers").
@@ -32,6 +32,7 @@
 
 #include "common.cuh"
 #include "g4attn.h"
+#include "g4attn_internal.h"
 #include "sm100.cuh"
 
 namespace g4 {
@@ -46,18 +47,16 @@ constexpr int kStagesV = 2;
 constexpr int kThreads = 256;
 constexpr int kSoftmaxWarp0 = 4;
 
-// D: head dims this CTA handles (the whole head, or half of it when kPair).
-template <int D, bool kPair>
+template <int D>
 struct Layout {
-  static constexpr int kStagesK = kPair ? 2 : 3;          // K is needed one S before V
+  static constexpr int kStagesK = 3;                      // K is needed one S before V
   static constexpr int kChunks = D / 64;                  // 64-element (128-byte) columns
   static constexpr uint32_t kQChunk = BM * 128;           // bytes of one Q chunk
   static constexpr uint32_t kKVChunk = BN * 128;          // bytes of one K or V chunk
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kK = kQ + kChunks * kQChunk;
   static constexpr uint32_t kV = kK + kStagesK * kChunks * kKVChunk;
-  static constexpr uint32_t kX = kV + kStagesV * kChunks * kKVChunk;  // partial-S inbox
-  static constexpr uint32_t kBars = kX + (kPair ? BM * BN * 4 : 0);
+  static constexpr uint32_t kBars = kV + kStagesV * kChunks * kKVChunk;
   static constexpr uint32_t kAlloc = kBars + 256;  // + barriers and scalars
   static_assert(kAlloc <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
   static constexpr uint32_t kTmemCols = (128 + D) <= 256 ? 256 : 512;
@@ -76,9 +75,7 @@ struct Bars {  // offsets (in 8-byte words) of the mbarriers from Layout::kBars
     o_done = 15,   // one phase per PV (rescale waits: always within one phase)
     drain = 16,
     o_last = 17,   // single phase: the last PV (the epilogue may lag several PVs)
-    rx_full = 18,  // pair: the peer's partial S of this tile is in the inbox
-    tx_ok = 19,    // pair: the peer has read what this CTA sent it
-    count = 20
+    count = 18
   };
 };
 
@@ -90,14 +87,14 @@ struct Scalars {  // ints after the barriers
 
 }  // namespace
 
-template <int D, bool kPair>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, RowIntervals rows,
                       __nv_bfloat16* __restrict__ out, int T_, int Hq, int Hkv, int layer_type,
                       int window, float scale_log2, int gp_log2, int* status) {
-  using Ly = Layout<D, kPair>;
+  using Ly = Layout<D>;
   constexpr int kStagesK = Ly::kStagesK;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte-swizzle atoms assume a 1024-byte aligned base
@@ -113,11 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = &sc->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // kPair: the two CTAs of a cluster share the rows and split the head dims
-  const uint32_t rank = kPair ? cluster_rank() : 0u;
-  const int dcol0 = (int)rank * D;  // first head dim of this CTA
-  const int n_rt = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
-  const int tile = n_rt - 1 - (kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x);  // latest first
+  const int tile = (int)gridDim.x - 1 - (int)blockIdx.x;  // latest rows first
   const int b = blockIdx.z;
   const int h0 = blockIdx.y << gp_log2;    // first query head of the tile
   const int p0 = tile * (BM >> gp_log2);   // first position of the tile
@@ -138,8 +131,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(Bars::o_done), 1);
     mbar_init(bar(Bars::drain), 1);
     mbar_init(bar(Bars::o_last), 1);
-    mbar_init(bar(Bars::rx_full), 4 * 32);
-    mbar_init(bar(Bars::tx_ok), 4 * 32);
     sc->abort = 0;
     sc->klo = 0x7fffffff;
     sc->khi = -1;
@@ -179,7 +170,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if constexpr (kPair) cluster_sync_all();  // the peer's barriers exist before any remote use
   const uint32_t tmem = sc->tmem_base;
   const int kt0 = sc->klo / BN;
   const int n_tiles = sc->khi / BN - kt0 + 1;
@@ -198,8 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (is_k) {
         mbar_arrive_expect_tx(bar(Bars::q_full), BM * D * 2);
         for (int c = 0; c < Ly::kChunks; ++c)
-          tma_load_4d(base + Ly::kQ + c * Ly::kQChunk, &tm_q, bar(Bars::q_full), dcol0 + c * 64,
-                      h0, p0, b);
+          tma_load_4d(base + Ly::kQ + c * Ly::kQChunk, &tm_q, bar(Bars::q_full), c * 64, h0, p0,
+                      b);
       }
       int issued = 0;
       for (int j = 0; j < n_tiles; ++j) {
@@ -208,8 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int key0 = (kt0 + j) * BN;
         mbar_arrive_expect_tx(bar(full + s), BN * D * 2);
         for (int c = 0; c < Ly::kChunks; ++c)
-          tma_load_3d(ring + (s * Ly::kChunks + c) * Ly::kKVChunk, tm, bar(full + s),
-                      dcol0 + c * 64, key0, b * Hkv + kvh);
+          tma_load_3d(ring + (s * Ly::kChunks + c) * Ly::kKVChunk, tm, bar(full + s), c * 64,
+                      key0, b * Hkv + kvh);
         issued = j + 1;
       }
       if (*abort) {  // let the copies already issued land before the CTA exits
@@ -287,36 +277,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tmem + lane_off + (j & 1) * BN, sr);
       tmem_ld32(tmem + lane_off + (j & 1) * BN + 32, sr + 32);
       tmem_wait_ld();
-      if constexpr (kPair) {
-        // S = this CTA's partial (its half of the head dims) + the peer's.
-        // Send ours into the peer's inbox row r (16-byte slot q at q ^ (r & 15)),
-        // then read the peer's from our inbox; both CTAs add the same two fp32
-        // values, so both softmaxes see bit-identical scores.
-        if (j > 0) {  // the peer has read the previous tile's partial
-          ok = __all_sync(0xffffffffu, mbar_wait_cluster(bar(Bars::tx_ok), (j - 1) & 1, abort));
-          if (!ok) break;
-        }
-        const uint32_t inbox_row = base + Ly::kX + r * (BN * 4);
-#pragma unroll
-        for (int q = 0; q < BN / 4; ++q) {
-          const uint32_t dst = map_peer(inbox_row + ((q ^ (r & 15)) << 4), rank ^ 1u);
-          st_cluster_v4(dst, __uint_as_float(sr[4 * q]), __uint_as_float(sr[4 * q + 1]),
-                        __uint_as_float(sr[4 * q + 2]), __uint_as_float(sr[4 * q + 3]));
-        }
-        mbar_arrive_remote(map_peer(bar(Bars::rx_full), rank ^ 1u));
-        ok = __all_sync(0xffffffffu, mbar_wait_cluster(bar(Bars::rx_full), j & 1, abort));
-        if (!ok) break;
-        const float4* inbox = reinterpret_cast<const float4*>(gbase + Ly::kX + r * (BN * 4));
-#pragma unroll
-        for (int q = 0; q < BN / 4; ++q) {
-          const float4 v = inbox[q ^ (r & 15)];
-          sr[4 * q] = __float_as_uint(__uint_as_float(sr[4 * q]) + v.x);
-          sr[4 * q + 1] = __float_as_uint(__uint_as_float(sr[4 * q + 1]) + v.y);
-          sr[4 * q + 2] = __float_as_uint(__uint_as_float(sr[4 * q + 2]) + v.z);
-          sr[4 * q + 3] = __float_as_uint(__uint_as_float(sr[4 * q + 3]) + v.w);
-        }
-        mbar_arrive_remote(map_peer(bar(Bars::tx_ok), rank ^ 1u));
-      }
       const int key0 = (kt0 + j) * BN;
       float x[BN];
       float mt = -INFINITY;
@@ -384,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = out + (((long)b * T_ + i) * Hq + hrow) * (kPair ? 2 * D : D) + dcol0;
+      __nv_bfloat16* dst = out + (((long)b * T_ + i) * Hq + hrow) * D;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
@@ -407,12 +367,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  if constexpr (kPair) {
-    // the peer's last access to this CTA is its read receipt for the last
-    // tile: wait for it (bounded) before the CTA's shared memory goes away
-    if (warp >= kSoftmaxWarp0 && n_tiles > 0)
-      mbar_wait_cluster(bar(Bars::tx_ok), (n_tiles - 1) & 1, nullptr);
-  }
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && *abort) record_status(status, G4ATTN_EDEVICE);
@@ -474,22 +428,12 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
   return make_bf16_map(m, ptr, rank, dims, strides_bytes, box);
 }
 
-// Query heads packed per tile: the largest power of two <= 8 dividing
-// Hq / Hkv (every head of a tile reads the same KV head).
-int pack_log2(const LayerCfg& L) {
-  const int g = L.Hq / L.Hkv;
-  int lg = 0;
-  while (lg < 3 && g % (2 << lg) == 0) ++lg;
-  return lg;
-}
-
-template <int D, bool kPair>
+template <int D>
 cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
                       RowIntervals rows, void* out, int* status, cudaStream_t s) {
-  static_assert(!kPair || D == 256, "pairs split head_dim 512");
   CUtensorMap tq, tk, tv;
-  const int gp_log2 = pack_log2(L);
-  constexpr int DF = kPair ? 2 * D : D;  // full head dim
+  const int gp_log2 = gqa_pack_log2(L.Hq, L.Hkv);
+  constexpr int DF = D;
   const uint64_t es = 2;
   {  // q_hat [B, T, Hq, D]: dims (D, Hq, T, B)
     const uint64_t dims[4] = {(uint64_t)DF, (uint64_t)L.Hq, (uint64_t)T, (uint64_t)B};
@@ -504,27 +448,18 @@ cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc 
     if (!make_map(&tk, kv.k, 3, dims, str, box)) return cudaErrorInvalidValue;
     if (!make_map(&tv, kv.v, 3, dims, str, box)) return cudaErrorInvalidValue;
   }
-  using Ly = Layout<D, kPair>;
-  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D, kPair>,
+  using Ly = Layout<D>;
+  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
   if (e != cudaSuccess) return e;
   const float scale_log2 = L.scale * 1.4426950408889634f;
   const int bp = BM >> gp_log2;  // positions per tile
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((T + bp - 1) / bp * (kPair ? 2 : 1), L.Hq >> gp_log2, B);
+  cfg.gridDim = dim3((T + bp - 1) / bp, L.Hq >> gp_log2, B);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = Ly::kAlloc;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  if (kPair) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
-  e = cudaLaunchKernelEx(&cfg, attn_sm100_kernel<D, kPair>, tq, tk, tv, rows,
+  e = cudaLaunchKernelEx(&cfg, attn_sm100_kernel<D>, tq, tk, tv, rows,
                          static_cast<__nv_bfloat16*>(out), T, L.Hq, L.Hkv, L.layer_type, L.window,
                          scale_log2, gp_log2, status);
   if (e != cudaSuccess) return e;
@@ -541,10 +476,10 @@ bool attention_sm100_supported(const LayerCfg& L) {
 cudaError_t launch_attention_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
                                    RowIntervals rows, void* out, int* status, cudaStream_t s) {
   switch (L.d) {
-    case 64: return run_sm100<64, false>(L, B, T, q_hat, kv, rows, out, status, s);
-    case 128: return run_sm100<128, false>(L, B, T, q_hat, kv, rows, out, status, s);
-    case 256: return run_sm100<256, false>(L, B, T, q_hat, kv, rows, out, status, s);
-    case 512: return run_sm100<256, true>(L, B, T, q_hat, kv, rows, out, status, s);
+    case 64: return run_sm100<64>(L, B, T, q_hat, kv, rows, out, status, s);
+    case 128: return run_sm100<128>(L, B, T, q_hat, kv, rows, out, status, s);
+    case 256: return run_sm100<256>(L, B, T, q_hat, kv, rows, out, status, s);
+    case 512: return launch_attention_pair(L, B, T, q_hat, kv, rows, out, status, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -61,10 +61,23 @@ cudaError_t launch_block_intervals(const LayerCfg& L, int B, int T, const int32_
                                    int32_t* lo, int32_t* hi, cudaStream_t s);
 cudaError_t launch_attention_simt(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
                                   RowIntervals rows, void* out, cudaStream_t s);
-// tcgen05 prefill attention (bf16, head_dim 64/128/256); q_hat [B, T, Hq, d].
+// tcgen05 prefill attention (bf16, head_dim 64/128/256/512); q_hat [B, T, Hq, d].
 bool attention_sm100_supported(const LayerCfg& L);
 cudaError_t launch_attention_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
                                    RowIntervals rows, void* out, int* status, cudaStream_t s);
+// head_dim 512 on 2-CTA clusters (called by launch_attention_sm100).
+cudaError_t launch_attention_pair(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
+                                  RowIntervals rows, void* out, int* status, cudaStream_t s);
+
+// Query heads packed into one 128-row prefill tile, as a power of two: the
+// largest 2^g <= 8 dividing Hq / Hkv (every head of a tile reads the same KV
+// head, so a tile spans 128 / 2^g positions).
+inline int gqa_pack_log2(int Hq, int Hkv) {
+  const int g = Hq / Hkv;
+  int lg = 0;
+  while (lg < 3 && g % (2 << lg) == 0) ++lg;
+  return lg;
+}
 cudaError_t launch_append(const LayerCfg& L, int B, const void* k_raw, const void* v_raw,
                           const void* wk, void* cache_k, void* cache_v, int32_t* len, int cap,
                           int rolling, int* status, cudaStream_t s);

@@ -49,6 +49,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test: has the phase of parity `parity` completed?
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase of parity `parity` to complete.  Gives up after
 // `limit_ns` of wall time (or as soon as *abort is set by another thread of
 // the CTA), sets *abort and returns false: no wait in these kernels can spin
@@ -92,18 +105,23 @@ __device__ __forceinline__ void cluster_sync_all() {
                ::: "memory");
 }
 
-// Arrive on an mbarrier of another CTA of the cluster, releasing this
-// thread's earlier shared-memory writes (local or remote) at cluster scope.
+// Arrive on an mbarrier of another CTA of the cluster (default semantics:
+// release at CTA scope).  Used as a "buffer free" signal to a CTA that
+// writes into this CTA's shared memory only after observing it.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t cluster_addr, float a, float b, float c,
-                                              float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(a),
-               "f"(b), "f"(c), "f"(d)
-               : "memory");
+// Store 16 bytes into shared memory of another CTA of the cluster and
+// signal their arrival (complete_tx of 16 bytes) on `cluster_bar`, an
+// mbarrier in that same CTA.  No fence: the receiver observes the data
+// through the barrier phase that the bytes complete.
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t cluster_bar,
+                                            uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(cluster_addr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_bar)
+      : "memory");
 }
 
 // try_wait with cluster-scope acquire (sees the peer's released writes).

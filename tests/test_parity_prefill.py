@@ -69,8 +69,9 @@ def test_short_prompts(T):
     run_case(W.PrefillWorkload(f"g{T}", W.global_(8, 1, 512), 1, T), seed=T)
 
 
-def test_blocks_at_the_edges_and_block_longer_than_window():
-    L = W.sliding(2, 1, 256, 32)
+@pytest.mark.parametrize("hd", [256, 512])
+def test_blocks_at_the_edges_and_block_longer_than_window(hd):
+    L = W.sliding(2, 1, hd, 32)
     w = W.PrefillWorkload("edges", L, 2, 200)
     inp = W.prefill_inputs(w, DEV, 11)
     ids = torch.full((2, 200), -1, dtype=torch.int32)
@@ -153,7 +154,8 @@ def test_full_size_sampled(w, n):
 def test_few_tile_prompts_repeated(T):
     """Prompts of one to four key tiles, run several times: the epilogue must
     wait for the last PV product even when the softmax finishes early."""
-    for L in (W.sliding(8, 1, 256, 512), W.global_(8, 2, 256), W.sliding(4, 2, 128, 64)):
+    for L in (W.sliding(8, 1, 256, 512), W.global_(8, 2, 256), W.sliding(4, 2, 128, 64),
+              W.global_(8, 2, 512)):
         w = W.PrefillWorkload(f"rep{T}", L, 2, T)
         inp = W.prefill_inputs(w, DEV, T)
         ref = oracle_prefill(w, inp)
