@@ -11,14 +11,17 @@
 //               (warp 2), 64 keys each, two-stage rings (128-byte swizzle,
 //               no multicast); a K slot is refilled as soon as S_j is done,
 //               a V slot as soon as PV_j is done
-//   warp 1      owns TMEM; one thread issues the MMAs:
-//                 S_j = Q K_j^T   (M 128, N 64, K = d; A, B K-major in smem)
-//                 O  += P_j V_j   (M 128, N = d, K 64; P from TMEM, V MN-major)
+//   warp 1      owns TMEM; one thread issues S_j = Q K_j^T (M 128, N 64,
+//               K = d; B K-major in smem, A in smem or TMEM) once PV_{j-NS}
+//               is done
+//   warp 3      one thread issues O += P_j V_j (M 128, N = d, K 64; P from
+//               TMEM, V MN-major in smem)
 //   warps 4..7  softmax: thread r owns query row r (TMEM lane r); reads S_j,
 //               masks it with the row's key interval [lo, hi], writes
 //               P_j = exp2(S_j - m) as bf16 into swizzled shared memory, and
 //               at the end normalises O and stores it.
-// TMEM columns: S double buffer at 0 and 64, O at 128 (d columns).
+// TMEM columns: NS S buffers of 64 (NS = 4 for d = 256, else 2), O after
+// them (at 256, resp. 128; d columns).
 // Key tiles outside the union of the 128 rows' intervals are never loaded.
 //
 // The online softmax rescales O lazily: a row keeps the max it exponentiates
@@ -49,33 +52,50 @@ constexpr int kSoftmaxWarp0 = 4;
 
 template <int D>
 struct Layout {
-  static constexpr int kStagesK = 3;                      // K is needed one S before V
+  // d = 256: the first 128 dims of Q live in tensor memory (the QK^T MMA
+  // reads that half of A from TMEM), which takes 32 KB of operand reads per
+  // tile off shared memory and leaves room for four K stages; they are staged
+  // through the V ring at the start.  Three S buffers: S runs up to two tiles
+  // ahead of PV.  Smaller heads: Q in shared memory, two S buffers (two CTAs
+  // per SM fit the tensor memory).
+  static constexpr int kQTmemChunks = D == 256 ? 2 : 0;
+  static constexpr bool kQT = kQTmemChunks > 0;
+  static constexpr int kStagesK = kQT ? 4 : 3;            // K is needed one S before V
   static constexpr int kChunks = D / 64;                  // 64-element (128-byte) columns
   static constexpr uint32_t kQChunk = BM * 128;           // bytes of one Q chunk
   static constexpr uint32_t kKVChunk = BN * 128;          // bytes of one K or V chunk
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kChunks * kQChunk;
+  static constexpr uint32_t kQ = 0;                       // Q chunks kQTmemChunks.. in smem
+  static constexpr uint32_t kK = kQ + (kChunks - kQTmemChunks) * kQChunk;
   static constexpr uint32_t kV = kK + kStagesK * kChunks * kKVChunk;
   static constexpr uint32_t kBars = kV + kStagesV * kChunks * kKVChunk;
   static constexpr uint32_t kAlloc = kBars + 256;  // + barriers and scalars
   static_assert(kAlloc <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
-  static constexpr uint32_t kTmemCols = (128 + D) <= 256 ? 256 : 512;
-  static constexpr uint32_t kColO = 128;
+  static_assert(kQTmemChunks * kQChunk <= kStagesV * kChunks * kKVChunk,
+                "Q staging fits the V ring");
+  static constexpr int kNS = kQT ? 3 : 2;
+  static constexpr uint32_t kColQ = kNS * BN;             // Q (bf16 pairs) when kQT
+  static constexpr uint32_t kColO = kQT ? 256 : kNS * BN;
+  static constexpr uint32_t kTmemCols = (kColO + D) <= 256 ? 256 : 512;
+  static_assert(!kQT || kColQ + kQTmemChunks * 32 <= kColO, "TMEM columns overlap");
 };
 
-struct Bars {  // offsets (in 8-byte words) of the mbarriers from Layout::kBars
+// Offsets (in 8-byte words) of the mbarriers from Layout::kBars.
+template <int NS>
+struct BarsT {
   enum {
     q_full = 0,
-    k_full = 1,    // [3]
-    k_empty = 4,   // [3]
-    v_full = 7,    // [2]
-    v_empty = 9,   // [2]
-    s_full = 11,   // [2]
-    p_full = 13,   // [2]
-    o_done = 15,   // one phase per PV (rescale waits: always within one phase)
-    drain = 16,
-    o_last = 17,   // single phase: the last PV (the epilogue may lag several PVs)
-    count = 18
+    q_tmem = 1,           // Q is in TMEM (the staging area in the V ring is free)
+    k_full = 2,           // [4]
+    k_empty = 6,          // [4]
+    v_full = 10,          // [2]
+    v_empty = 12,         // [2]
+    drain = 14,           // (S issuer)
+    drain2 = 15,          // (PV issuer)
+    o_last = 16,          // single phase: the last PV (the epilogue may lag several PVs)
+    s_full = 17,          // [NS]
+    p_full = s_full + NS,  // [NS]
+    o_done = p_full + NS,  // [NS] PV_j done (one per S buffer: rescale waits stay in one phase)
+    count = o_done + NS
   };
 };
 
@@ -95,7 +115,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                       __nv_bfloat16* __restrict__ out, int T_, int Hq, int Hkv, int layer_type,
                       int window, float scale_log2, int gp_log2, int* status) {
   using Ly = Layout<D>;
+  using Bars = BarsT<Ly::kNS>;
   constexpr int kStagesK = Ly::kStagesK;
+  constexpr int kNS = Ly::kNS;
+  static_assert(8 * Bars::count + 16 <= 256, "barriers and scalars overflow their area");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte-swizzle atoms assume a 1024-byte aligned base
   if (smem_u32(smem_raw) & 1023u) {
@@ -118,18 +141,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(Bars::q_full), 1);
+    mbar_init(bar(Bars::q_tmem), 4 * 32);
     for (int s = 0; s < kStagesK; ++s) {
       mbar_init(bar(Bars::k_full + s), 1);
       mbar_init(bar(Bars::k_empty + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStagesV; ++s) {
       mbar_init(bar(Bars::v_full + s), 1);
       mbar_init(bar(Bars::v_empty + s), 1);
+    }
+    for (int s = 0; s < kNS; ++s) {
       mbar_init(bar(Bars::s_full + s), 1);
       mbar_init(bar(Bars::p_full + s), 4 * 32);
+      mbar_init(bar(Bars::o_done + s), 1);
     }
-    mbar_init(bar(Bars::o_done), 1);
     mbar_init(bar(Bars::drain), 1);
+    mbar_init(bar(Bars::drain2), 1);
     mbar_init(bar(Bars::o_last), 1);
     sc->abort = 0;
     sc->klo = 0x7fffffff;
@@ -185,14 +212,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int full = is_k ? Bars::k_full : Bars::v_full;
       const int empty = is_k ? Bars::k_empty : Bars::v_empty;
       const int nst = is_k ? kStagesK : kStagesV;
-      if (is_k) {
+      int n_load = n_tiles;
+      if (is_k) {  // Q, into the V ring when it is staged for TMEM
         mbar_arrive_expect_tx(bar(Bars::q_full), BM * D * 2);
         for (int c = 0; c < Ly::kChunks; ++c)
-          tma_load_4d(base + Ly::kQ + c * Ly::kQChunk, &tm_q, bar(Bars::q_full), c * 64, h0, p0,
-                      b);
+          tma_load_4d(c < Ly::kQTmemChunks ? base + Ly::kV + c * Ly::kQChunk
+                                           : base + Ly::kQ + (c - Ly::kQTmemChunks) * Ly::kQChunk,
+                      &tm_q, bar(Bars::q_full), c * 64, h0, p0, b);
+      } else if (Ly::kQT && !mbar_wait(bar(Bars::q_tmem), 0, abort)) {
+        n_load = 0;  // the staged Q is still being read
       }
       int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
+      for (int j = 0; j < n_load; ++j) {
         const int s = j % nst;
         if (!mbar_wait(bar(empty + s), ((j / nst) & 1) ^ 1, abort)) break;
         const int key0 = (kt0 + j) * BN;
@@ -208,60 +239,72 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(bar(full + j % nst), (j / nst) & 1, nullptr);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA issuers
+    // Two threads feed the tensor core: warp 1 issues S_j = Q K_j^T, warp 3
+    // issues O += P_j V_j.  The tensor core's issue queue is short and a
+    // tcgen05.mma blocks while it is full, so with a single issuer a ready PV
+    // waited behind the whole next S (~1000 cycles).  A commit tracks only
+    // its own thread's MMAs: S_j, which overwrites the buffer P_{j-NS} lives
+    // in, waits until PV_{j-NS} has completed (o_done), not just been issued.
+    // No progress for 2 s sets the abort flag.
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(BM, BN, 0, 0);
-      constexpr uint32_t idesc_o = idesc_bf16(BM, D, 0, 1);
-      auto issue_pv = [&](int j) {
-        const int s = j % kStagesV;
-        const uint32_t vbase = base + Ly::kV + s * Ly::kChunks * Ly::kKVChunk;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // A = P_j in TMEM: row m in lane m, 16 keys = 8 packed columns per step
-          const uint64_t bd = desc_sw128(vbase + kk * 16 * 128, Ly::kKVChunk, 1024);
-          mma_ts(tmem + Ly::kColO, tmem + (j & 1) * BN + kk * 8, bd, idesc_o,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(bar(Bars::v_empty + s));
-        mma_commit(bar(Bars::o_done));
-      };
-      bool ok = mbar_wait(bar(Bars::q_full), 0, abort);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kStagesK;
-        if (!(ok = mbar_wait(bar(Bars::k_full + s), (j / kStagesK) & 1, abort))) break;
-        tc_fence_after();
-        const uint32_t kbase = base + Ly::kK + s * Ly::kChunks * Ly::kKVChunk;
-#pragma unroll
-        for (int kc = 0; kc < D / 16; ++kc) {
-          const int c = kc >> 2, sub = kc & 3;
-          const uint64_t a = desc_sw128(base + Ly::kQ + c * Ly::kQChunk + sub * 32, 16, 1024);
-          const uint64_t bd = desc_sw128(kbase + c * Ly::kKVChunk + sub * 32, 16, 1024);
-          mma_ss(tmem + (j & 1) * BN, a, bd, idesc_s, kc > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(Bars::s_full + (j & 1)));
-        mma_commit(bar(Bars::k_empty + s));
-        if (j >= 1) {
-          if (!(ok = mbar_wait(bar(Bars::p_full + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort)))
+      bool ok = mbar_wait(bar(Bars::q_full), 0, abort) &&
+                (!Ly::kQT || mbar_wait(bar(Bars::q_tmem), 0, abort));
+      if (ok) tc_fence_after();
+      if (warp == 1) {
+        constexpr uint32_t idesc_s = idesc_bf16(BM, BN, 0, 0);
+        // descriptors: per-MMA ones are constant offsets from these bases
+        const uint64_t dq0 = desc_sw128(base + Ly::kQ, 16, 1024);
+        const uint64_t dk0 = desc_sw128(base + Ly::kK, 16, 1024);
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int s = j % kStagesK;
+          if (j >= kNS && !(ok = mbar_wait(bar(Bars::o_done + (j - kNS) % kNS),
+                                           ((j - kNS) / kNS) & 1, abort)))
             break;
-          if (!(ok = mbar_wait(bar(Bars::v_full + (j - 1) % kStagesV), ((j - 1) / kStagesV) & 1,
-                               abort)))
-            break;
+          if (!(ok = mbar_wait(bar(Bars::k_full + s), (j / kStagesK) & 1, abort))) break;
           tc_fence_after();
-          issue_pv(j - 1);
+          const uint64_t dk = desc_add(dk0, s * Ly::kChunks * Ly::kKVChunk);
+          const uint32_t d = tmem + (j % kNS) * BN;
+#pragma unroll
+          for (int kc = 0; kc < D / 16; ++kc) {
+            const int c = kc >> 2, sub = kc & 3;
+            const uint64_t bd = desc_add(dk, c * Ly::kKVChunk + sub * 32);
+            if (c < Ly::kQTmemChunks) {  // A from TMEM: 16 dims = 8 packed columns per step
+              mma_ts(d, tmem + Ly::kColQ + kc * 8, bd, idesc_s, kc > 0 ? 1u : 0u);
+            } else {
+              mma_ss(d, desc_add(dq0, (c - Ly::kQTmemChunks) * Ly::kQChunk + sub * 32), bd,
+                     idesc_s, kc > 0 ? 1u : 0u);
+            }
+          }
+          mma_commit(bar(Bars::s_full + j % kNS));
+          mma_commit(bar(Bars::k_empty + s));
         }
+      } else {
+        constexpr uint32_t idesc_o = idesc_bf16(BM, D, 0, 1);
+        const uint64_t dv0 = desc_sw128(base + Ly::kV, Ly::kKVChunk, 1024);
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const int s = j % kStagesV;
+          if (!(ok = mbar_wait(bar(Bars::p_full + j % kNS), (j / kNS) & 1, abort))) break;
+          if (!(ok = mbar_wait(bar(Bars::v_full + s), (j / kStagesV) & 1, abort))) break;
+          tc_fence_after();
+          const uint64_t dv = desc_add(dv0, s * Ly::kChunks * Ly::kKVChunk);
+          const uint32_t pa = tmem + (j % kNS) * BN;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // A = P_j in TMEM: row m in lane m, 16 keys = 8 packed columns per step
+            mma_ts(tmem + Ly::kColO, pa + kk * 8, desc_add(dv, kk * 16 * 128), idesc_o,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(bar(Bars::v_empty + s));
+          mma_commit(bar(Bars::o_done + j % kNS));
+        }
+        if (ok && n_tiles > 0) mma_commit(bar(Bars::o_last));
       }
-      if (ok && mbar_wait(bar(Bars::p_full + ((n_tiles - 1) & 1)), ((n_tiles - 1) >> 1) & 1,
-                          abort) &&
-          mbar_wait(bar(Bars::v_full + (n_tiles - 1) % kStagesV),
-                    ((n_tiles - 1) / kStagesV) & 1, abort)) {
-        tc_fence_after();
-        issue_pv(n_tiles - 1);
-        mma_commit(bar(Bars::o_last));
-      }
-      if (*abort) {  // every MMA issued so far completes before TMEM is freed
-        mma_commit(bar(Bars::drain));
-        mbar_wait(bar(Bars::drain), 0, nullptr);
+      if (*abort) {  // this thread's MMAs complete before TMEM is freed
+        const int dr = warp == 1 ? Bars::drain : Bars::drain2;
+        mma_commit(bar(dr));
+        mbar_wait(bar(dr), 0, nullptr);
       }
     }
   } else if (warp >= kSoftmaxWarp0) {
@@ -269,13 +312,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)((warp - kSoftmaxWarp0) * 32) << 16;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::s_full + (j & 1)), (j >> 1) & 1, abort));
+    if constexpr (Ly::kQT) {
+      // row r of the staged half of Q (128-byte swizzle) -> TMEM as bf16 pairs
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::q_full), 0, abort));
+      if (ok) {
+#pragma unroll 1
+        for (int c = 0; c < Ly::kQTmemChunks; ++c) {
+          const uint4* row = reinterpret_cast<const uint4*>(gbase + Ly::kV + c * Ly::kQChunk + r * 128);
+          uint32_t qw[32];
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const uint4 v = row[g ^ (r & 7)];
+            qw[4 * g] = v.x;
+            qw[4 * g + 1] = v.y;
+            qw[4 * g + 2] = v.z;
+            qw[4 * g + 3] = v.w;
+          }
+          tmem_st32(tmem + lane_off + Ly::kColQ + 32 * c, qw);
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();  // the V loads may now overwrite the staging area
+        tc_fence_before();
+        mbar_arrive(bar(Bars::q_tmem));
+      }
+    }
+    for (int j = 0; ok && j < n_tiles; ++j) {
+      const int sb = j % kNS;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::s_full + sb), (j / kNS) & 1, abort));
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[BN];
-      tmem_ld32(tmem + lane_off + (j & 1) * BN, sr);
-      tmem_ld32(tmem + lane_off + (j & 1) * BN + 32, sr + 32);
+      tmem_ld32(tmem + lane_off + sb * BN, sr);
+      tmem_ld32(tmem + lane_off + sb * BN + 32, sr + 32);
       tmem_wait_ld();
       const int key0 = (kt0 + j) * BN;
       float x[BN];
@@ -298,7 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool first = m_used == -INFINITY;
       const bool grow = !first && mt > m_used + 8.f;
       if (__any_sync(0xffffffffu, grow)) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::o_done), (j - 1) & 1, abort));
+        // PV_{j-1} must be done; S_j done implies PV_{j-NS} is, so o_done
+        // of that buffer is at most one phase behind
+        const int pj = j - 1;
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(bar(Bars::o_done + pj % kNS), (pj / kNS) & 1, abort));
         if (!ok) break;
         tc_fence_after();
         const float alpha = grow ? exp2f(m_used - mt) : 1.f;
@@ -332,11 +404,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
         pk[e] = *reinterpret_cast<uint32_t*>(&bb);
       }
-      tmem_st32(tmem + lane_off + (j & 1) * BN, pk);
+      tmem_st32(tmem + lane_off + sb * BN, pk);
       tmem_wait_st();
       l += rs;
       tc_fence_before();
-      mbar_arrive(bar(Bars::p_full + (j & 1)));
+      mbar_arrive(bar(Bars::p_full + sb));
     }
     // ------------------------------------------------------------ epilogue
     if (ok)  // warp-uniform: the tcgen05 loads below are warp-collective
