@@ -77,6 +77,7 @@ struct Layout {
   static constexpr uint32_t kColO = kQT ? 256 : kNS * BN;
   static constexpr uint32_t kTmemCols = (kColO + D) <= 256 ? 256 : 512;
   static_assert(!kQT || kColQ + kQTmemChunks * 32 <= kColO, "TMEM columns overlap");
+  static_assert(kChunks * kQChunk <= kStagesK * kChunks * kKVChunk, "O staging fits the K ring");
 };
 
 // Offsets (in 8-byte words) of the mbarriers from Layout::kBars.
@@ -111,7 +112,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, RowIntervals rows,
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_o, RowIntervals rows,
                       __nv_bfloat16* __restrict__ out, int T_, int Hq, int Hkv, int layer_type,
                       int window, float scale_log2, int gp_log2, int* status) {
   using Ly = Layout<D>;
@@ -167,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_o);
   }
   if (warp == 1) {
     tmem_alloc(base + Ly::kBars + 8 * Bars::count, Ly::kTmemCols);
@@ -413,29 +416,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     if (ok)  // warp-uniform: the tcgen05 loads below are warp-collective
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::o_last), 0, abort));
+    // O / l as bf16 into the (now idle) K ring in the 128-byte-swizzled
+    // layout of the output tile, then four TMA tile stores: each row of a
+    // thread would otherwise go out as 16-byte pieces 512 bytes apart
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* dst = out + (((long)b * T_ + i) * Hq + hrow) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32(tmem + lane_off + Ly::kColO + c0, o);
-        tmem_wait_ld();
-        if (i < T_) {
-          uint32_t pk[16];
+      for (int c = 0; c < Ly::kChunks; ++c) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t o[32];
+          tmem_ld32(tmem + lane_off + Ly::kColO + 64 * c + 32 * h, o);
+          tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             __nv_bfloat162 bb = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
                                                       __uint_as_float(o[2 * e + 1]) * inv);
-            pk[e] = *reinterpret_cast<uint32_t*>(&bb);
+            pk[16 * h + e] = *reinterpret_cast<uint32_t*>(&bb);
           }
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
+        uint4* row = reinterpret_cast<uint4*>(gbase + Ly::kK + c * Ly::kQChunk + r * 128);
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          row[g ^ (r & 7)] = make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
       }
+      fence_proxy_async_smem();
+    }
+    // (ok is uniform over the 128 softmax threads: all rows see the same waits)
+    named_sync(1, 4 * 32);
+    if (ok && r == 0) {
+      for (int c = 0; c < Ly::kChunks; ++c)
+        tma_store_4d(&tm_o, base + Ly::kK + c * Ly::kQChunk, c * 64, h0, p0, b);
+      bulk_commit();
+      bulk_wait_read();
     }
   }
 
@@ -503,7 +518,7 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
 template <int D>
 cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
                       RowIntervals rows, void* out, int* status, cudaStream_t s) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const int gp_log2 = gqa_pack_log2(L.Hq, L.Hkv);
   constexpr int DF = D;
   const uint64_t es = 2;
@@ -512,6 +527,8 @@ cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc 
     const uint64_t str[3] = {DF * es, (uint64_t)L.Hq * DF * es, (uint64_t)T * L.Hq * DF * es};
     const uint32_t box[4] = {64, (uint32_t)(1 << gp_log2), (uint32_t)(BM >> gp_log2), 1};
     if (!make_map(&tq, q_hat, 4, dims, str, box)) return cudaErrorInvalidValue;
+    // out [B, T, Hq, D]: the same geometry (the epilogue stores its tile)
+    if (!make_map(&to, out, 4, dims, str, box)) return cudaErrorInvalidValue;
   }
   {  // K, V [B * Hkv, cap, D]; only positions < T exist (rows past T read as 0)
     const uint64_t dims[3] = {(uint64_t)DF, (uint64_t)T, (uint64_t)B * L.Hkv};
@@ -531,7 +548,7 @@ cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc 
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = Ly::kAlloc;
   cfg.stream = s;
-  e = cudaLaunchKernelEx(&cfg, attn_sm100_kernel<D>, tq, tk, tv, rows,
+  e = cudaLaunchKernelEx(&cfg, attn_sm100_kernel<D>, tq, tk, tv, to, rows,
                          static_cast<__nv_bfloat16*>(out), T, L.Hq, L.Hkv, L.layer_type, L.window,
                          scale_log2, gp_log2, status);
   if (e != cudaSuccess) return e;
