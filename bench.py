@@ -95,12 +95,11 @@ def decode_bytes(L: W.LayerShape, lens, es=2) -> float:
 # ---------------------------------------------------------------------------
 # environment
 
-def profiled_traffic(profile: str, workload: str, bench_workload: str):
-    """DRAM bytes per launch of a kernel from a committed ncu summary, or None
-    if the summary is for another workload or the kernel source has changed
-    since the counters were taken (its sha256 is recorded in the summary)."""
-    if workload != bench_workload:
-        return None
+def profile_field(profile: str, row: str):
+    """A number from a committed ncu summary under profiles/ (the table row
+    `| row | value |`), or None if the summary or row is missing or the
+    kernel source has changed since the counters were taken (the summary
+    records the source's sha256)."""
     path = os.path.join(ROOT, "profiles", profile)
     if not os.path.exists(path):
         return None
@@ -110,15 +109,22 @@ def profiled_traffic(profile: str, workload: str, bench_workload: str):
         if line.startswith(("kernel source:", "source_sha256:")):
             k, v = line.split(":", 1)
             fields[k] = v.strip()
-        elif line.startswith("| traffic_bytes_per_launch |"):
-            fields["traffic"] = line.split("|")[2].strip()
-    src = os.path.join(ROOT, fields.get("kernel source:", "").strip() or fields.get("kernel source", ""))
-    if "traffic" not in fields or not os.path.exists(src):
+        elif line.startswith(f"| {row} |"):
+            fields["value"] = line.split("|")[2].strip()
+    src = os.path.join(ROOT, fields.get("kernel source", ""))
+    if "value" not in fields or not os.path.isfile(src):
         return None
     with open(src, "rb") as f:
         if hashlib.sha256(f.read()).hexdigest() != fields.get("source_sha256"):
             return None
-    return float(fields["traffic"])
+    return float(fields["value"])
+
+
+def profiled_traffic(profile: str, workload: str, bench_workload: str):
+    """DRAM bytes per launch of a kernel captured on this very workload."""
+    if workload != bench_workload:
+        return None
+    return profile_field(profile, "traffic_bytes_per_launch")
 
 
 def peaks():
@@ -425,6 +431,10 @@ def bench_decode(args, dist: Dist, pk: dict):
     g_split_bytes = decode_bytes(Gl, lens)
     peak = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     achieved = g_split_bytes / (g_ms * 1e-3) / 1e9
+    # DRAM traffic from a smaller capture of the same kernel, scaled by the
+    # bytes it streams (each cached byte is read once; the partials scale too)
+    ratio = profile_field("decode_mma_26b_a4b_global_b4.md", "traffic_per_algorithmic_byte")
+    traffic = None if ratio is None else ratio * g_split_bytes
     res = {"metric": "decode KV-cache GB/s", "value": dist.world * nbytes * K / (total_ms * 1e-3) / 1e9,
            "unit": "GB/s", "ms_per_step": total_ms / K, "bytes_per_step": nbytes,
            "workload": w.name if w.batch == 64 else f"{w.name}-b{w.batch}", "batch": w.batch, "len_range": [w.len_lo, w.len_hi],
@@ -433,7 +443,7 @@ def bench_decode(args, dist: Dist, pk: dict):
            "roofline": {"bound": "hbm", "kernel": "decode split-KV (global layer)",
                         "achieved": achieved, "peak": peak, "unit": "GB/s",
                         "frac": achieved / peak, "frac_of_8000": achieved / 8000.0,
-                        "traffic": None, "algorithmic_per_launch": g_split_bytes,
+                        "traffic": traffic, "algorithmic_per_launch": g_split_bytes,
                         "avg_launch_ms": g_ms},
            "gpu_launches": launches, "clocks": clk.summary()}
     del g_cache, s_cache
