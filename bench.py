@@ -200,17 +200,28 @@ def visible_index(local_rank: int) -> int:
 
 
 class Dist:
-    def __init__(self):
+    """One process per GPU (RANK / WORLD_SIZE / LOCAL_RANK / MASTER_* from the
+    launcher). NCCL on GPUs; gloo with CPU tensors when asked (the host-logic
+    tests run two CPU ranks). Collectives carry only timings."""
+
+    def __init__(self, backend: str | None = None, timeout_s: float = 120.0):
         self.world = int(os.environ.get("WORLD_SIZE", "1"))
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.device = "cpu"
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            torch.cuda.set_device(self.local)
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                    device_id=torch.device("cuda", self.local))
+            backend = backend or "nccl"
+            timeout = datetime.timedelta(seconds=timeout_s)
+            if backend == "nccl":
+                torch.cuda.set_device(self.local)
+                self.device = "cuda"
+                dist.init_process_group("nccl", timeout=timeout,
+                                        device_id=torch.device("cuda", self.local))
+            else:
+                dist.init_process_group(backend, timeout=timeout)
             self.pg = dist
 
     def barrier(self):
@@ -220,13 +231,19 @@ class Dist:
     def max(self, x: float) -> float:
         if not self.pg:
             return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
 
     def close(self):
         if self.pg:
             self.pg.destroy_process_group()
+
+
+def job_rate(world: int, units_per_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the units every rank processed (weak scaling:
+    the same per rank) over the slowest rank's time."""
+    return world * units_per_step * steps / (max_ms * 1e-3)
 
 
 def desc_of(L: W.LayerShape, dtype=torch.bfloat16) -> G.LayerDesc:
@@ -309,7 +326,7 @@ def bench_prefill(args, dist: Dist, pk: dict):
     torch.cuda.synchronize()
     attn_ms = [a0[i].elapsed_time(a1[i]) for i in range(K)]
     total_ms = dist.max(sum(step_ms))
-    value = dist.world * flops * K / (total_ms * 1e-3) / 1e12
+    value = job_rate(dist.world, flops, K, total_ms) / 1e12
     attn_avg = statistics.mean(attn_ms)
     achieved = flops / (attn_avg * 1e-3) / 1e12
     status = G.g4attn_get_device_status()
@@ -357,7 +374,7 @@ def bench_prefill(args, dist: Dist, pk: dict):
         e1[i].record(stream)
     torch.cuda.synchronize()
     e2e_ms = dist.max(sum(e0[i].elapsed_time(e1[i]) for i in range(K)))
-    e2e_value = dist.world * flops * K / (e2e_ms * 1e-3) / 1e12
+    e2e_value = job_rate(dist.world, flops, K, e2e_ms) / 1e12
     res["e2e"] = {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                   "d2h_bytes_per_step": d2h}
     del flush, ws
@@ -435,7 +452,7 @@ def bench_decode(args, dist: Dist, pk: dict):
     # bytes it streams (each cached byte is read once; the partials scale too)
     ratio = profile_field("decode_mma_26b_a4b_global_b4.md", "traffic_per_algorithmic_byte")
     traffic = None if ratio is None else ratio * g_split_bytes
-    res = {"metric": "decode KV-cache GB/s", "value": dist.world * nbytes * K / (total_ms * 1e-3) / 1e9,
+    res = {"metric": "decode KV-cache GB/s", "value": job_rate(dist.world, nbytes, K, total_ms) / 1e9,
            "unit": "GB/s", "ms_per_step": total_ms / K, "bytes_per_step": nbytes,
            "workload": w.name if w.batch == 64 else f"{w.name}-b{w.batch}", "batch": w.batch, "len_range": [w.len_lo, w.len_hi],
            "layers": ["sliding 16/8 d256 w1024 rolling 1024", "global K=V 16/2 d512",
