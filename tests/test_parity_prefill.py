@@ -161,3 +161,19 @@ def test_few_tile_prompts_repeated(T):
         ref = oracle_prefill(w, inp)
         for _ in range(4):
             check(gpu_prefill(w, inp), ref, w.dtype, f"{w.name} d{L.head_dim}")
+
+
+@pytest.mark.parametrize("shape", ["sliding-d256", "global-d128", "short-many"])
+def test_many_work_tiles_per_cta(shape):
+    """More work tiles than SMs: each persistent CTA runs several tiles in a
+    row (barrier phases, Q replacement and the overlapped epilogue carry
+    across tiles), with key ranges of different lengths."""
+    if shape == "sliding-d256":
+        w = W.PrefillWorkload("many-s", W.sliding(8, 1, 256, 128), 2, 4096)
+    elif shape == "global-d128":
+        w = W.PrefillWorkload("many-g", W.global_(8, 4, 128, k_eq_v=False), 1, 4096)
+    else:  # one key tile per work tile, many work tiles
+        w = W.PrefillWorkload("many-short", W.sliding(16, 2, 256, 64), 40, 63)
+    rows = sample_rows(w.T, 24) if w.T > 1000 else None
+    for _ in range(2):
+        run_case(w, seed=17, rows=rows)
