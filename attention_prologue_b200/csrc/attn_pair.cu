@@ -40,7 +40,8 @@
 //                  O   += P_j V_j   (M 128, N 256, K 64; P from TMEM)
 //                with S up to two tiles ahead of PV (three S buffers)
 //   warps 8..11  senders: own partial of S_j -> fp16 -> the peer's inbox
-//   warps 4..7   softmax: copy the TMEM half of Q in at the start; then per
+//   warps 4..7   softmax (lazy rescale when a row max grows by more than
+//                2^16): copy the TMEM half of Q in at the start; then per
 //                tile the own partial of S_j + the peer's,
 //                mask, lazy O rescale, P_j as bf16 into TMEM over S_j; at the
 //                end normalise and store O
@@ -461,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const bool first = m_used == -INFINITY;
-      const bool grow = !first && mt > m_used + 8.f;
+      const bool grow = !first && mt > m_used + 16.f;
       if (__any_sync(0xffffffffu, grow)) {
         // PV_{j-1} must be done; S_j done implies PV_{j-kNS} is, so o_done
         // of that buffer is at most one phase behind

@@ -35,7 +35,12 @@
 // The tensor core's issue queue is short and a tcgen05.mma blocks while it
 // is full; two issuing threads keep a ready PV from waiting behind an S.
 // The online softmax rescales O lazily: a row keeps the max it exponentiates
-// against until a tile raises it by more than 8 (log2 units), so P < 2^8.
+// against until a tile raises it by more than 16 (log2 units), so P < 2^16
+// (exact in bf16 up to its relative rounding; O and l stay far inside fp32).
+// A rescale waits for the previous PV, and the first PV of a tile waits for
+// the previous tile's O to be read out, so rescales must stay rare: with a
+// threshold of 8 the rows whose first key tile was mostly masked rescaled at
+// the second tile and stalled every tile boundary.
 //
 // Every mbarrier wait is bounded (sm100.cuh); on a timeout the CTA records
 // G4ATTN_EDEVICE, drains its in-flight copies and MMAs, frees TMEM and exits.
@@ -388,9 +393,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         mt *= scale_log2;  // scale > 0: the max of the scaled scores
-        // lazy rescale: only when the row max grows by more than 2^8
+        // lazy rescale: only when the row max grows by more than 2^16
         const bool first = m_used == -INFINITY;
-        const bool grow = !first && mt > m_used + 8.f;
+        const bool grow = !first && mt > m_used + 16.f;
         if (__any_sync(0xffffffffu, grow)) {
           // PV of the previous key tile must be done (j >= 1 here); S_g done
           // implies PV_{g-NS} is, so o_done of that buffer is one phase behind
@@ -520,10 +525,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int i = prev.p0 + (r >> gp_log2);
         if (i < T_) {
           const int hrow = prev.h0 + (r & ((1 << gp_log2) - 1));
-          uint4* dst = reinterpret_cast<uint4*>(out + (((long)prev.b * T_ + i) * Hq + hrow) * D);
+          // 32-byte stores: each writes a whole sector (the rows of a warp lie
+          // 512 bytes or more apart, so 16-byte stores would half-fill them)
+          uint32_t* dst = reinterpret_cast<uint32_t*>(out + (((long)prev.b * T_ + i) * Hq + hrow) * D);
 #pragma unroll
-          for (int e = 0; e < D / 8; ++e)
-            dst[e] = make_uint4(ob[4 * e], ob[4 * e + 1], ob[4 * e + 2], ob[4 * e + 3]);
+          for (int e = 0; e < D / 16; ++e) st_global_v8(dst + 8 * e, ob + 8 * e);
         }
       }
       if (!has) break;
