@@ -116,7 +116,9 @@ __device__ __forceinline__ void rope_sincos(long pos, double inv_freq, float* s,
   double a = (double)pos * inv_freq;
   double n = rint(a * (1.0 / two_pi));
   double r = fma(-n, two_pi, a);
-  sincosf((float)r, s, c);
+  // |r| <= pi: the hardware approximation's absolute error there (~4e-7) is
+  // far below the fp32 and bf16 tolerances
+  __sincosf((float)r, s, c);
 }
 
 // Prologue of one head vector by one warp:
@@ -168,19 +170,21 @@ __device__ __forceinline__ void prologue_vec(const T* __restrict__ src, const T*
 }
 
 // RoPE factors of one token for the pairs a lane holds (k = lane*E + e,
-// E = D/64): rot[e] = 0 marks a pass-through pair.
+// E = D/64): rot[e] = 0 marks a pass-through pair.  inv_freq: the layer's
+// frequencies in shared memory (a per-lane index into the kernel's parameter
+// space would serialise the warp's 32 reads).
 template <int D>
-__device__ __forceinline__ void rope_factors(long pos, const RopeParams& rope, float* c, float* s,
-                                             bool* rot) {
+__device__ __forceinline__ void rope_factors(long pos, const double* inv_freq, int rotated_pairs,
+                                             float* c, float* s, bool* rot) {
   constexpr int E = D / 64;
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const int k = lane * E + e;
-    rot[e] = k < rope.rotated_pairs;
+    rot[e] = k < rotated_pairs;
     c[e] = 1.f;
     s[e] = 0.f;
-    if (rot[e]) rope_sincos(pos, rope.inv_freq[k], &s[e], &c[e]);
+    if (rot[e]) rope_sincos(pos, inv_freq[k], &s[e], &c[e]);
   }
 }
 

@@ -55,14 +55,17 @@ __global__ void __launch_bounds__(kWarps * 32)
                           const T* __restrict__ v_raw, const T* __restrict__ wk, int B, int T_,
                           int Hq, int Hkv, KVDst d0, KVDst d1, int32_t* __restrict__ len_out,
                           const __grid_constant__ RopeParams rope, float eps) {
-  constexpr int E = D / 64, NB = 4;
+  constexpr int E = D / 64, NB = 8;
+  __shared__ double inv_freq[D / 2];
+  for (int k = threadIdx.x; k < D / 2; k += blockDim.x) inv_freq[k] = rope.inv_freq[k];
+  __syncthreads();
   const long tok = (long)blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (tok >= (long)B * T_) return;
   const int lane = threadIdx.x & 31;
   const long t = tok % T_, b = tok / T_;
   float c[E], s[E];
   bool rot[E];
-  rope_factors<D>(t, rope, c, s, rot);
+  rope_factors<D>(t, inv_freq, rope.rotated_pairs, c, s, rot);
   float w0[E], w1[E];
   Vec<T, E>::load(wq + lane * E, w0);
   Vec<T, E>::load(wq + D / 2 + lane * E, w1);
