@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                           const T* __restrict__ v_raw, const T* __restrict__ wk, int B, int T_,
                           int Hq, int Hkv, KVDst d0, KVDst d1, int32_t* __restrict__ len_out,
                           const __grid_constant__ RopeParams rope, float eps) {
-  constexpr int E = D / 64, NB = 8;
+  constexpr int E = D / 64, NB = D >= 512 ? 4 : 8;
   __shared__ double inv_freq[D / 2];
   for (int k = threadIdx.x; k < D / 2; k += blockDim.x) inv_freq[k] = rope.inv_freq[k];
   __syncthreads();
@@ -66,6 +66,17 @@ __global__ void __launch_bounds__(kWarps * 32)
   float c[E], s[E];
   bool rot[E];
   rope_factors<D>(t, inv_freq, rope.rotated_pairs, c, s, rot);
+  // the first K/V head's loads go out with the query heads' (one round
+  // trip to memory instead of two when Hkv == 1)
+  const T* vsrc = v_raw ? v_raw : k_raw;
+  float kv0[2][E], kv1[2][E];
+  if (k_raw) {
+    const long off = tok * Hkv * D;
+    Vec<T, E>::load(k_raw + off + lane * E, kv0[0]);
+    Vec<T, E>::load(k_raw + off + D / 2 + lane * E, kv1[0]);
+    Vec<T, E>::load(vsrc + off + lane * E, kv0[1]);
+    Vec<T, E>::load(vsrc + off + D / 2 + lane * E, kv1[1]);
+  }
   float w0[E], w1[E];
   Vec<T, E>::load(wq + lane * E, w0);
   Vec<T, E>::load(wq + D / 2 + lane * E, w1);
@@ -86,14 +97,23 @@ __global__ void __launch_bounds__(kWarps * 32)
   if (!k_raw) return;
   Vec<T, E>::load(wk + lane * E, w0);
   Vec<T, E>::load(wk + D / 2 + lane * E, w1);
-  const T* vsrc = v_raw ? v_raw : k_raw;
   for (int h = 0; h < Hkv; ++h) {
     float x0[2][E], x1[2][E];
     const long off = (tok * Hkv + h) * D;
-    Vec<T, E>::load(k_raw + off + lane * E, x0[0]);
-    Vec<T, E>::load(k_raw + off + D / 2 + lane * E, x1[0]);
-    Vec<T, E>::load(vsrc + off + lane * E, x0[1]);
-    Vec<T, E>::load(vsrc + off + D / 2 + lane * E, x1[1]);
+    if (h == 0) {
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        x0[0][e] = kv0[0][e];
+        x1[0][e] = kv1[0][e];
+        x0[1][e] = kv0[1][e];
+        x1[1][e] = kv1[1][e];
+      }
+    } else {
+      Vec<T, E>::load(k_raw + off + lane * E, x0[0]);
+      Vec<T, E>::load(k_raw + off + D / 2 + lane * E, x1[0]);
+      Vec<T, E>::load(vsrc + off + lane * E, x0[1]);
+      Vec<T, E>::load(vsrc + off + D / 2 + lane * E, x1[1]);
+    }
     norm_rope<D, 1>(x0, x1, w0, w1, c, s, rot, true, eps);
     norm_rope<D, 1>(x0 + 1, x1 + 1, nullptr, nullptr, c, s, rot, false, eps);
     put_kv<T, D>(d0, Hkv, b, h, t, x0[0], x1[0], x0[1], x1[1]);
