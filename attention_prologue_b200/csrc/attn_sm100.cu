@@ -29,8 +29,7 @@
 //               through registers); then normalise the previous tile's O
 //               and write it out (each thread its row) while the next tile
 //               runs
-// TMEM columns: NS = 3 S buffers of 64, (d = 256) Q dims 0..127 as bf16 pairs
-// at 192, O at 256 (d <= 128: O at 192).
+// TMEM columns: NS = 4 S buffers of 64, O at 256.
 //
 // The tensor core's issue queue is short and a tcgen05.mma blocks while it
 // is full; two issuing threads keep a ready PV from waiting behind an S.
@@ -61,19 +60,18 @@ namespace {
 constexpr int BM = 128;  // query rows per work tile
 constexpr int BN = 64;   // keys per key tile
 constexpr int kStagesV = 2;
-constexpr int kNS = 3;   // S buffers in TMEM
+constexpr int kNS = 4;   // S buffers in TMEM
 constexpr int kThreads = 384;
 constexpr int kSoftmaxWarp0 = 4;
 constexpr int kEpiWarp0 = 8;
 
 template <int D>
 struct Layout {
-  // d = 256: Q dims 0..127 live in TMEM (that half of the QK^T A operand is
-  // read from TMEM), dims 128..255 in shared memory; smaller heads keep all
-  // of Q in shared memory.  The room saved holds a fourth K stage.
-  static constexpr int kQTmemChunks = D == 256 ? 2 : 0;
+  // Q lives in shared memory (TMEM holds NS = 4 S buffers and O: 512
+  // columns at d = 256); d = 256 then leaves room for three K stages.
+  static constexpr int kQTmemChunks = 0;
   static constexpr bool kQT = kQTmemChunks > 0;
-  static constexpr int kStagesK = 4;
+  static constexpr int kStagesK = D == 256 ? 3 : 4;
   static constexpr int kChunks = D / 64;                  // 64-element (128-byte) columns
   static constexpr uint32_t kQChunk = BM * 128;           // bytes of one 128-row chunk
   static constexpr uint32_t kKVChunk = BN * 128;          // bytes of one K or V chunk
@@ -105,9 +103,9 @@ struct Bars {  // offsets (in 8-byte words) of the mbarriers from Layout::kBars
     v_full = 16,   // [2]
     v_empty = 18,  // [2]
     s_full = 20,   // [NS]
-    p_full = 23,   // [NS]
-    o_done = 26,   // [NS] PV_j done (one per S buffer: rescale waits stay in one phase)
-    count = 29
+    p_full = 24,   // [NS]
+    o_done = 28,   // [NS] PV_j done (one per S buffer: rescale waits stay in one phase)
+    count = 32
   };
 };
 
@@ -288,10 +286,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                mbar_wait(bar(Bars::q_tmem), k & 1, abort);
           for (int j = 0; ok && j < ti.n; ++j, ++g) {
             const int s = g % kStagesK;
+            // the K tile first: it lands well ahead, so the wait that gates
+            // the issue is the last one (each wait costs a poll round trip)
+            if (!(ok = mbar_wait(bar(Bars::k_full + s), (g / kStagesK) & 1, abort))) break;
             if (g >= kNS && !(ok = mbar_wait(bar(Bars::o_done + (g - kNS) % kNS),
                                              ((g - kNS) / kNS) & 1, abort)))
               break;
-            if (!(ok = mbar_wait(bar(Bars::k_full + s), (g / kStagesK) & 1, abort))) break;
             tc_fence_after();
             const uint64_t dk = desc_add(dk0, s * Ly::kChunks * Ly::kKVChunk);
             const uint32_t d = tmem + (g % kNS) * BN;
@@ -315,8 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t dv0 = desc_sw128(base + Ly::kV, Ly::kKVChunk, 1024);
           for (int j = 0; ok && j < ti.n; ++j, ++g) {
             const int s = g % kStagesV;
-            if (!(ok = mbar_wait(bar(Bars::p_full + g % kNS), (g / kNS) & 1, abort))) break;
             if (!(ok = mbar_wait(bar(Bars::v_full + s), (g / kStagesV) & 1, abort))) break;
+            if (!(ok = mbar_wait(bar(Bars::p_full + g % kNS), (g / kNS) & 1, abort))) break;
             // the first PV of a tile overwrites O: the previous tile's O is read out
             if (j == 0 && k > 0 && !(ok = mbar_wait(bar(Bars::o_free), (k - 1) & 1, abort)))
               break;
