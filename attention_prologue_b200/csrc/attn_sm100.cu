@@ -95,17 +95,17 @@ struct Bars {  // offsets (in 8-byte words) of the mbarriers from Layout::kBars
     q_empty = 2,  // the last S of a tile is done: Q may be replaced
     o_last = 3,   // the last PV of a tile is done
     o_free = 4,   // the epilogue warps have read O out of TMEM (128 arrivals)
-    l_ready = 5,  // the softmax warps have written the row sums (128 arrivals)
-    drain = 6,    // (S issuer)
-    drain2 = 7,   // (PV issuer)
-    k_full = 8,   // [4]
-    k_empty = 12,  // [4]
-    v_full = 16,   // [2]
-    v_empty = 18,  // [2]
-    s_full = 20,   // [NS]
-    p_full = 24,   // [NS]
-    o_done = 28,   // [NS] PV_j done (one per S buffer: rescale waits stay in one phase)
-    count = 32
+    l_ready = 5,  // [2] row sums of tiles k with k % 2 = i written (128 arrivals)
+    drain = 7,    // (S issuer)
+    drain2 = 8,   // (PV issuer)
+    k_full = 9,   // [4]
+    k_empty = 13,  // [4]
+    v_full = 17,   // [2]
+    v_empty = 19,  // [2]
+    s_full = 21,   // [NS]
+    p_full = 25,   // [NS]
+    o_done = 29,   // [NS] PV_j done (one per S buffer: rescale waits stay in one phase)
+    count = 33
   };
 };
 
@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(Bars::o_last), 1);
     mbar_init(bar(Bars::o_free), 4 * 32);
     mbar_init(bar(Bars::l_ready), 4 * 32);
+    mbar_init(bar(Bars::l_ready + 1), 4 * 32);
     mbar_init(bar(Bars::drain), 1);
     mbar_init(bar(Bars::drain2), 1);
     for (int s = 0; s < kStagesK; ++s) {
@@ -441,10 +442,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(Bars::p_full + sb));
       }
       if (!ok) break;
-      // the row sum for the epilogue warps (two buffers: the epilogue of
-      // tile k - 2 has finished before tile k's Q was loaded)
+      // the row sum for the epilogue warps, in buffer k % 2 with its own
+      // barrier: a tile of at most NS key tiles needs no PV of its own
+      // before its softmax ends, so the softmax can finish tile k while the
+      // epilogue has yet to wait for tile k - 1 (one barrier for both would
+      // then be two phases ahead of that wait); it cannot finish tile k + 1,
+      // whose Q is loaded only after the epilogue of tile k - 1
       lbuf[(k & 1) * BM + r] = l;
-      mbar_arrive(bar(Bars::l_ready));
+      mbar_arrive(bar(Bars::l_ready + (k & 1)));
     }
   } else {
     // ------------------------------------------------------------ Q and epilogue
@@ -498,8 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (k > 0) {
         // ---- epilogue of tile k - 1: O / l as bf16, each thread its row
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::o_last), (k - 1) & 1, abort) &&
-                                         mbar_wait(bar(Bars::l_ready), (k - 1) & 1, abort));
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(bar(Bars::o_last), (k - 1) & 1, abort) &&
+                            mbar_wait(bar(Bars::l_ready + ((k - 1) & 1)), ((k - 1) >> 1) & 1, abort));
         if (!ok) break;
         tc_fence_after();
         const float lsum = lbuf[((k - 1) & 1) * BM + r];
