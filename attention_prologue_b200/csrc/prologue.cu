@@ -30,7 +30,7 @@ int* status_ptr() {
   return ptrs[dev];
 }
 
-constexpr int kWarps = 8;  // warps per block of the per-vector kernels
+constexpr int kWarps = 4;  // warps per block of the per-vector kernels
 
 template <typename T, int D>
 __device__ __forceinline__ void put_kv(const KVDst& d, int Hkv, long b, int h, long t,
@@ -46,8 +46,11 @@ __device__ __forceinline__ void put_kv(const KVDst& d, int Hkv, long b, int h, l
 // Prologue of a whole prompt, one warp per token: the RoPE factors of the
 // token (position t) are computed once and applied to its Hq query heads and
 // Hkv key heads; the value heads are normalised without weight or rotation
-// (from the key projection with K=V).  Heads are processed NB at a time with
-// all their loads issued first.  k_raw == nullptr: queries only.
+// (from the key projection with K=V).  Heads are processed NB = 4 at a time
+// with all their loads issued first (four at a time and four warps a block
+// leave ~95 registers a thread: 20 warps per SM, against 16 with eight heads
+// a batch; the prologue is bound by memory latency).  k_raw == nullptr:
+// queries only.
 template <typename T, int D>
 __global__ void __launch_bounds__(kWarps * 32)
     token_prologue_kernel(const T* __restrict__ q_raw, const T* __restrict__ wq,
@@ -55,7 +58,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                           const T* __restrict__ v_raw, const T* __restrict__ wk, int B, int T_,
                           int Hq, int Hkv, KVDst d0, KVDst d1, int32_t* __restrict__ len_out,
                           const __grid_constant__ RopeParams rope, float eps) {
-  constexpr int E = D / 64, NB = D >= 512 ? 4 : 8;
+  constexpr int E = D / 64, NB = 4;
   __shared__ double inv_freq[D / 2];
   for (int k = threadIdx.x; k < D / 2; k += blockDim.x) inv_freq[k] = rope.inv_freq[k];
   __syncthreads();
@@ -63,11 +66,20 @@ __global__ void __launch_bounds__(kWarps * 32)
   if (tok >= (long)B * T_) return;
   const int lane = threadIdx.x & 31;
   const long t = tok % T_, b = tok / T_;
-  float c[E], s[E];
-  bool rot[E];
-  rope_factors<D>(t, inv_freq, rope.rotated_pairs, c, s, rot);
-  // the first K/V head's loads go out with the query heads' (one round
-  // trip to memory instead of two when Hkv == 1)
+  // the loads of the first batch of query heads and of the first K/V head
+  // go out together, and the RoPE factors (fp64 angle reduction) are
+  // computed while they are in flight
+  float x0[NB][E], x1[NB][E];
+  auto load_q = [&](int h0) {
+#pragma unroll
+    for (int j = 0; j < NB; ++j) {
+      const int h = min(h0 + j, Hq - 1);  // tail: recompute the last head, store once
+      const T* src = q_raw + (tok * Hq + h) * D;
+      Vec<T, E>::load(src + lane * E, x0[j]);
+      Vec<T, E>::load(src + D / 2 + lane * E, x1[j]);
+    }
+  };
+  load_q(0);
   const T* vsrc = v_raw ? v_raw : k_raw;
   float kv0[2][E], kv1[2][E];
   if (k_raw) {
@@ -80,15 +92,11 @@ __global__ void __launch_bounds__(kWarps * 32)
   float w0[E], w1[E];
   Vec<T, E>::load(wq + lane * E, w0);
   Vec<T, E>::load(wq + D / 2 + lane * E, w1);
+  float c[E], s[E];
+  bool rot[E];
+  rope_factors<D>(t, inv_freq, rope.rotated_pairs, c, s, rot);
   for (int h0 = 0; h0 < Hq; h0 += NB) {
-    float x0[NB][E], x1[NB][E];
-#pragma unroll
-    for (int j = 0; j < NB; ++j) {
-      const int h = min(h0 + j, Hq - 1);  // tail: recompute the last head, store once
-      const T* src = q_raw + (tok * Hq + h) * D;
-      Vec<T, E>::load(src + lane * E, x0[j]);
-      Vec<T, E>::load(src + D / 2 + lane * E, x1[j]);
-    }
+    if (h0 > 0) load_q(h0);
     norm_rope<D, NB>(x0, x1, w0, w1, c, s, rot, true, eps);
 #pragma unroll
     for (int j = 0; j < NB; ++j)
