@@ -558,7 +558,9 @@ def run_reference(args, dist: Dist):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    # 200 steps: the prefill's timed region (~30 ms) then spans several NVML
+    # clock samples; the decode half takes ~1.2 s
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=W.E2B_SLIDING.name,
