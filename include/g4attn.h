@@ -229,10 +229,13 @@ int g4attn_decode_noalloc(const g4attn_layer_desc *desc, const g4attn_cache *cac
 int g4attn_get_device_status(void *stream);
 
 /* Optional timing hook: the next g4attn_prefill or g4attn_decode call on any
- * stream records start_event immediately before and stop_event immediately
- * after its attention kernel (the dominant launch), on the call's stream, and
- * then forgets both.  The events are cudaEvent_t handles owned by the caller.
- * Passing NULLs cancels a pending request. */
+ * stream records start_event on the call's stream after enqueueing everything
+ * that precedes its attention kernel (the dominant launch) and stop_event
+ * right after enqueueing that kernel, then forgets both.  The interval holds
+ * the attention kernel alone; when the stream has drained before the kernel
+ * is enqueued it also holds the host's setup of that launch (tensor maps),
+ * so time it behind preceding work.  The events are cudaEvent_t handles
+ * owned by the caller.  Passing NULLs cancels a pending request. */
 void g4attn_time_next_attention(void *start_event, void *stop_event);
 
 /* Number of kernel launches the library has enqueued since it was loaded. */
