@@ -65,7 +65,9 @@ def _load():
         lib.or_prologue_q.argtypes = [LP, P, L, I, P, I, L, P]
         lib.or_prologue_kv.argtypes = [LP, P, P, L, I, P, I, L, P, P]
         lib.or_prefill_kv.argtypes = [LP, I, I, P, P, P, I, I, P, P, I]
+        lib.or_prefill_kv_at.argtypes = [LP, I, I, I, P, P, P, I, I, P, P, I]
         lib.or_prefill_rows.argtypes = [LP, I, I, P, P, I, I, P, P, P, P, I, P, I]
+        lib.or_prefill_chunk_rows.argtypes = [LP, I, I, I, P, P, I, I, P, P, P, P, I, P, I]
         lib.or_decode.argtypes = [LP, LP, P, P, I, I, P, P, I, I, I, P, P, P, P, P, I, P, I]
         lib.or_decode.restype = I
         lib.or_partial.argtypes = [P, P, P, L, I, I, I, D, P, P, P]
@@ -198,8 +200,9 @@ def prologue_kv(layer: Layer, k_vec, v_vec, wk, pos: int):
 
 # --- whole-layer entry points --------------------------------------------
 
-def prefill_kv(layer: Layer, k_raw, v_raw, wk, nthreads: int | None = None):
-    """Post-prologue K and V of every token, float64 [B, T, Hkv, d]."""
+def prefill_kv(layer: Layer, k_raw, v_raw, wk, nthreads: int | None = None, p0: int = 0):
+    """Post-prologue K and V of every token, float64 [B, T, Hkv, d]; the
+    tokens sit at positions p0 .. p0 + T - 1 (RoPE)."""
     k, dt = _raw(k_raw)
     v, _ = _raw(v_raw)
     w, wdt = _raw(wk)
@@ -207,8 +210,9 @@ def prefill_kv(layer: Layer, k_raw, v_raw, wk, nthreads: int | None = None):
     kh = np.empty((B, T, Hkv, d), np.float64)
     vh = np.empty((B, T, Hkv, d), np.float64)
     c = layer._c()
-    _load().or_prefill_kv(ctypes.byref(c), B, T, _p(k), _p(v) if v is not None else None,
-                          _p(w), dt, wdt, _p(kh), _p(vh), nthreads or default_threads())
+    _load().or_prefill_kv_at(ctypes.byref(c), B, T, int(p0), _p(k),
+                             _p(v) if v is not None else None, _p(w), dt, wdt, _p(kh), _p(vh),
+                             nthreads or default_threads())
     return kh, vh
 
 
@@ -235,6 +239,49 @@ def prefill(layer: Layer, q_raw, k_raw, v_raw, wq, wk, block_ids=None, rows=None
     """Prologue + masked softmax attention of a whole prompt."""
     kh, vh = prefill_kv(layer, k_raw, v_raw, wk, nthreads)
     return prefill_rows(layer, q_raw, wq, kh, vh, block_ids, rows, nthreads)
+
+
+def prefill_chunk_rows(layer: Layer, q_raw, wq, khat, vhat, p0: int, block_ids=None, rows=None,
+                       nthreads: int | None = None) -> np.ndarray:
+    """Cached (chunked) prefill ("gemma4-pt-claude" README, "Tests": the
+    cached path reproduces the uncached forward pass, image spans included).
+    q_raw [B, T, Hq, d] holds the chunk's queries at positions p0 .. p0+T-1;
+    khat/vhat [B, p0 + T, Hkv, d] the post-prologue keys and values of every
+    position up to the chunk's last; block_ids [B, p0 + T] or None.  Each
+    row attends over the interval of its position in a prompt of p0 + T
+    tokens.  Returns float64 [B, n_rows, Hq, d]."""
+    q, dt = _raw(q_raw)
+    w, wdt = _raw(wq)
+    B, T, Hq, d = q_raw.shape
+    if khat.shape[1] != p0 + T or vhat.shape[1] != p0 + T:
+        raise ValueError("khat/vhat must hold positions 0 .. p0 + T - 1")
+    ids = _i32(block_ids)
+    if ids is not None and ids.shape != (B, p0 + T):
+        raise ValueError("block_ids must be [B, p0 + T]")
+    rows_a = _i32(rows)
+    n_rows = T if rows_a is None else rows_a.size
+    out = np.empty((B, n_rows, Hq, d), np.float64)
+    khat = np.ascontiguousarray(khat, np.float64)
+    vhat = np.ascontiguousarray(vhat, np.float64)
+    c = layer._c()
+    _load().or_prefill_chunk_rows(ctypes.byref(c), B, T, int(p0), _p(q), _p(w), dt, wdt, _p(ids),
+                                  _p(khat), _p(vhat), _p(rows_a), n_rows, _p(out),
+                                  nthreads or default_threads())
+    return out
+
+
+def prefill_chunk(layer: Layer, q_raw, k_raw, v_raw, wq, wk, khat_cache, vhat_cache,
+                  block_ids=None, rows=None, nthreads: int | None = None):
+    """A chunk of T tokens after p0 = khat_cache.shape[1] cached ones: the
+    key/value prologue of the chunk at positions p0 .. p0+T-1, appended to
+    the cached keys/values, then chunked attention.  Returns (out,
+    khat, vhat) with khat/vhat [B, p0 + T, Hkv, d]."""
+    p0 = khat_cache.shape[1]
+    kh, vh = prefill_kv(layer, k_raw, v_raw, wk, nthreads, p0=p0)
+    khat = np.concatenate([khat_cache, kh], axis=1)
+    vhat = np.concatenate([vhat_cache, vh], axis=1)
+    out = prefill_chunk_rows(layer, q_raw, wq, khat, vhat, p0, block_ids, rows, nthreads)
+    return out, khat, vhat
 
 
 def decode(layer_q: Layer, q_raw, wq, cache_k, cache_v, capacity: int, rolling: bool, lens,

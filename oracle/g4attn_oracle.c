@@ -29,7 +29,9 @@
  * (k, k + d/2) for k < R = fraction*d/2 with frequency theta^(-2k/d) and leaves
  * the other pairs untouched (a zero-padded frequency vector); pairs are split
  * halves (rotate-half); positions are 0-based token indices; the KV head of
- * query head h is h / (Hq/Hkv).
+ * query head h is h / (Hq/Hkv); a chunk of a cached prefill sees keys up to
+ * its own last position, so an image block cut by the chunk's end is seen up
+ * to there (rows of earlier chunks are not recomputed).
  *
  * Parity status of the readings: the rotated-dimension selection, the pairing
  * convention, eps and the softmax scale are not fixed by any value the pages
@@ -226,13 +228,14 @@ static void or_attend(const double *q, const double *kbase,
 
 typedef struct {
   const or_layer *L;
-  int B, T;
+  int B, T;   /* T query rows per sequence (the chunk) */
+  int p0;     /* position of the chunk's first row */
   const void *q_raw, *wq;
   int dtype, w_dtype;
-  const int *block_ids;
+  const int *block_ids;      /* [B][p0 + T] */
   const int *rows;
   int n_rows;
-  const double *khat, *vhat; /* [B][T][Hkv][d] */
+  const double *khat, *vhat; /* [B][p0 + T][Hkv][d] */
   double *out;               /* [B][n_rows][Hq][d] */
   int tid, nthreads;
 } or_prefill_job;
@@ -243,21 +246,23 @@ static void *or_prefill_worker(void *arg) {
   int d = L->head_dim, Hq = L->num_heads, Hkv = L->num_kv_heads;
   int g = Hq / Hkv;
   double *q = (double *)malloc(sizeof(double) * d);
-  double *s = (double *)malloc(sizeof(double) * (J->T + 1));
+  const int Tk = J->p0 + J->T; /* positions a row of the chunk may see */
+  double *s = (double *)malloc(sizeof(double) * (Tk + 1));
   long items = (long)J->B * J->n_rows * Hq;
   for (long it = J->tid; it < items; it += J->nthreads) {
     int h = (int)(it % Hq);
     int r = (int)((it / Hq) % J->n_rows);
     int b = (int)(it / ((long)Hq * J->n_rows));
-    int i = J->rows ? J->rows[r] : r;
+    int i = J->rows ? J->rows[r] : r; /* row of the chunk */
+    int pos = J->p0 + i;
     long qoff = (((long)b * J->T + i) * Hq + h) * d;
-    or_prologue_q(L, J->q_raw, qoff, J->dtype, J->wq, J->w_dtype, i, q);
+    or_prologue_q(L, J->q_raw, qoff, J->dtype, J->wq, J->w_dtype, pos, q);
     int lo, hi;
-    or_interval(L, J->block_ids ? J->block_ids + (long)b * J->T : NULL, J->T,
-                i, &lo, &hi);
+    or_interval(L, J->block_ids ? J->block_ids + (long)b * Tk : NULL, Tk, pos,
+                &lo, &hi);
     int kvh = h / g;
-    const double *kb = J->khat + ((long)b * J->T * Hkv + kvh) * d;
-    const double *vb = J->vhat + ((long)b * J->T * Hkv + kvh) * d;
+    const double *kb = J->khat + ((long)b * Tk * Hkv + kvh) * d;
+    const double *vb = J->vhat + ((long)b * Tk * Hkv + kvh) * d;
     double *o = J->out + (((long)b * J->n_rows + r) * Hq + h) * d;
     or_attend(q, kb, vb, (long)Hkv * d, lo, hi, d, L->softmax_scale, s, o);
   }
@@ -269,6 +274,7 @@ static void *or_prefill_worker(void *arg) {
 typedef struct {
   const or_layer *L;
   int B, T;
+  int p0; /* position of the first token */
   const void *k_raw, *v_raw, *wk;
   int dtype, w_dtype;
   double *khat, *vhat;
@@ -281,7 +287,7 @@ static void *or_kv_worker(void *arg) {
   int d = L->head_dim, Hkv = L->num_kv_heads;
   long items = (long)J->B * J->T * Hkv;
   for (long it = J->tid; it < items; it += J->nthreads) {
-    long t = (it / Hkv) % J->T;
+    long t = J->p0 + (it / Hkv) % J->T;
     long off = it * d;
     or_prologue_kv(L, J->k_raw, J->v_raw, off, J->dtype, J->wk, J->w_dtype, t,
                    J->khat + off, J->vhat + off);
@@ -298,15 +304,16 @@ static void or_run(void *(*fn)(void *), void *jobs, size_t job_size,
   free(th);
 }
 
-/* Post-prologue keys and values of every token: khat, vhat [B][T][Hkv][d].
- * k_raw/v_raw are [B][T][Hkv][d] in `dtype`; v_raw is ignored with k_eq_v. */
-void or_prefill_kv(const or_layer *L, int B, int T, const void *k_raw,
-                   const void *v_raw, const void *wk, int dtype, int w_dtype,
-                   double *khat, double *vhat, int nthreads) {
+/* Post-prologue keys and values of T tokens at positions p0 .. p0+T-1:
+ * khat, vhat [B][T][Hkv][d].  k_raw/v_raw are [B][T][Hkv][d] in `dtype`;
+ * v_raw is ignored with k_eq_v. */
+void or_prefill_kv_at(const or_layer *L, int B, int T, int p0, const void *k_raw,
+                      const void *v_raw, const void *wk, int dtype, int w_dtype,
+                      double *khat, double *vhat, int nthreads) {
   if (nthreads < 1) nthreads = 1;
   or_kv_job *jobs = (or_kv_job *)calloc(nthreads, sizeof(or_kv_job));
   for (int t = 0; t < nthreads; ++t) {
-    or_kv_job j = {L, B, T, k_raw, v_raw, wk, dtype, w_dtype, khat, vhat,
+    or_kv_job j = {L, B, T, p0, k_raw, v_raw, wk, dtype, w_dtype, khat, vhat,
                    t, nthreads};
     jobs[t] = j;
   }
@@ -314,25 +321,51 @@ void or_prefill_kv(const or_layer *L, int B, int T, const void *k_raw,
   free(jobs);
 }
 
-/* Attention output of the listed query rows, given khat/vhat from
- * or_prefill_kv.  q_raw is [B][T][Hq][d]; rows lists query positions
- * (NULL = all T rows, n_rows = T); out is [B][n_rows][Hq][d]. */
+/* The same for a whole prompt (positions 0 .. T-1). */
+void or_prefill_kv(const or_layer *L, int B, int T, const void *k_raw,
+                   const void *v_raw, const void *wk, int dtype, int w_dtype,
+                   double *khat, double *vhat, int nthreads) {
+  or_prefill_kv_at(L, B, T, 0, k_raw, v_raw, wk, dtype, w_dtype, khat, vhat,
+                   nthreads);
+}
+
+/* Cached (chunked) prefill ("gemma4-pt-claude" README, "Tests": a cached
+ * path must reproduce the uncached forward pass, image spans included):
+ * the T query rows of a chunk at positions p0 .. p0+T-1 attend, each over
+ * the interval of its position in a prompt of p0 + T tokens, to keys held
+ * for all p0 + T positions.  q_raw is [B][T][Hq][d]; block_ids, when given,
+ * is [B][p0 + T] (an image block is seen up to the chunk's last position);
+ * khat/vhat are [B][p0 + T][Hkv][d]; rows lists rows of the chunk (NULL =
+ * all T, n_rows = T); out is [B][n_rows][Hq][d]. */
+void or_prefill_chunk_rows(const or_layer *L, int B, int T, int p0,
+                           const void *q_raw, const void *wq, int dtype,
+                           int w_dtype, const int *block_ids,
+                           const double *khat, const double *vhat,
+                           const int *rows, int n_rows, double *out,
+                           int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  or_prefill_job *jobs =
+      (or_prefill_job *)calloc(nthreads, sizeof(or_prefill_job));
+  for (int t = 0; t < nthreads; ++t) {
+    or_prefill_job j = {L,       B,         T,    p0,     q_raw, wq,
+                        dtype,   w_dtype,   block_ids, rows, n_rows, khat,
+                        vhat,    out,       t,    nthreads};
+    jobs[t] = j;
+  }
+  or_run(or_prefill_worker, jobs, sizeof(or_prefill_job), nthreads);
+  free(jobs);
+}
+
+/* Attention output of the listed query rows of a whole prompt, given
+ * khat/vhat from or_prefill_kv.  q_raw is [B][T][Hq][d]; rows lists query
+ * positions (NULL = all T rows, n_rows = T); out is [B][n_rows][Hq][d]. */
 void or_prefill_rows(const or_layer *L, int B, int T, const void *q_raw,
                      const void *wq, int dtype, int w_dtype,
                      const int *block_ids, const double *khat,
                      const double *vhat, const int *rows, int n_rows,
                      double *out, int nthreads) {
-  if (nthreads < 1) nthreads = 1;
-  or_prefill_job *jobs =
-      (or_prefill_job *)calloc(nthreads, sizeof(or_prefill_job));
-  for (int t = 0; t < nthreads; ++t) {
-    or_prefill_job j = {L,    B,     T,      q_raw, wq,       dtype,
-                        w_dtype, block_ids, rows, n_rows, khat, vhat,
-                        out,  t,     nthreads};
-    jobs[t] = j;
-  }
-  or_run(or_prefill_worker, jobs, sizeof(or_prefill_job), nthreads);
-  free(jobs);
+  or_prefill_chunk_rows(L, B, T, 0, q_raw, wq, dtype, w_dtype, block_ids, khat,
+                        vhat, rows, n_rows, out, nthreads);
 }
 
 /* ------------------------------------------------------------------ */

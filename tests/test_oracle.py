@@ -507,3 +507,69 @@ def test_row_sampling_and_threads_are_bit_exact():
 def test_window_plus_one_reading_is_available():
     L = sliding_layer(window=5, window_plus_one=True)
     assert oracle.interval(L, None, 20, 10) == (5, 10)  # w + 1 keys
+
+
+# ---------------------------------------------------------------------------
+# cached (chunked) prefill: "gemma4-pt-claude" README, "Tests" -- the cached
+# path reproduces the uncached forward pass, bidirectional image spans included
+
+def _chunked(L, q, k, v, wq, wk, ids, cuts):
+    """Run the prompt through the oracle's cached path in chunks [cuts[i], cuts[i+1])."""
+    B, T = q.shape[:2]
+    kh = np.zeros((B, 0, L.num_kv_heads, L.head_dim))
+    vh = np.zeros((B, 0, L.num_kv_heads, L.head_dim))
+    outs = []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        o, kh, vh = oracle.prefill_chunk(L, q[:, a:b], k[:, a:b], None if v is None else v[:, a:b],
+                                         wq, wk, kh, vh,
+                                         block_ids=None if ids is None else ids[:, :b])
+        outs.append(o)
+    return np.concatenate(outs, axis=1), kh, vh
+
+
+@pytest.mark.parametrize("case", ["sliding_blocks", "global_kv", "global_gqa"])
+def test_chunked_prefill_reproduces_the_whole_prompt(case):
+    rng = np.random.default_rng(11)
+    ids = None
+    if case == "sliding_blocks":
+        L = sliding_layer(window=6)
+        T = 40
+        # cuts between blocks (a block cut in two cannot be reproduced: its
+        # earlier rows would need later keys); windows reach across every cut
+        ids = ids_with_blocks(2, T, [(5, 12), (20, 31), (33, 35)])
+        cuts = [0, 13, 32, 40]
+    elif case == "global_kv":
+        L = global_layer()
+        T = 33
+        cuts = [0, 1, 17, 33]
+    else:
+        L = global_layer(k_eq_v=False, num_heads=8, num_kv_heads=2, head_dim=64)
+        T = 25
+        cuts = [0, 12, 25]
+    q, k, v, wq, wk = inputs(L, ids.shape[0] if ids is not None else 1, T, rng)
+    got, kh, vh = _chunked(L, q, k, v, wq, wk, ids, cuts)
+    ref = dense_reference(L, q, k, v, wq, wk, ids)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    # the keys/values accumulated chunk by chunk are those of the whole prompt
+    # (the RoPE position of a chunk's token is its position in the prompt)
+    kf, vf = oracle.prefill_kv(L, k, v, wk)
+    np.testing.assert_array_equal(kh, kf)
+    np.testing.assert_array_equal(vh, vf)
+
+
+def test_chunk_sees_an_image_block_up_to_its_last_position():
+    # A block that runs past the chunk's end is seen up to the chunk's last
+    # position: the chunk's rows equal the rows of the prompt cut there.
+    rng = np.random.default_rng(12)
+    L = sliding_layer(window=4)
+    T, cut = 30, 20
+    ids = ids_with_blocks(1, T, [(14, 27)])
+    q, k, v, wq, wk = inputs(L, 1, T, rng)
+    kh, vh = oracle.prefill_kv(L, k[:, :10], v[:, :10], wk)
+    got, _, _ = oracle.prefill_chunk(L, q[:, 10:cut], k[:, 10:cut], v[:, 10:cut], wq, wk, kh, vh,
+                                     block_ids=ids[:, :cut])
+    ref = dense_reference(L, q[:, :cut], k[:, :cut], v[:, :cut], wq, wk, ids[:, :cut])[:, 10:]
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    # and they differ from the whole prompt's rows, which see the block's tail
+    full = dense_reference(L, q, k, v, wq, wk, ids)[:, 10:cut]
+    assert np.abs(got[:, 4:] - full[:, 4:]).max() > 1e-3
