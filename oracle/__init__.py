@@ -48,7 +48,8 @@ class _Layer(ctypes.Structure):
                 ("k_eq_v", ctypes.c_int), ("num_heads", ctypes.c_int),
                 ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
                 ("softmax_scale", ctypes.c_double), ("rms_eps", ctypes.c_double),
-                ("rope_mode", ctypes.c_int), ("window_plus_one", ctypes.c_int)]
+                ("rope_mode", ctypes.c_int), ("window_plus_one", ctypes.c_int),
+                ("logit_softcap", ctypes.c_double)]
 
 
 def _load():
@@ -92,12 +93,14 @@ class Layer:
     rms_eps: float = 1e-6
     rope_mode: int = ROPE_ZEROPAD
     window_plus_one: bool = False
+    logit_softcap: float = 0.0  # 0: none; else s <- cap * tanh(s / cap)
 
     def _c(self) -> _Layer:
         return _Layer(int(self.layer_type), int(self.window), float(self.rotary_fraction),
                       float(self.rope_theta), int(bool(self.k_eq_v)), int(self.num_heads),
                       int(self.num_kv_heads), int(self.head_dim), float(self.softmax_scale),
-                      float(self.rms_eps), int(self.rope_mode), int(bool(self.window_plus_one)))
+                      float(self.rms_eps), int(self.rope_mode), int(bool(self.window_plus_one)),
+                      float(self.logit_softcap))
 
 
 def default_threads() -> int:

@@ -67,6 +67,7 @@ typedef struct {
   double rms_eps;
   int rope_mode;           /* OR_ROPE_ZEROPAD (default) or OR_ROPE_PREFIX */
   int window_plus_one;     /* 1: the printed j in [i-w, i] reading (w+1 keys) */
+  double logit_softcap;    /* 0: none; else s <- cap * tanh(s / cap) */
 } or_layer;
 
 /* Exact value of element i of a bf16 (raw bits), fp32 or fp64 array. */
@@ -197,18 +198,22 @@ void or_interval(const or_layer *L, const int *ids, int T, int i, int *lo,
 }
 
 /* Masked softmax attention of one query over keys lo..hi (explicit loop):
- *   o = sum_j e^{s_j - M} v_j / sum_j e^{s_j - M},  s_j = scale * q . k_j.
+ *   o = sum_j e^{s_j - M} v_j / sum_j e^{s_j - M},  s_j = scale * q . k_j,
+ * and with a logit soft-cap c > 0 ("gemma4-pt-claude" README, "Attention
+ * Backend": attn_logits_soft_cap; the page prints no formula, the reading
+ * is the usual one) s_j <- c * tanh(s_j / c) before the softmax.
  * kbase/vbase point to key/value rows spaced `stride` doubles apart.  The
  * two-pass form (max first) is the plain definition; no online rescaling. */
 static void or_attend(const double *q, const double *kbase,
                       const double *vbase, long stride, int lo, int hi, int d,
-                      double scale, double *s_buf, double *o) {
+                      double scale, double cap, double *s_buf, double *o) {
   double m = -INFINITY;
   for (int j = lo; j <= hi; ++j) {
     const double *kj = kbase + (long)j * stride;
     double dot = 0.0;
     for (int k = 0; k < d; ++k) dot += q[k] * kj[k];
     double s = scale * dot;
+    if (cap > 0.0) s = cap * tanh(s / cap);
     s_buf[j - lo] = s;
     if (s > m) m = s;
   }
@@ -264,7 +269,8 @@ static void *or_prefill_worker(void *arg) {
     const double *kb = J->khat + ((long)b * Tk * Hkv + kvh) * d;
     const double *vb = J->vhat + ((long)b * Tk * Hkv + kvh) * d;
     double *o = J->out + (((long)b * J->n_rows + r) * Hq + h) * d;
-    or_attend(q, kb, vb, (long)Hkv * d, lo, hi, d, L->softmax_scale, s, o);
+    or_attend(q, kb, vb, (long)Hkv * d, lo, hi, d, L->softmax_scale,
+              L->logit_softcap, s, o);
   }
   free(q);
   free(s);
@@ -449,7 +455,8 @@ static void *or_decode_worker(void *arg) {
         vd[k] = or_load(J->cache_v, base + k, J->cache_dtype);
       }
     }
-    or_attend(q, kk, vv, d, 0, (int)(n - 1), d, Lq->softmax_scale, s,
+    or_attend(q, kk, vv, d, 0, (int)(n - 1), d, Lq->softmax_scale,
+              Lq->logit_softcap, s,
               J->out + ((long)si * Hq + h) * d);
     free(kk);
     free(vv);

@@ -573,3 +573,54 @@ def test_chunk_sees_an_image_block_up_to_its_last_position():
     # and they differ from the whole prompt's rows, which see the block's tail
     full = dense_reference(L, q, k, v, wq, wk, ids)[:, 10:cut]
     assert np.abs(got[:, 4:] - full[:, 4:]).max() > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# logit soft-cap ("gemma4-pt-claude" README, "Attention Backend":
+# attn_logits_soft_cap; reading s <- c * tanh(s / c))
+
+def test_softcap_two_keys_is_a_sigmoid_of_capped_scores():
+    L = global_layer(k_eq_v=False, num_heads=1, num_kv_heads=1, softmax_scale=0.37,
+                     logit_softcap=0.8)
+    q, k, v, wq, wk = inputs(L, 1, 2, rng=np.random.default_rng(21))
+    out = oracle.prefill(L, q, k, v, wq, wk)
+    qh = oracle.prologue_q(L, q[0, 1, 0], wq, 1)
+    k0, v0 = oracle.prologue_kv(L, k[0, 0, 0], v[0, 0, 0], wk, 0)
+    k1, v1 = oracle.prologue_kv(L, k[0, 1, 0], v[0, 1, 0], wk, 1)
+    c0, c1 = (0.8 * math.tanh(0.37 * (qh @ kk) / 0.8) for kk in (k0, k1))
+    sig = 1.0 / (1.0 + math.exp(-(c1 - c0)))
+    np.testing.assert_allclose(out[0, 1, 0], sig * v1 + (1 - sig) * v0, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("mk", [sliding_layer, global_layer])
+def test_softcap_vanishes_as_the_cap_grows(mk):
+    rng = np.random.default_rng(22)
+    L = mk()
+    q, k, v, wq, wk = inputs(L, 1, 20, rng)
+    plain = oracle.prefill(L, q, k, v, wq, wk)
+    L.logit_softcap = 1e9  # c tanh(s / c) = s - s^3 / (3 c^2) + ...
+    np.testing.assert_allclose(oracle.prefill(L, q, k, v, wq, wk), plain, rtol=0, atol=1e-12)
+
+
+def test_softcap_bounds_every_weight():
+    # |capped score| < c, so each of the n weights of a row lies in
+    # (e^{-2c} / n, e^{2c} / n); one-hot values read the weights out
+    L = global_layer(k_eq_v=False, num_heads=1, num_kv_heads=1, head_dim=32, softmax_scale=50.0,
+                     logit_softcap=0.3)
+    T = 24
+    rng = np.random.default_rng(23)
+    q, k, _, wq, wk = inputs(L, 1, T, rng)
+    v = np.zeros((1, T, 1, 32), np.float32)
+    for j in range(T):
+        v[0, j, 0, j] = 1.0  # V-norm scales a one-hot row to e_j / sqrt(1/32 + eps)
+    g = math.sqrt(1 / 32 + L.rms_eps)
+    out = oracle.prefill(L, q, k, v, wq, wk)[0, :, 0] * g
+    for i in range(T):
+        w = out[i, :i + 1]
+        n = i + 1
+        assert abs(w.sum() - 1.0) < 1e-12
+        assert w.min() > math.exp(-0.6) / n - 1e-15 and w.max() < math.exp(0.6) / n + 1e-15
+    # without the cap the same scores (scale 50) are far from uniform
+    L.logit_softcap = 0.0
+    plain = oracle.prefill(L, q, k, v, wq, wk)[0, :, 0] * g
+    assert plain[T - 1, :T].max() > 0.5
