@@ -69,6 +69,8 @@ def _load():
         lib.or_prefill_kv_at.argtypes = [LP, I, I, I, P, P, P, I, I, P, P, I]
         lib.or_prefill_rows.argtypes = [LP, I, I, P, P, I, I, P, P, P, P, I, P, I]
         lib.or_prefill_chunk_rows.argtypes = [LP, I, I, I, P, P, I, I, P, P, P, P, I, P, I]
+        lib.or_prefill_chunk_rows_masked.argtypes = [LP, I, I, I, P, P, I, I, P, P, P, P, P, I,
+                                                     P, I]
         lib.or_decode.argtypes = [LP, LP, P, P, I, I, P, P, I, I, I, P, P, P, P, P, I, P, I]
         lib.or_decode.restype = I
         lib.or_partial.argtypes = [P, P, P, L, I, I, I, D, P, P, P]
@@ -220,8 +222,13 @@ def prefill_kv(layer: Layer, k_raw, v_raw, wk, nthreads: int | None = None, p0: 
 
 
 def prefill_rows(layer: Layer, q_raw, wq, khat, vhat, block_ids=None, rows=None,
-                 nthreads: int | None = None) -> np.ndarray:
-    """Attention output of the given query rows, float64 [B, n_rows, Hq, d]."""
+                 nthreads: int | None = None, attention_mask=None) -> np.ndarray:
+    """Attention output of the given query rows, float64 [B, n_rows, Hq, d].
+    attention_mask [B, T] (1 = keep, 0 = padding) drops padding keys; a row
+    left without keys outputs 0."""
+    if attention_mask is not None:
+        return prefill_chunk_rows(layer, q_raw, wq, khat, vhat, 0, block_ids, rows, nthreads,
+                                  attention_mask)
     q, dt = _raw(q_raw)
     w, wdt = _raw(wq)
     B, T, Hq, d = q_raw.shape
@@ -238,21 +245,22 @@ def prefill_rows(layer: Layer, q_raw, wq, khat, vhat, block_ids=None, rows=None,
 
 
 def prefill(layer: Layer, q_raw, k_raw, v_raw, wq, wk, block_ids=None, rows=None,
-            nthreads: int | None = None) -> np.ndarray:
+            nthreads: int | None = None, attention_mask=None) -> np.ndarray:
     """Prologue + masked softmax attention of a whole prompt."""
     kh, vh = prefill_kv(layer, k_raw, v_raw, wk, nthreads)
-    return prefill_rows(layer, q_raw, wq, kh, vh, block_ids, rows, nthreads)
+    return prefill_rows(layer, q_raw, wq, kh, vh, block_ids, rows, nthreads, attention_mask)
 
 
 def prefill_chunk_rows(layer: Layer, q_raw, wq, khat, vhat, p0: int, block_ids=None, rows=None,
-                       nthreads: int | None = None) -> np.ndarray:
+                       nthreads: int | None = None, attention_mask=None) -> np.ndarray:
     """Cached (chunked) prefill ("gemma4-pt-claude" README, "Tests": the
     cached path reproduces the uncached forward pass, image spans included).
     q_raw [B, T, Hq, d] holds the chunk's queries at positions p0 .. p0+T-1;
     khat/vhat [B, p0 + T, Hkv, d] the post-prologue keys and values of every
     position up to the chunk's last; block_ids [B, p0 + T] or None.  Each
     row attends over the interval of its position in a prompt of p0 + T
-    tokens.  Returns float64 [B, n_rows, Hq, d]."""
+    tokens; attention_mask [B, p0 + T] (1 = keep, 0 = padding) drops padding
+    keys.  Returns float64 [B, n_rows, Hq, d]."""
     q, dt = _raw(q_raw)
     w, wdt = _raw(wq)
     B, T, Hq, d = q_raw.shape
@@ -266,10 +274,15 @@ def prefill_chunk_rows(layer: Layer, q_raw, wq, khat, vhat, p0: int, block_ids=N
     out = np.empty((B, n_rows, Hq, d), np.float64)
     khat = np.ascontiguousarray(khat, np.float64)
     vhat = np.ascontiguousarray(vhat, np.float64)
+    keep = None
+    if attention_mask is not None:
+        keep = np.ascontiguousarray(np.asarray(attention_mask) != 0, np.uint8)
+        if keep.shape != (B, p0 + T):
+            raise ValueError("attention_mask must be [B, p0 + T]")
     c = layer._c()
-    _load().or_prefill_chunk_rows(ctypes.byref(c), B, T, int(p0), _p(q), _p(w), dt, wdt, _p(ids),
-                                  _p(khat), _p(vhat), _p(rows_a), n_rows, _p(out),
-                                  nthreads or default_threads())
+    _load().or_prefill_chunk_rows_masked(ctypes.byref(c), B, T, int(p0), _p(q), _p(w), dt, wdt,
+                                         _p(ids), _p(keep), _p(khat), _p(vhat), _p(rows_a),
+                                         n_rows, _p(out), nthreads or default_threads())
     return out
 
 

@@ -202,13 +202,18 @@ void or_interval(const or_layer *L, const int *ids, int T, int i, int *lo,
  * and with a logit soft-cap c > 0 ("gemma4-pt-claude" README, "Attention
  * Backend": attn_logits_soft_cap; the page prints no formula, the reading
  * is the usual one) s_j <- c * tanh(s_j / c) before the softmax.
+ * keep (indexed by key position, NULL = every key kept) drops padding keys
+ * ("Gemma4ConditionalGenerate" arguments: attention_mask 1 = keep, 0 =
+ * padding); a query left with no key gets o = 0.
  * kbase/vbase point to key/value rows spaced `stride` doubles apart.  The
  * two-pass form (max first) is the plain definition; no online rescaling. */
 static void or_attend(const double *q, const double *kbase,
                       const double *vbase, long stride, int lo, int hi, int d,
-                      double scale, double cap, double *s_buf, double *o) {
+                      double scale, double cap, const unsigned char *keep,
+                      double *s_buf, double *o) {
   double m = -INFINITY;
   for (int j = lo; j <= hi; ++j) {
+    if (keep && !keep[j]) continue;
     const double *kj = kbase + (long)j * stride;
     double dot = 0.0;
     for (int k = 0; k < d; ++k) dot += q[k] * kj[k];
@@ -219,7 +224,9 @@ static void or_attend(const double *q, const double *kbase,
   }
   double den = 0.0;
   for (int k = 0; k < d; ++k) o[k] = 0.0;
+  if (m == -INFINITY) return; /* no key left */
   for (int j = lo; j <= hi; ++j) {
+    if (keep && !keep[j]) continue;
     double p = exp(s_buf[j - lo] - m);
     den += p;
     const double *vj = vbase + (long)j * stride;
@@ -238,6 +245,7 @@ typedef struct {
   const void *q_raw, *wq;
   int dtype, w_dtype;
   const int *block_ids;      /* [B][p0 + T] */
+  const unsigned char *keep; /* [B][p0 + T] or NULL */
   const int *rows;
   int n_rows;
   const double *khat, *vhat; /* [B][p0 + T][Hkv][d] */
@@ -270,7 +278,7 @@ static void *or_prefill_worker(void *arg) {
     const double *vb = J->vhat + ((long)b * Tk * Hkv + kvh) * d;
     double *o = J->out + (((long)b * J->n_rows + r) * Hq + h) * d;
     or_attend(q, kb, vb, (long)Hkv * d, lo, hi, d, L->softmax_scale,
-              L->logit_softcap, s, o);
+              L->logit_softcap, J->keep ? J->keep + (long)b * Tk : NULL, s, o);
   }
   free(q);
   free(s);
@@ -342,24 +350,38 @@ void or_prefill_kv(const or_layer *L, int B, int T, const void *k_raw,
  * for all p0 + T positions.  q_raw is [B][T][Hq][d]; block_ids, when given,
  * is [B][p0 + T] (an image block is seen up to the chunk's last position);
  * khat/vhat are [B][p0 + T][Hkv][d]; rows lists rows of the chunk (NULL =
- * all T, n_rows = T); out is [B][n_rows][Hq][d]. */
+ * all T, n_rows = T); out is [B][n_rows][Hq][d].  keep, when given, is the
+ * padding mask [B][p0 + T] (1 = keep, 0 = padding key). */
+void or_prefill_chunk_rows_masked(const or_layer *L, int B, int T, int p0,
+                                  const void *q_raw, const void *wq, int dtype,
+                                  int w_dtype, const int *block_ids,
+                                  const unsigned char *keep,
+                                  const double *khat, const double *vhat,
+                                  const int *rows, int n_rows, double *out,
+                                  int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  or_prefill_job *jobs =
+      (or_prefill_job *)calloc(nthreads, sizeof(or_prefill_job));
+  for (int t = 0; t < nthreads; ++t) {
+    or_prefill_job j = {L,     B,       T,         p0,   q_raw,  wq,
+                        dtype, w_dtype, block_ids, keep, rows,   n_rows,
+                        khat,  vhat,    out,       t,    nthreads};
+    jobs[t] = j;
+  }
+  or_run(or_prefill_worker, jobs, sizeof(or_prefill_job), nthreads);
+  free(jobs);
+}
+
+/* The same with every key kept. */
 void or_prefill_chunk_rows(const or_layer *L, int B, int T, int p0,
                            const void *q_raw, const void *wq, int dtype,
                            int w_dtype, const int *block_ids,
                            const double *khat, const double *vhat,
                            const int *rows, int n_rows, double *out,
                            int nthreads) {
-  if (nthreads < 1) nthreads = 1;
-  or_prefill_job *jobs =
-      (or_prefill_job *)calloc(nthreads, sizeof(or_prefill_job));
-  for (int t = 0; t < nthreads; ++t) {
-    or_prefill_job j = {L,       B,         T,    p0,     q_raw, wq,
-                        dtype,   w_dtype,   block_ids, rows, n_rows, khat,
-                        vhat,    out,       t,    nthreads};
-    jobs[t] = j;
-  }
-  or_run(or_prefill_worker, jobs, sizeof(or_prefill_job), nthreads);
-  free(jobs);
+  or_prefill_chunk_rows_masked(L, B, T, p0, q_raw, wq, dtype, w_dtype,
+                               block_ids, NULL, khat, vhat, rows, n_rows, out,
+                               nthreads);
 }
 
 /* Attention output of the listed query rows of a whole prompt, given
@@ -456,7 +478,7 @@ static void *or_decode_worker(void *arg) {
       }
     }
     or_attend(q, kk, vv, d, 0, (int)(n - 1), d, Lq->softmax_scale,
-              Lq->logit_softcap, s,
+              Lq->logit_softcap, NULL, s,
               J->out + ((long)si * Hq + h) * d);
     free(kk);
     free(vv);

@@ -56,10 +56,11 @@ def ids_with_blocks(B, T, runs):
 # ---------------------------------------------------------------------------
 # independent dense formulation (brute force on tiny inputs)
 
-def dense_reference(L, q, k, v, wq, wk, ids):
+def dense_reference(L, q, k, v, wq, wk, ids, keep=None):
     """Whole-matrix float64 formulation: RoPE as complex multiplication, the
     mask as an explicit boolean matrix built from the set definition (window
-    OR same image run), softmax with numpy."""
+    OR same image run, AND a kept key when a padding mask is given), softmax
+    with numpy; a row with no allowed key is 0."""
     q, k = q.astype(np.float64), k.astype(np.float64)
     v = k if L.k_eq_v else v.astype(np.float64)
     B, T, Hq, d = q.shape
@@ -103,11 +104,16 @@ def dense_reference(L, q, k, v, wq, wk, ids):
                         run[t] = r
                 same = (run[:, None] == run[None, :]) & (run[:, None] >= 0)
                 allowed = allowed | same
+        if keep is not None:
+            allowed = allowed & (keep[b][None, :] != 0)
         s = np.einsum("ihd,jhd->hij", qh[b], kh[b]) * L.softmax_scale
+        if L.logit_softcap > 0:
+            s = L.logit_softcap * np.tanh(s / L.logit_softcap)
         s = np.where(allowed[None], s, -np.inf)
-        s = s - s.max(axis=-1, keepdims=True)
-        p = np.exp(s)
-        p /= p.sum(axis=-1, keepdims=True)
+        m = s.max(axis=-1, keepdims=True)
+        p = np.exp(s - np.where(np.isfinite(m), m, 0.0))  # a row with no key: all 0
+        den = p.sum(axis=-1, keepdims=True)
+        p = p / np.where(den > 0, den, 1.0)
         out[b] = np.einsum("hij,jhd->ihd", p, vh[b])
     return out
 
@@ -624,3 +630,45 @@ def test_softcap_bounds_every_weight():
     L.logit_softcap = 0.0
     plain = oracle.prefill(L, q, k, v, wq, wk)[0, :, 0] * g
     assert plain[T - 1, :T].max() > 0.5
+
+
+# ---------------------------------------------------------------------------
+# padding ("Gemma4ConditionalGenerate" arguments: attention_mask, 1 = keep,
+# 0 = padding): padding keys are never attended; a row left with no key is 0
+
+@pytest.mark.parametrize("case", ["sliding_left_pad", "global_left_pad", "sliding_holes_softcap"])
+def test_padding_mask_matches_the_dense_reference(case):
+    rng = np.random.default_rng(31)
+    ids = None
+    if case == "sliding_left_pad":
+        L = sliding_layer(window=6)
+        T = 30
+        ids = ids_with_blocks(2, T, [(12, 19)])
+        keep = np.ones((2, T), np.int32)
+        keep[0, :5] = 0  # sequence 0 left-padded by 5, sequence 1 not at all
+    elif case == "global_left_pad":
+        L = global_layer()
+        T = 26
+        keep = np.ones((1, T), np.int32)
+        keep[0, :9] = 0
+    else:
+        L = sliding_layer(window=5, logit_softcap=2.0)
+        T = 24
+        keep = (rng.random((1, T)) > 0.3).astype(np.int32)
+        keep[0, 10:16] = 0  # rows 10..15 (window 5) see no key at all
+    B = keep.shape[0]
+    q, k, v, wq, wk = inputs(L, B, T, rng)
+    got = oracle.prefill(L, q, k, v, wq, wk, block_ids=ids, attention_mask=keep)
+    ref = dense_reference(L, q, k, v, wq, wk, ids, keep)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    if case == "sliding_holes_softcap":
+        assert not got[0, 14].any()  # a row with no key left is exactly 0
+
+
+def test_all_ones_padding_mask_changes_nothing():
+    rng = np.random.default_rng(32)
+    L = sliding_layer(window=7)
+    q, k, v, wq, wk = inputs(L, 2, 21, rng)
+    plain = oracle.prefill(L, q, k, v, wq, wk)
+    masked = oracle.prefill(L, q, k, v, wq, wk, attention_mask=np.ones((2, 21), np.int32))
+    np.testing.assert_array_equal(masked, plain)
