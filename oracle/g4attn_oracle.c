@@ -201,7 +201,9 @@ void or_interval(const or_layer *L, const int *ids, int T, int i, int *lo,
  *   o = sum_j e^{s_j - M} v_j / sum_j e^{s_j - M},  s_j = scale * q . k_j,
  * and with a logit soft-cap c > 0 ("gemma4-pt-claude" README, "Attention
  * Backend": attn_logits_soft_cap; the page prints no formula, the reading
- * is the usual one) s_j <- c * tanh(s_j / c) before the softmax.
+ * is the usual tanh cap, the form the "Gemma 4" Keras docs' argument table
+ * names for the output-logit cap) s_j <- c * tanh(s_j / c) before the
+ * softmax.
  * keep (indexed by key position, NULL = every key kept) drops padding keys
  * ("Gemma4ConditionalGenerate" arguments: attention_mask 1 = keep, 0 =
  * padding); a query left with no key gets o = 0.
