@@ -508,6 +508,10 @@ def pick_stride(w, inp, threads, target_s):
     return max(1, int(math.ceil(w.T * per_row / target_s)))
 
 
+def rows_phrase(stride: int) -> str:
+    return "every query row" if stride == 1 else f"every {stride}th query row"
+
+
 def cpu_baseline(w, inp, target_s=12.0):
     import oracle
     oracle.build()
@@ -515,7 +519,7 @@ def cpu_baseline(w, inp, target_s=12.0):
     stride = pick_stride(w, inp, threads, target_s)
     v, secs, n = oracle_sample(w, inp, stride, threads)
     return {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{w.name}: every {stride}th query row ({n} rows x {w.layer.num_heads} heads, "
+            "sample": f"{w.name}: {rows_phrase(stride)} ({n} rows x {w.layer.num_heads} heads, "
                       f"{secs:.1f} s) plus the K/V prologue charged pro rata; float64 C, "
                       f"{threads} threads"}
 
@@ -546,7 +550,7 @@ def run_reference(args, dist: Dist):
                        "heads": [w.layer.num_heads, w.layer.num_kv_heads],
                        "head_dim": w.layer.head_dim, "window": w.layer.window},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                             "sample": f"every {stride}th query row of {w.name}, all heads"},
+                             "sample": f"{rows_phrase(stride)} of {w.name}, all heads"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
