@@ -7,6 +7,7 @@
 #include <mutex>
 #include <atomic>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "g4attn.h"
@@ -16,6 +17,40 @@ namespace g4 {
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// The unique id of the calling thread's current CUDA context (cuCtxGetId:
+// never reused within a process, unlike the context handle).  Device
+// addresses of the library's __device__ variables are cached per context id,
+// so a context destroyed and re-created (cudaDeviceReset) gets a fresh lookup.
+bool current_context_id(unsigned long long* id) {
+  using GetCurrentFn = CUresult (*)(CUcontext*);
+  using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static std::once_flag once;
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetIdFn>(p);
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return false;
+  if (!ctx) {
+    // a thread that has made no runtime call yet: let the runtime make the
+    // device's primary context current (never reached while a stream of
+    // this thread is being captured, which needs a current context)
+    if (cudaFree(nullptr) != cudaSuccess || get_current(&ctx) != CUDA_SUCCESS || !ctx)
+      return false;
+  }
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 static std::mutex g_time_mu;
 static cudaEvent_t g_time_ev0 = nullptr, g_time_ev1 = nullptr;
@@ -36,9 +71,8 @@ static int make_cfg(const g4attn_layer_desc* d, LayerCfg* L) {
   if (!d) return G4ATTN_EINVAL;
   if (d->layer_type != G4ATTN_SLIDING && d->layer_type != G4ATTN_GLOBAL) return G4ATTN_EINVAL;
   if (d->dtype != G4ATTN_BF16 && d->dtype != G4ATTN_FP32) return G4ATTN_EINVAL;
-  if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256 && d->head_dim != 512)
-    return G4ATTN_EINVAL;
-  if (d->num_heads < 1 || d->num_kv_heads < 1 || d->num_kv_heads > 32) return G4ATTN_EINVAL;
+  if (d->head_dim < 2 || (d->head_dim & 1)) return G4ATTN_EINVAL;
+  if (d->num_heads < 1 || d->num_kv_heads < 1) return G4ATTN_EINVAL;
   if (d->num_heads % d->num_kv_heads != 0) return G4ATTN_EINVAL;
   if (d->layer_type == G4ATTN_SLIDING && d->window < 1) return G4ATTN_EINVAL;
   if (!(d->rotary_fraction >= 0.f && d->rotary_fraction <= 1.f)) return G4ATTN_EINVAL;
@@ -49,6 +83,12 @@ static int make_cfg(const g4attn_layer_desc* d, LayerCfg* L) {
   if (!(d->softmax_scale > 0.f) || !std::isfinite(d->softmax_scale)) return G4ATTN_EINVAL;
   if (!(d->rms_eps >= 0.f) || !std::isfinite(d->rms_eps)) return G4ATTN_EINVAL;
   if (d->k_eq_v != 0 && d->k_eq_v != 1) return G4ATTN_EINVAL;
+  // a valid layer without a kernel: head sizes other than 64/128/256/512, or
+  // more than 32 KV heads (the cache append runs one warp per KV head in a
+  // single block of at most 1024 threads)
+  if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256 && d->head_dim != 512)
+    return G4ATTN_EUNSUPPORTED;
+  if (d->num_kv_heads > 32) return G4ATTN_EUNSUPPORTED;
   L->layer_type = d->layer_type;
   L->window = d->layer_type == G4ATTN_SLIDING ? d->window : 0;
   L->k_eq_v = d->k_eq_v;

@@ -16,7 +16,7 @@
 //   warp 0      TMA producer of K tiles (all work tiles in sequence)
 //   warp 2      TMA producer of V tiles
 //   warp 1      owns TMEM; one thread issues S_j = Q K_j^T (M 128, N 64,
-//               K = d; A in smem or TMEM, B K-major), S_j only once PV_{j-NS}
+//               K = d; A and B K-major in smem), S_j only once PV_{j-NS}
 //               is done (a commit tracks its own thread's MMAs)
 //   warp 3      one thread issues O += P_j V_j (M 128, N = d, K 64; P from
 //               TMEM, V MN-major); the first PV of a tile waits until the
@@ -25,8 +25,7 @@
 //               edge tiles, lazy O rescale, P_j = exp2(S_j - m) as bf16 into
 //               TMEM over S_j; hands the row sums to the epilogue warps
 //   warps 8..11 Q and epilogue: after the last S of a tile, load the next
-//               tile's Q (its shared-memory half by TMA, its TMEM half
-//               through registers); then normalise the previous tile's O
+//               tile's Q by TMA; then normalise the previous tile's O
 //               and write it out (each thread its row) while the next tile
 //               runs
 // TMEM columns: NS = 4 S buffers of 64, O at 256.
@@ -69,29 +68,24 @@ template <int D>
 struct Layout {
   // Q lives in shared memory (TMEM holds NS = 4 S buffers and O: 512
   // columns at d = 256); d = 256 then leaves room for three K stages.
-  static constexpr int kQTmemChunks = 0;
-  static constexpr bool kQT = kQTmemChunks > 0;
   static constexpr int kStagesK = D == 256 ? 3 : 4;
   static constexpr int kChunks = D / 64;                  // 64-element (128-byte) columns
   static constexpr uint32_t kQChunk = BM * 128;           // bytes of one 128-row chunk
   static constexpr uint32_t kKVChunk = BN * 128;          // bytes of one K or V chunk
-  static constexpr uint32_t kQ = 0;                       // Q chunks kQTmemChunks..
-  static constexpr uint32_t kK = kQ + (kChunks - kQTmemChunks) * kQChunk;
+  static constexpr uint32_t kQ = 0;                       // Q chunks
+  static constexpr uint32_t kK = kQ + kChunks * kQChunk;
   static constexpr uint32_t kV = kK + kStagesK * kChunks * kKVChunk;
   static constexpr uint32_t kL = kV + kStagesV * kChunks * kKVChunk;  // row sums [2][128]
   static constexpr uint32_t kBars = kL + 2 * BM * 4;
   static constexpr uint32_t kAlloc = kBars + 512;  // + barriers and scalars
   static_assert(kAlloc <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
-  static constexpr uint32_t kColQ = kNS * BN;             // Q (bf16 pairs) when kQT
-  static constexpr uint32_t kColO = kQT ? 256 : kNS * BN;
+  static constexpr uint32_t kColO = kNS * BN;
   static constexpr uint32_t kTmemCols = (kColO + D) <= 256 ? 256 : 512;
-  static_assert(!kQT || kColQ + kQTmemChunks * 32 <= kColO, "TMEM columns overlap");
 };
 
 struct Bars {  // offsets (in 8-byte words) of the mbarriers from Layout::kBars
   enum {
-    q_full = 0,   // Q of the current tile in smem (staging + resident half)
-    q_tmem = 1,   // the TMEM half of Q is in place (128 arrivals)
+    q_full = 0,   // Q of the current tile in smem
     q_empty = 2,  // the last S of a tile is done: Q may be replaced
     o_last = 3,   // the last PV of a tile is done
     o_free = 4,   // the epilogue warps have read O out of TMEM (128 arrivals)
@@ -158,8 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
-                      RowIntervals rows, const __nv_bfloat16* __restrict__ q_hat,
-                      __nv_bfloat16* __restrict__ out, int T_,
+                      RowIntervals rows, __nv_bfloat16* __restrict__ out, int T_,
                       int Hq, int Hkv, int layer_type, int window, float scale_log2, int gp_log2,
                       int n_work, int* status) {
   using Ly = Layout<D>;
@@ -191,7 +184,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar(Bars::q_full), 1);
-    mbar_init(bar(Bars::q_tmem), 4 * 32);
     mbar_init(bar(Bars::q_empty), 1);
     mbar_init(bar(Bars::o_last), 1);
     mbar_init(bar(Bars::o_free), 4 * 32);
@@ -283,8 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           constexpr uint32_t idesc_s = idesc_bf16(BM, BN, 0, 0);
           const uint64_t dq0 = desc_sw128(base + Ly::kQ, 16, 1024);
           const uint64_t dk0 = desc_sw128(base + Ly::kK, 16, 1024);
-          ok = mbar_wait(bar(Bars::q_full), k & 1, abort) &&
-               mbar_wait(bar(Bars::q_tmem), k & 1, abort);
+          ok = mbar_wait(bar(Bars::q_full), k & 1, abort);
           for (int j = 0; ok && j < ti.n; ++j, ++g) {
             const int s = g % kStagesK;
             // the K tile first: it lands well ahead, so the wait that gates
@@ -299,13 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kc = 0; kc < D / 16; ++kc) {
               const int c = kc >> 2, sub = kc & 3;
-              const uint64_t bd = desc_add(dk, c * Ly::kKVChunk + sub * 32);
-              if (c < Ly::kQTmemChunks) {  // A from TMEM: 16 dims = 8 packed columns per step
-                mma_ts(d, tmem + Ly::kColQ + kc * 8, bd, idesc_s, kc > 0 ? 1u : 0u);
-              } else {
-                mma_ss(d, desc_add(dq0, (c - Ly::kQTmemChunks) * Ly::kQChunk + sub * 32), bd,
-                       idesc_s, kc > 0 ? 1u : 0u);
-              }
+              mma_ss(d, desc_add(dq0, c * Ly::kQChunk + sub * 32),
+                     desc_add(dk, c * Ly::kKVChunk + sub * 32), idesc_s, kc > 0 ? 1u : 0u);
             }
             mma_commit(bar(Bars::s_full + g % kNS));
             mma_commit(bar(Bars::k_empty + s));
@@ -465,41 +451,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       TileInfo ti{};
       if (has) {
         ti = info(t);
-        const int i = ti.p0 + (r >> gp_log2);
-        const int hrow = ti.h0 + (r & ((1 << gp_log2) - 1));
-        // the TMEM half of this row of Q, read ahead of the wait below
-        uint32_t qw[Ly::kQTmemChunks * 32 + 1];
-        if constexpr (Ly::kQT) {
-          const uint4* src =
-              reinterpret_cast<const uint4*>(q_hat + (((long)ti.b * T_ + i) * Hq + hrow) * D);
-#pragma unroll
-          for (int e = 0; e < Ly::kQTmemChunks * 8; ++e) {
-            const uint4 v = i < T_ ? src[e] : make_uint4(0, 0, 0, 0);
-            qw[4 * e] = v.x;
-            qw[4 * e + 1] = v.y;
-            qw[4 * e + 2] = v.z;
-            qw[4 * e + 3] = v.w;
-          }
-        }
         // Q of tile k replaces tile k - 1's once the last S of tile k - 1 is done
         if (k > 0)
           ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::q_empty), (k - 1) & 1, abort));
         if (!ok) break;
-        if (leader) {  // the shared-memory half by TMA
-          mbar_arrive_expect_tx(bar(Bars::q_full), (Ly::kChunks - Ly::kQTmemChunks) * BM * 128);
-          for (int c = Ly::kQTmemChunks; c < Ly::kChunks; ++c)
-            tma_load_4d(base + Ly::kQ + (c - Ly::kQTmemChunks) * Ly::kQChunk, &tm_q,
-                        bar(Bars::q_full), c * 64, ti.h0, ti.p0, ti.b);
+        if (leader) {
+          mbar_arrive_expect_tx(bar(Bars::q_full), Ly::kChunks * BM * 128);
+          for (int c = 0; c < Ly::kChunks; ++c)
+            tma_load_4d(base + Ly::kQ + c * Ly::kQChunk, &tm_q, bar(Bars::q_full), c * 64, ti.h0,
+                        ti.p0, ti.b);
         }
-        if constexpr (Ly::kQT) {
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < Ly::kQTmemChunks; ++c)
-            tmem_st32(tmem + lane_off + Ly::kColQ + 32 * c, qw + 32 * c);
-          tmem_wait_st();
-        }
-        tc_fence_before();
-        mbar_arrive(bar(Bars::q_tmem));
       }
       if (k > 0) {
         // ---- epilogue of tile k - 1: O / l as bf16, each thread its row
@@ -643,7 +604,6 @@ cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc 
   cfg.dynamicSmemBytes = Ly::kAlloc;
   cfg.stream = s;
   e = cudaLaunchKernelEx(&cfg, attn_sm100_kernel<D>, tq, tk, tv, rows,
-                         static_cast<const __nv_bfloat16*>(q_hat),
                          static_cast<__nv_bfloat16*>(out), T, L.Hq, L.Hkv, L.layer_type, L.window,
                          scale_log2, gp_log2, n_work, status);
   if (e != cudaSuccess) return e;

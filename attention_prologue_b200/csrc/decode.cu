@@ -166,12 +166,17 @@ __global__ void __launch_bounds__(128)
   const long base = ((long)b * Hq + h) * nc;
   float M = -INFINITY;
   for (int c = 0; c < cnt; ++c) M = fmaxf(M, part_ml[2 * (base + c)]);
+  // a chunk with m = -inf (no key, or a split CTA that gave up) weighs 0
+  auto weight = [&](int c) {
+    const float m = part_ml[2 * (base + c)];
+    return m == -INFINITY ? 0.f : expf(m - M);
+  };
   float den = 0.f;
-  for (int c = 0; c < cnt; ++c) den += expf(part_ml[2 * (base + c)] - M) * part_ml[2 * (base + c) + 1];
-  const float inv = 1.f / den;
+  for (int c = 0; c < cnt; ++c) den += weight(c) * part_ml[2 * (base + c) + 1];
+  const float inv = den > 0.f ? 1.f / den : 0.f;  // no key at all: a zero output
   for (int dim = threadIdx.x; dim < D; dim += blockDim.x) {
     float acc = 0.f;
-    for (int c = 0; c < cnt; ++c) acc += expf(part_ml[2 * (base + c)] - M) * part_o[(base + c) * D + dim];
+    for (int c = 0; c < cnt; ++c) acc += weight(c) * part_o[(base + c) * D + dim];
     dst[dim] = from_f<T>(acc * inv);
   }
 }

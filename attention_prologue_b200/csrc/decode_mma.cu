@@ -271,7 +271,18 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
   }
   __syncthreads();  // every tile consumed: no copy is in flight, the ring can be reused
   if (*abort) {
+    // an empty partial (m = -inf, l = 0, o~ = 0): the combine then ignores
+    // this chunk instead of reading what an earlier call left in the buffer
     if (threadIdx.x == 0) record_status(status, G4ATTN_EDEVICE);
+    for (int e = threadIdx.x; e < g * D; e += blockDim.x) {
+      const int h = e / D, dim = e - h * D;
+      const long pidx = ((long)b * Hq + kvh * g + h) * nc + c;
+      part_o[pidx * D + dim] = 0.f;
+      if (dim == 0) {
+        part_ml[2 * pidx] = -INFINITY;
+        part_ml[2 * pidx + 1] = 0.f;
+      }
+    }
     return;
   }
   // merge the 4 warps' partial softmaxes (each relative to its own maxima)

@@ -7,10 +7,12 @@
 //
 // The array is kDecodeScratchBytes (16 MiB) of device memory on every GPU
 // that loads the library, held until the process exits.  All calls on a
-// device share it and it keeps whatever the last call left there; the decode
-// kernels write every partial before the combine reads it, so nothing has to
-// start at zero.  Calls whose kernels overlap on the GPU (two streams, or two
-// host threads) race on the array and must be serialised by the caller.
+// device share it and it keeps whatever the last call left there; every
+// split CTA writes its partials before the combine reads them (a CTA that
+// gives up on a bounded wait writes an empty partial, which the combine
+// ignores), so nothing has to start at zero.  Calls whose kernels overlap on
+// the GPU (two streams, or two host threads) race on the array and must be
+// serialised by the caller.
 #include <mutex>
 
 #include "g4attn.h"
@@ -24,17 +26,24 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBy
 
 // Device address of g_decode_scratch on the current device.  The host-side
 // name of the array is only a stand-in, so the address is looked up once per
-// device (with that device current) and cached; nullptr if the lookup fails.
+// device (with that device current) and cached, keyed on the id of the
+// device's current context: after the context is destroyed and re-created
+// (cudaDeviceReset) the array lives elsewhere and is looked up again.
+// nullptr if the lookup fails.
 static float* decode_scratch_ptr() {
   static std::mutex mu;
+  static unsigned long long ids[64] = {0};
   static void* ptrs[64] = {nullptr};
   int dev = 0;
+  unsigned long long id = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!current_context_id(&id)) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
+  if (!ptrs[dev] || ids[dev] != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return nullptr;
     ptrs[dev] = p;
+    ids[dev] = id;
   }
   return static_cast<float*>(ptrs[dev]);
 }

@@ -120,6 +120,10 @@ bool make_bf16_map(CUtensorMap_st* m, const void* ptr, int rank, const uint64_t*
 // Device status word of the current device (nullptr if it cannot be found).
 int* status_ptr();
 
+// Unique id of the current CUDA context (false if there is none or the
+// driver cannot say); caches of device addresses are keyed on it.
+bool current_context_id(unsigned long long* id);
+
 // Kernel launches counter (incremented by every launcher).
 void count_launch(int n = 1);
 

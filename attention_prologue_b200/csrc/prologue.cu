@@ -16,16 +16,22 @@ namespace g4 {
 
 __device__ int g_status;  // first error recorded by a kernel, 0 = none
 
+// Device address of g_status in the current context, looked up once per
+// context (the host-side name of a __device__ variable is only a stand-in).
 int* status_ptr() {
   static std::mutex mu;
+  static unsigned long long ids[64] = {0};
   static int* ptrs[64] = {nullptr};
   int dev = 0;
+  unsigned long long id = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!current_context_id(&id)) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
+  if (!ptrs[dev] || ids[dev] != id) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess || !p) return nullptr;
     ptrs[dev] = static_cast<int*>(p);
+    ids[dev] = id;
   }
   return ptrs[dev];
 }

@@ -1,24 +1,28 @@
 """Benchmark of the Gemma 4 attention layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-decode] [--decode-only] [--decode-batch B]
-                    [--no-e2e] [--no-cpu-baseline]
+                    [--workload NAME] [--no-extra-prefill] [--no-decode] [--decode-only]
+                    [--decode-batch B] [--no-e2e] [--no-cpu-baseline]
 
 Headline: prefill attention TFLOP/s counting unmasked FLOPs only
 (4 * d * sum_i |I_i| * Hq * B; 2d for QK^T and 2d for PV per allowed pair) on
 the E2B-shaped sliding layer (B 1, T 8192, 8 query heads on 1 KV head, head
 dim 256, window 512), one g4attn_prefill call (prologue included) per step.
-The same JSON line carries the second half of the metric, decode KV-cache
-GB/s on the 26B-A4B-shaped step (64 sequences, cache lengths uniform in
-[4096, 131072]; a sliding layer on a 1024-slot rolling cache, a K=V global
-layer and a KV-shared layer reading it).
+The same JSON line carries the other prefill workloads under "prefill" (the
+12B-shaped multimodal sliding layer and the 31B-shaped K=V global layer at
+head_dim 512, each with its own roofline and CPU baseline), and the second
+half of the metric, decode KV-cache GB/s on the 26B-A4B-shaped step (64
+sequences, cache lengths uniform in [4096, 131072]; a sliding layer on a
+1024-slot rolling cache, a K=V global layer and a KV-shared layer reading it),
+under "decode".
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream; L2 is flushed (a 256 MiB write) before every timed
 prefill step, outside the events; the decode step reads ~36 GB, far more than
 L2.  Barrier + synchronize on both sides; the maximum over ranks is reported.
 With N > 1 every rank runs its own instance (independent sequences, no
-collective on the data path): weak scaling.
+collective on the data path): weak scaling.  NVML clock samples (1 ms
+period) are taken over every timed region.
 
 --impl reference times the float64 CPU oracle (the only other implementation
 of this layer) on the same workload and metric, on a bounded row sample.
@@ -143,9 +147,10 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, index: int, period_s: float = 0.001, paused: bool = False):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
+        self._paused = paused
         self._period = period_s
         self._index = index
         self._t = None
@@ -161,6 +166,9 @@ class ClockSampler:
     def _run(self):
         nv = self._nv
         while not self._stop.is_set():
+            if self._paused:
+                time.sleep(self._period)
+                continue
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
                 r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
@@ -182,11 +190,22 @@ class ClockSampler:
         if self._t:
             self._t.join()
 
-    def summary(self):
+    def pause(self):
+        """Stop sampling (between timed regions) until resume()."""
+        self._paused = True
+
+    def resume(self):
+        self._paused = False
+
+    def summary(self, ms_per_step: float | None = None):
         if not self.samples:
             return None
-        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        mhz = float(statistics.median(self.samples))
+        out = {"sm_mhz": mhz, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+               "samples": len(self.samples)}
+        if ms_per_step is not None:  # SM clock cycles per step at the median clock
+            out["mcycles_per_step"] = ms_per_step * mhz / 1e3
+        return out
 
 
 def visible_index(local_rank: int) -> int:
@@ -263,10 +282,29 @@ def made_events(n):
 # ---------------------------------------------------------------------------
 # prefill
 
-def bench_prefill(args, dist: Dist, pk: dict):
-    w = W.PREFILL_WORKLOADS[args.workload]
-    if args.seq_len:  # a shorter prompt of the same layer (profiling runs)
-        w = W.scaled_down(w, T=args.seq_len)
+# committed ncu summaries of the attention kernel, by workload: (file, the
+# workload the capture ran, how its traffic maps onto a full launch)
+PROFILES = {
+    W.E2B_SLIDING.name: ("attn_sm100_e2b_sliding.md", "same"),
+    W.G12B_SLIDING_MM.name: ("attn_sm100_12b_sliding_mm.md", "same"),
+    W.G31B_GLOBAL.name: ("attn_pair_31b_global.md", "same"),
+}
+
+
+def prefill_traffic(w: W.PrefillWorkload):
+    """DRAM bytes per launch of the attention kernel on this workload, from a
+    committed capture of the same kernel source on the same workload."""
+    prof = PROFILES.get(w.name)
+    if prof is None:
+        return None
+    return profile_field(prof[0], "traffic_bytes_per_launch")
+
+
+def bench_prefill(args, dist: Dist, pk: dict, w: W.PrefillWorkload, clk: ClockSampler,
+                  e2e: bool, steps: int):
+    """One g4attn_prefill call per step on workload w (CUDA graph replay),
+    then the attention kernel alone (events the library records around it),
+    then optionally the same call end to end from pinned host memory."""
     dev = torch.device("cuda", dist.local)
     inp = W.prefill_inputs(w, dev, seed=dist.rank)
     d = desc_of(w.layer)
@@ -283,7 +321,7 @@ def bench_prefill(args, dist: Dist, pk: dict):
 
     for _ in range(args.warmup):
         step()
-    K = args.steps
+    K = steps
     s0, s1, a0, a1 = (made_events(K) for _ in range(4))
     # One step as a CUDA graph (the library's launches of one g4attn_prefill
     # call), replayed K times: no host launch gaps inside the timed steps.
@@ -301,19 +339,21 @@ def bench_prefill(args, dist: Dist, pk: dict):
     torch.cuda.synchronize()
     dist.barrier()
     launches0 = G.g4attn_launch_count()
-    with ClockSampler(visible_index(dist.local)) as clk:
-        torch.cuda.synchronize()
-        dist.barrier()
-        for i in range(K):
-            flush.fill_(i & 0xFF)
-            s0[i].record(stream)
-            if graph is None:
-                step()
-            else:
-                graph.replay()
-            s1[i].record(stream)
-        torch.cuda.synchronize()
-        dist.barrier()
+    n_clk = len(clk.samples)
+    clk.resume()
+    torch.cuda.synchronize()
+    dist.barrier()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        s0[i].record(stream)
+        if graph is None:
+            step()
+        else:
+            graph.replay()
+        s1[i].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk_steps = len(clk.samples) - n_clk
     launches = (G.g4attn_launch_count() - launches0 if graph is None
                 else per_step_launches * K)
     step_ms = [s0[i].elapsed_time(s1[i]) for i in range(K)]
@@ -324,6 +364,7 @@ def bench_prefill(args, dist: Dist, pk: dict):
         G.g4attn_time_next_attention(a0[i], a1[i])
         step()
     torch.cuda.synchronize()
+    clk.pause()
     attn_ms = [a0[i].elapsed_time(a1[i]) for i in range(K)]
     total_ms = dist.max(sum(step_ms))
     value = job_rate(dist.world, flops, K, total_ms) / 1e12
@@ -334,16 +375,18 @@ def bench_prefill(args, dist: Dist, pk: dict):
         raise RuntimeError(f"device status after prefill: {G.g4attn_status_string(status)}")
 
     peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    kernel = "attn_pair_kernel" if w.layer.head_dim == 512 else "attn_sm100_kernel"
     res = dict(
-        value=value, ms_per_step=total_ms / K, flops=flops, launches=launches,
-        clocks=clk.summary(),
-        roofline={"bound": "tensor", "kernel": "attention (g4attn_prefill)", "achieved": achieved,
-                  "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                  "traffic": profiled_traffic("attn_sm100_e2b_sliding.md", w.name,
-                                              W.E2B_SLIDING.name),
+        metric="prefill attn TFLOP/s (unmasked)", value=value, unit="TFLOP/s",
+        ms_per_step=total_ms / K, steps=K, flops=flops, launches=launches,
+        clock_samples_in_steps=clk_steps,
+        roofline={"bound": "tensor", "kernel": f"{kernel} (g4attn_prefill)",
+                  "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                  "frac": achieved / peak, "traffic": prefill_traffic(w),
                   "algorithmic_per_launch": flops, "avg_launch_ms": attn_avg},
         e2e=None, inputs=inp, workload=w, graph=graph is not None)
-    if args.no_e2e:
+    if not e2e:
+        del flush, ws, graph
         return res
 
     # end to end: host (pinned) inputs -> device, prefill, output -> host
@@ -367,24 +410,39 @@ def bench_prefill(args, dist: Dist, pk: dict):
     e0, e1 = made_events(K), made_events(K)
     torch.cuda.synchronize()
     dist.barrier()
+    clk.resume()
     for i in range(K):
         flush.fill_(i & 0xFF)
         e0[i].record(stream)
         e2e_step()
         e1[i].record(stream)
     torch.cuda.synchronize()
+    clk.pause()
     e2e_ms = dist.max(sum(e0[i].elapsed_time(e1[i]) for i in range(K)))
     e2e_value = job_rate(dist.world, flops, K, e2e_ms) / 1e12
     res["e2e"] = {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                   "d2h_bytes_per_step": d2h}
-    del flush, ws
+    del flush, ws, graph
     return res
+
+
+def public_prefill(res: dict) -> dict:
+    """A prefill leg as it goes into the JSON line (no tensors)."""
+    w = res["workload"]
+    out = {k: v for k, v in res.items() if k not in ("inputs", "workload", "graph", "e2e")}
+    out["workload"] = w.name
+    out["config"] = {"global_batch": w.B, "seq_len": w.T,
+                     "heads": [w.layer.num_heads, w.layer.num_kv_heads],
+                     "head_dim": w.layer.head_dim, "window": w.layer.window,
+                     "image_blocks": [w.n_blocks, w.block_len] if w.n_blocks else None,
+                     "k_eq_v": w.layer.k_eq_v}
+    return out
 
 
 # ---------------------------------------------------------------------------
 # decode
 
-def bench_decode(args, dist: Dist, pk: dict):
+def bench_decode(args, dist: Dist, pk: dict, clk: ClockSampler):
     from dataclasses import replace
     w = W.A4B_DECODE if not args.decode_batch else replace(W.A4B_DECODE, batch=args.decode_batch)
     dev = torch.device("cuda", dist.local)
@@ -431,13 +489,16 @@ def bench_decode(args, dist: Dist, pk: dict):
     torch.cuda.synchronize()
     dist.barrier()
     launches0 = G.g4attn_launch_count()
-    with ClockSampler(visible_index(dist.local)) as clk:
-        for i in range(K):
-            reset()
-            s0[i].record(stream)
-            step((a0[i], a1[i]))
-            s1[i].record(stream)
-        torch.cuda.synchronize()
+    n_clk = len(clk.samples)
+    clk.resume()
+    for i in range(K):
+        reset()
+        s0[i].record(stream)
+        step((a0[i], a1[i]))
+        s1[i].record(stream)
+    torch.cuda.synchronize()
+    clk.pause()
+    clk_steps = len(clk.samples) - n_clk
     dist.barrier()
     launches = G.g4attn_launch_count() - launches0
     total_ms = dist.max(sum(s0[i].elapsed_time(s1[i]) for i in range(K)))
@@ -462,66 +523,148 @@ def bench_decode(args, dist: Dist, pk: dict):
                         "frac": achieved / peak, "frac_of_8000": achieved / 8000.0,
                         "traffic": traffic, "algorithmic_per_launch": g_split_bytes,
                         "avg_launch_ms": g_ms},
-           "gpu_launches": launches, "clocks": clk.summary()}
+           "gpu_launches": launches, "clock_samples_in_steps": clk_steps, "cpu_baseline": None}
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = decode_cpu_baseline(w, lens, (S, s_tok, s_cache), (Gl, g_tok, g_cache),
+                                                  (X, x_tok))
     del g_cache, s_cache
     torch.cuda.empty_cache()
     return res
 
 
+def decode_cpu_baseline(w, lens, s_state, g_state, x_state, n_global_seqs=4):
+    """The float64 oracle's decode of the same step on the host cores: the
+    sliding layer for every sequence, the global and KV-shared layers for a
+    few sequences (copying a 131072-position cache to the host is ~0.5 GB per
+    sequence); GB/s = the attended cache bytes of what was computed / its
+    time.  The caches hold the new token already (the step appended it)."""
+    import oracle
+    oracle.build()
+    threads = oracle.default_threads()
+    S, s_tok, s_cache = s_state
+    Gl, g_tok, g_cache = g_state
+    X, x_tok = x_state
+    post = np.asarray(lens, np.int64) + 1  # after the append
+
+    def olayer(L):
+        return oracle.Layer(layer_type=L.layer_type, window=L.window,
+                            rotary_fraction=L.rotary_fraction, rope_theta=L.rope_theta,
+                            k_eq_v=L.k_eq_v, num_heads=L.num_heads,
+                            num_kv_heads=L.num_kv_heads, head_dim=L.head_dim,
+                            softmax_scale=L.scale, rms_eps=L.rms_eps)
+
+    secs, nbytes = 0.0, 0.0
+    # sliding layer, all sequences (rolling cache of `window` slots)
+    ck, cv = s_cache.k.cpu(), s_cache.v.cpu()
+    t0 = time.perf_counter()
+    oracle.decode(olayer(S), s_tok["q_raw"].cpu(), s_tok["q_norm_w"].cpu(), ck, cv,
+                  s_cache.capacity, True, post, nthreads=threads)
+    secs += time.perf_counter() - t0
+    nbytes += decode_bytes(S, lens)
+    # global and KV-shared layers: the first n sequences
+    sel = list(range(n_global_seqs))
+    n_max = int(post[sel].max())
+    ck = g_cache.k[sel][:, :, :n_max].cpu()
+    cv = g_cache.v[sel][:, :, :n_max].cpu()
+    for L, tok in ((Gl, g_tok), (X, x_tok)):
+        t0 = time.perf_counter()
+        oracle.decode(olayer(L), tok["q_raw"][sel].cpu(), tok["q_norm_w"].cpu(), ck, cv, n_max,
+                      False, post[sel], nthreads=threads)
+        secs += time.perf_counter() - t0
+        nbytes += decode_bytes(L, np.asarray(lens)[sel])
+    return {"value": nbytes / secs / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{w.name}: sliding layer all {w.batch} sequences, global and KV-shared "
+                      f"layers the first {n_global_seqs} sequences ({nbytes / 1e9:.2f} GB of "
+                      f"attended K/V, {secs:.1f} s); float64 C, {threads} threads"}
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline leg and the reference arm)
 
-def oracle_sample(w: W.PrefillWorkload, inp: dict, stride: int, threads: int):
-    """Oracle on every `stride`-th query row (all heads, all sequences), plus
-    its key/value prologue charged pro rata.  Returns (TFLOP/s, seconds, rows)."""
+def row_pairs(w: W.PrefillWorkload, ids, rows) -> float:
+    """sum over sequences and the given rows of |I_i| (image blocks included)."""
+    L, T = w.layer, w.T
+    i = np.asarray(rows, np.int64)
+    if L.layer_type == W.GLOBAL:
+        return float(w.B * (i + 1).sum())
+    total = 0
+    for b in range(w.B):
+        lo = np.maximum(0, i - L.window + 1)
+        hi = i.copy()
+        if ids is not None:
+            row = ids[b].cpu().numpy()
+            for n, r in enumerate(rows):
+                if row[r] >= 0:
+                    s = r
+                    while s > 0 and row[s - 1] == row[r]:
+                        s -= 1
+                    e = r
+                    while e + 1 < T and row[e + 1] == row[r]:
+                        e += 1
+                    lo[n] = min(lo[n], s)
+                    hi[n] = e
+        total += int((hi - lo + 1).sum())
+    return float(total)
+
+
+def oracle_layer_of(L: W.LayerShape):
     import oracle
-    cpu = {k: (v.cpu() if v is not None else None) for k, v in inp.items()}
-    ol = oracle.Layer(layer_type=w.layer.layer_type, window=w.layer.window,
-                      rotary_fraction=w.layer.rotary_fraction, rope_theta=w.layer.rope_theta,
-                      k_eq_v=w.layer.k_eq_v, num_heads=w.layer.num_heads,
-                      num_kv_heads=w.layer.num_kv_heads, head_dim=w.layer.head_dim,
-                      softmax_scale=w.layer.scale, rms_eps=w.layer.rms_eps)
+    return oracle.Layer(layer_type=L.layer_type, window=L.window,
+                        rotary_fraction=L.rotary_fraction, rope_theta=L.rope_theta,
+                        k_eq_v=L.k_eq_v, num_heads=L.num_heads, num_kv_heads=L.num_kv_heads,
+                        head_dim=L.head_dim, softmax_scale=L.scale, rms_eps=L.rms_eps)
+
+
+def cpu_inputs(inp: dict) -> dict:
+    return {k: (v.cpu() if v is not None else None) for k, v in inp.items()}
+
+
+def oracle_sample(w: W.PrefillWorkload, cpu: dict, stride: int, threads: int, kv=None):
+    """Oracle on every `stride`-th query row (all heads, all sequences), plus
+    its key/value prologue charged pro rata.  Returns (TFLOP/s, seconds,
+    rows, (khat, vhat))."""
+    import oracle
+    ol = oracle_layer_of(w.layer)
     t0 = time.perf_counter()
-    kh, vh = oracle.prefill_kv(ol, cpu["k_raw"], cpu["v_raw"], cpu["k_norm_w"], threads)
+    if kv is None:
+        kv = oracle.prefill_kv(ol, cpu["k_raw"], cpu["v_raw"], cpu["k_norm_w"], threads)
     t_kv = time.perf_counter() - t0
+    kh, vh = kv
     rows = list(range(0, w.T, stride))
     ids = cpu["image_block_ids"]
     t0 = time.perf_counter()
     oracle.prefill_rows(ol, cpu["q_raw"], cpu["q_norm_w"], kh, vh,
                         None if ids is None else ids.numpy(), rows, threads)
     t_rows = time.perf_counter() - t0
-    i = np.asarray(rows, np.int64)
-    if w.layer.layer_type == W.GLOBAL:
-        pairs = w.B * (i + 1).sum()
-    else:
-        pairs = w.B * (i - np.maximum(0, i - w.layer.window + 1) + 1).sum()
-    flops = 4.0 * w.layer.head_dim * w.layer.num_heads * float(pairs)
+    flops = 4.0 * w.layer.head_dim * w.layer.num_heads * row_pairs(w, ids, rows)
     secs = t_rows + t_kv * len(rows) / w.T
-    return flops / secs / 1e12, secs, len(rows)
+    return flops / secs / 1e12, secs, len(rows), kv
 
 
-def pick_stride(w, inp, threads, target_s):
-    """Row stride whose sample takes about target_s seconds (calibrated)."""
+def pick_stride(w, cpu, threads, target_s):
+    """Row stride whose sample takes about target_s seconds (calibrated on a
+    64-row probe; returns the probe's key/value prologue for reuse)."""
     probe = max(1, w.T // 64)
-    _, secs, _ = oracle_sample(w, inp, probe, threads)
-    per_row = secs / math.ceil(w.T / probe)
-    return max(1, int(math.ceil(w.T * per_row / target_s)))
+    _, secs, n, kv = oracle_sample(w, cpu, probe, threads)
+    per_row = secs / n
+    return max(1, int(math.ceil(w.T * per_row / target_s))), kv
 
 
 def rows_phrase(stride: int) -> str:
     return "every query row" if stride == 1 else f"every {stride}th query row"
 
 
-def cpu_baseline(w, inp, target_s=12.0):
+def cpu_baseline(w, inp, target_s=10.0):
     import oracle
     oracle.build()
     threads = oracle.default_threads()
-    stride = pick_stride(w, inp, threads, target_s)
-    v, secs, n = oracle_sample(w, inp, stride, threads)
+    cpu = cpu_inputs(inp)
+    stride, kv = pick_stride(w, cpu, threads, target_s)
+    v, secs, n, _ = oracle_sample(w, cpu, stride, threads)
     return {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{w.name}: {rows_phrase(stride)} ({n} rows x {w.layer.num_heads} heads, "
-                      f"{secs:.1f} s) plus the K/V prologue charged pro rata; float64 C, "
-                      f"{threads} threads"}
+            "sample": f"{w.name}: {rows_phrase(stride)} ({n} rows x {w.layer.num_heads} heads x "
+                      f"{w.B} sequences, {secs:.1f} s) plus the K/V prologue charged pro rata; "
+                      f"TFLOP/s of the unmasked pairs of those rows; float64 C, {threads} threads"}
 
 
 def run_reference(args, dist: Dist):
@@ -530,15 +673,15 @@ def run_reference(args, dist: Dist):
     import oracle
     oracle.build()
     w = W.E2B_SLIDING
-    inp = W.prefill_inputs(w, "cpu", seed=0)
+    cpu = cpu_inputs(W.prefill_inputs(w, "cpu", seed=0))
     threads = oracle.default_threads()
     per_step = min(10.0, 150.0 / max(1, args.steps + args.warmup))
-    stride = pick_stride(w, inp, threads, per_step)
+    stride, kv = pick_stride(w, cpu, threads, per_step)
     for _ in range(args.warmup):
-        oracle_sample(w, inp, stride, threads)
+        oracle_sample(w, cpu, stride, threads)
     vals, secs = [], 0.0
     for _ in range(args.steps):
-        v, s, n = oracle_sample(w, inp, stride, threads)
+        v, s, n, _ = oracle_sample(w, cpu, stride, threads)
         vals.append(v)
         secs += s
     value = float(np.mean(vals))
@@ -562,15 +705,21 @@ def run_reference(args, dist: Dist):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    # 200 steps: the prefill's timed region (~30 ms) then spans several NVML
-    # clock samples; the decode half takes ~1.2 s
+    # 200 steps: the headline prefill's timed region (~15 ms) then spans many
+    # NVML clock samples; the other legs take at most as many steps as
+    # --extra-steps (the 31B global layer runs ~50 ms a step)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--extra-steps", type=int, default=10,
+                    help="timed steps of the other prefill workloads and of decode (at most "
+                         "--steps)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=W.E2B_SLIDING.name,
                     choices=[n for n in W.PREFILL_WORKLOADS if not n.startswith("tiny")])
     ap.add_argument("--seq-len", type=int, default=0,
                     help="override the prefill workload's prompt length (profiling runs)")
+    ap.add_argument("--no-extra-prefill", action="store_true",
+                    help="only the headline prefill workload")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true")
     ap.add_argument("--decode-batch", type=int, default=0,
@@ -591,30 +740,60 @@ def main(argv=None):
     torch.cuda.set_device(dist.local)
     G.lib()  # fail loudly if the CUDA library is missing
     pk, pk_src = peaks()
-    if args.decode_only:
-        dec = bench_decode(args, dist, pk)
-        dec["roofline"]["peak_source"] = f"{pk_src}: hbm_gbs"
-        if dist.rank == 0:
-            line = {"metric": METRIC, "value": dec["value"], "unit": "GB/s", "n_gpus": dist.world,
-                    "steps": args.steps, "warmup": args.warmup,
-                    "ms_per_step": dec["ms_per_step"], "higher_is_better": True,
-                    "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                    "config": {"workload": dec["workload"], "global_batch": dec["batch"] * dist.world},
-                    "roofline": dec["roofline"], "cpu_baseline": None, "e2e": None,
-                    "gpu_launches": dec["gpu_launches"], "clocks": dec["clocks"], "decode": dec}
-            print(json.dumps(line), flush=True)
-        dist.close()
-        return 0
-    pre = bench_prefill(args, dist, pk)
-    dec = None if args.no_decode else bench_decode(args, dist, pk)
-    cpu = None
-    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(pre["workload"], pre["inputs"])
-    w = pre["workload"]
+    extra_steps = max(1, min(args.steps, args.extra_steps))
+    want_cpu = dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline
+    with ClockSampler(visible_index(dist.local), paused=True) as clk:
+        if args.decode_only:
+            dec = bench_decode(args, dist, pk, clk)
+            dec["roofline"]["peak_source"] = f"{pk_src}: hbm_gbs"
+            dec["clocks"] = clk.summary(dec["ms_per_step"])
+            if dist.rank == 0:
+                line = {"metric": METRIC, "value": dec["value"], "unit": "GB/s",
+                        "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+                        "ms_per_step": dec["ms_per_step"], "higher_is_better": True,
+                        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                        "data": "synthetic",
+                        "config": {"workload": dec["workload"],
+                                   "global_batch": dec["batch"] * dist.world},
+                        "roofline": dec["roofline"], "cpu_baseline": dec["cpu_baseline"],
+                        "e2e": None, "gpu_launches": dec["gpu_launches"], "clocks": dec["clocks"],
+                        "decode": dec}
+                print(json.dumps(line), flush=True)
+            dist.close()
+            return 0
+
+        # the headline workload
+        w = W.PREFILL_WORKLOADS[args.workload]
+        if args.seq_len:  # a shorter prompt of the same layer (profiling runs)
+            w = W.scaled_down(w, T=args.seq_len)
+        pre = bench_prefill(args, dist, pk, w, clk, e2e=not args.no_e2e, steps=args.steps)
+        head_clocks = clk.summary(pre["ms_per_step"])
+        cpu = cpu_baseline(pre["workload"], pre["inputs"]) if want_cpu else None
+        pre.pop("inputs")
+        # the other prefill workloads (their own roofline and CPU baseline)
+        legs = {}
+        if not args.no_extra_prefill and not args.seq_len:
+            for name, ow in W.PREFILL_WORKLOADS.items():
+                if name.startswith("tiny") or name == w.name:
+                    continue
+                torch.cuda.empty_cache()
+                res = bench_prefill(args, dist, pk, ow, clk, e2e=False, steps=extra_steps)
+                res["roofline"]["peak_source"] = f"{pk_src}: bf16_tflops (burst)"
+                res["cpu_baseline"] = cpu_baseline(ow, res["inputs"]) if want_cpu else None
+                res.pop("inputs")
+                legs[name] = public_prefill(res)
+                del res
+                torch.cuda.empty_cache()
+        dec = None
+        if not args.no_decode:
+            dargs = argparse.Namespace(**{**vars(args), "steps": extra_steps})
+            dec = bench_decode(dargs, dist, pk, clk)
+            dec["roofline"]["peak_source"] = f"{pk_src}: hbm_gbs"
     roof = dict(pre["roofline"])
     roof["peak_source"] = f"{pk_src}: bf16_tflops (burst)"
-    if dec:
-        dec["roofline"]["peak_source"] = f"{pk_src}: hbm_gbs"
+    clocks = head_clocks or {}
+    clocks = dict(clocks, samples_in_headline_steps=pre["clock_samples_in_steps"],
+                  samples_all_timed_regions=len(clk.samples)) if clocks else None
     line = {"metric": METRIC, "value": pre["value"], "unit": "TFLOP/s", "n_gpus": dist.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -628,7 +807,7 @@ def main(argv=None):
                                else "one g4attn_prefill call (eager)",
                        "unmasked_gflop_per_step": pre["flops"] / 1e9},
             "roofline": roof, "cpu_baseline": cpu, "e2e": pre["e2e"],
-            "gpu_launches": pre["launches"], "clocks": pre["clocks"], "decode": dec}
+            "gpu_launches": pre["launches"], "clocks": clocks, "prefill": legs, "decode": dec}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()

@@ -100,7 +100,8 @@ typedef struct {
   int k_eq_v;            /* 1: V derives from the K projection (v_raw NULL) */
   int num_heads;         /* Hq, query heads */
   int num_kv_heads;      /* Hkv, divides Hq */
-  int head_dim;          /* d: 64, 128, 256 or 512 */
+  int head_dim;          /* d: 64, 128, 256 or 512 (other even sizes:
+                            G4ATTN_EUNSUPPORTED) */
   float softmax_scale;
   float rms_eps;
   int dtype;             /* G4ATTN_BF16 or G4ATTN_FP32 */
@@ -159,12 +160,16 @@ size_t g4attn_decode_workspace_size(const g4attn_layer_desc *desc,
  *                  256-byte aligned; its contents are not preserved.
  *  stream          cudaStream_t.
  *
- * Errors: G4ATTN_EINVAL for bad shapes, NULLs, head_dim not in
- * {64,128,256,512}, num_heads % num_kv_heads != 0, window <= 0 on a sliding
- * layer, rotary_fraction * d not an even integer, cache shape or dtype
- * mismatch, a rolling cache on a global layer; G4ATTN_ECACHE_OVERFLOW for a
- * non-rolling cache with capacity < T; G4ATTN_EWORKSPACE; G4ATTN_ECUDA if a
- * launch fails.  Nothing is written when an error is returned. */
+ * Errors: G4ATTN_EINVAL for bad shapes, NULLs, an odd or non-positive
+ * head_dim, num_heads % num_kv_heads != 0, window <= 0 on a sliding layer,
+ * rotary_fraction * d not an even integer, cache shape or dtype mismatch, a
+ * rolling cache on a global layer; G4ATTN_EUNSUPPORTED for a head_dim other
+ * than 64, 128, 256 or 512 or more than 32 KV heads; G4ATTN_ECACHE_OVERFLOW
+ * for a non-rolling cache with capacity < T; G4ATTN_EWORKSPACE; G4ATTN_ECUDA
+ * if a launch fails.  Nothing is written when an error is returned.
+ * image_block_ids are not checked: every maximal run of one non-negative id
+ * is a block, so an id that appears in two separate runs makes two blocks
+ * (not an error). */
 int g4attn_prefill(const g4attn_layer_desc *desc, int B, int T,
                    const void *q_raw, const void *k_raw, const void *v_raw,
                    const void *q_norm_w, const void *k_norm_w,

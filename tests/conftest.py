@@ -24,3 +24,18 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """The errors of every GPU-vs-oracle comparison of the run."""
+    try:
+        from helpers import STATS
+    except ImportError:  # pragma: no cover
+        return
+    if not STATS:
+        return
+    tr = terminalreporter
+    tr.section("parity errors against the float64 oracle")
+    for what, s in STATS:
+        tr.write_line(f"{what:<60s} max_abs {s['max_abs']:.3e}  mean_abs {s['mean_abs']:.3e}  "
+                      f"rel {s['rel']:.3e}")

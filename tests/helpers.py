@@ -18,6 +18,9 @@ BF16_MAX_ABS = 2e-2
 BF16_MEAN_ABS = 2e-3
 FP32_REL = 1e-5
 
+# every comparison's errors, printed at the end of the run (conftest.py)
+STATS: list[tuple[str, dict]] = []
+
 
 def desc_of(L: W.LayerShape, dtype: torch.dtype) -> G.LayerDesc:
     return G.make_desc(L.layer_type, L.num_heads, L.num_kv_heads, L.head_dim, window=L.window,
@@ -39,6 +42,7 @@ def check(got: torch.Tensor, ref: np.ndarray, dtype: torch.dtype, what: str = ""
     err = np.abs(g - ref)
     stats = dict(max_abs=float(err.max()), mean_abs=float(err.mean()),
                  rel=float(err.max() / max(np.abs(ref).max(), 1e-300)))
+    STATS.append((what, stats))
     if dtype == torch.float32:
         assert stats["rel"] <= FP32_REL, f"{what}: {stats}"
     else:

@@ -57,8 +57,9 @@ def ccache(d, B=1, C=64, rolling=0, **kw):
 
 
 @pytest.mark.parametrize("bad", [
-    dict(head_dim=96), dict(head_dim=1024), dict(num_heads=6, num_kv_heads=4),
-    dict(num_kv_heads=0), dict(num_heads=64, num_kv_heads=64), dict(window=0),
+    dict(head_dim=0, softmax_scale=1.0), dict(head_dim=-64, softmax_scale=1.0),
+    dict(head_dim=63), dict(num_heads=6, num_kv_heads=4),
+    dict(num_kv_heads=0), dict(window=0),
     dict(rotary_fraction=0.3), dict(rotary_fraction=1.5), dict(rope_theta=-1.0),
     dict(rms_eps=-1.0), dict(softmax_scale=float("inf")), dict(softmax_scale=0.0),
     dict(softmax_scale=-0.5), dict(layer_type=2),
@@ -67,6 +68,18 @@ def test_bad_descriptors_are_rejected(bad):
     d = desc(**bad)
     assert prefill_rc(d) == G.G4ATTN_EINVAL
     assert G.lib().g4attn_prefill_workspace_size(ctypes.byref(d), 1, 16) == 0
+
+
+@pytest.mark.parametrize("shape", [dict(head_dim=96), dict(head_dim=1024),
+                                   dict(num_heads=64, num_kv_heads=64)])
+def test_valid_layers_without_a_kernel_are_unsupported(shape):
+    """Head sizes other than 64/128/256/512 and more than 32 KV heads are
+    layers the pages allow but the library has no kernel for."""
+    d = desc(**shape)
+    assert prefill_rc(d) == G.G4ATTN_EUNSUPPORTED
+    assert G.lib().g4attn_prefill_workspace_size(ctypes.byref(d), 1, 16) == 0
+    c = ccache(d)
+    assert G.lib().g4attn_decode_workspace_size(ctypes.byref(d), ctypes.byref(c)) == 0
 
 
 def test_bad_dtype_code_is_rejected():

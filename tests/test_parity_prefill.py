@@ -135,18 +135,88 @@ def test_kv_shared_prefill_reads_the_source_cache():
     check(out, ref, shared.dtype, "kv-shared")
 
 
+# -- softmax scale 1.0 on the tensor-core kernels -----------------------------
+# The README's reading ("QK-norm replaces 1/sqrt(d)") gives logits sqrt(d)
+# times larger than the 1/sqrt(d) scale: the exponentials are far more
+# sensitive to absolute score errors (the head_dim-512 kernel exchanges
+# partial scores between the two CTAs of a pair).
+
+SCALE_ONE = [
+    W.scaled_down(W.E2B_SLIDING, T=1000, softmax_scale=1.0),                 # d 256 sliding
+    W.PrefillWorkload("g256-scale1", W.global_(8, 2, 256, softmax_scale=1.0), 1, 700),
+    W.scaled_down(W.G31B_GLOBAL, T=700, num_heads=8, num_kv_heads=1, softmax_scale=1.0),
+    W.scaled_down(W.G31B_GLOBAL, T=1500, num_heads=16, num_kv_heads=2, softmax_scale=1.0),
+]
+
+
+@pytest.mark.parametrize("w", SCALE_ONE, ids=lambda w: w.name)
+def test_tensor_cores_at_scale_one(w):
+    run_case(w, seed=21)
+
+
+@pytest.mark.parametrize("hd,layer", [(256, "sliding"), (512, "global")])
+@pytest.mark.parametrize("mix", [0.5, 2.0])
+def test_tensor_cores_with_large_correlated_logits(hd, layer, mix):
+    """Each query is a key of an earlier position plus noise (std `mix`), at
+    scale 1.0: the top logits reach hundreds and near-ties between a few keys
+    decide each row."""
+    L = (W.sliding(8, 2, hd, 256, softmax_scale=1.0) if layer == "sliding"
+         else W.global_(8, 1, hd, softmax_scale=1.0))
+    w = W.PrefillWorkload(f"corr-{layer}-d{hd}-mix{mix}", L, 1, 900)
+    inp = W.prefill_inputs(w, DEV, 31)
+    g = torch.Generator(device=DEV)
+    g.manual_seed(32)
+    T, Hq, Hkv = w.T, L.num_heads, L.num_kv_heads
+    grp = Hq // Hkv
+    lo = 0 if layer == "global" else None
+    t = torch.arange(T, device=DEV)
+    for h in range(Hq):
+        back = torch.randint(0, 256, (T,), generator=g, device=DEV)
+        j = (t - back).clamp(min=0)
+        if lo is None:  # stay inside the window
+            j = torch.maximum(j, (t - L.window + 1).clamp(min=0))
+        noise = torch.randn(T, L.head_dim, generator=g, device=DEV) * mix
+        inp["q_raw"][0, :, h] = (inp["k_raw"][0, j, h // grp].float() + noise).bfloat16()
+    out = gpu_prefill(w, inp)
+    check(out, oracle_prefill(w, inp), w.dtype, w.name)
+
+
 # -- full-size workloads, sampled rows ----------------------------------------
 
-@pytest.mark.parametrize("w,n", [(W.E2B_SLIDING, 96), (W.G12B_SLIDING_MM, 64),
-                                 (W.G31B_GLOBAL, 24)], ids=lambda x: getattr(x, "name", str(x)))
-def test_full_size_sampled(w, n):
-    rows = sample_rows(w.T, n)
+def stratified_rows(T: int, every: int = 64) -> list[int]:
+    """First and last rows, every `every`-th position (the first row of each
+    64-key tile) and the row before it (the last of the previous tile), and
+    the rows around each 128-row work-tile boundary of the first tiles."""
+    rows = {0, 1, 2, T - 2, T - 1}
+    for p in range(0, T, every):
+        rows.update((p, max(0, p - 1)))
+    for p in range(0, min(T, 2048), 16):
+        rows.update((p, p + 15))
+    return sorted(r for r in rows if 0 <= r < T)
+
+
+def block_edge_rows(w) -> list[int]:
+    """Rows at both ends of every image block of every sequence."""
+    ids = W.make_block_ids(w.B, w.T, w.n_blocks, w.block_len, 0).numpy()
+    rows = set()
+    for b in range(w.B):
+        row = ids[b]
+        starts = [i for i in range(w.T) if row[i] >= 0 and (i == 0 or row[i - 1] != row[i])]
+        for s in starts:
+            rows.update((s - 1, s, s + 1, s + w.block_len - 1, s + w.block_len))
+    return sorted(r for r in rows if 0 <= r < w.T)
+
+
+@pytest.mark.parametrize("w", [W.E2B_SLIDING, W.G12B_SLIDING_MM, W.G31B_GLOBAL],
+                         ids=lambda w: w.name)
+def test_full_size_sampled(w):
+    if w is W.G31B_GLOBAL:
+        rows = stratified_rows(w.T)  # >= 512 rows over the whole prompt
+        assert len(rows) >= 512
+    else:
+        rows = sample_rows(w.T, 96)
     if w.n_blocks:
-        ids = W.make_block_ids(w.B, w.T, w.n_blocks, w.block_len, 0)[0].numpy()
-        starts = [i for i in range(w.T) if ids[i] >= 0 and (i == 0 or ids[i - 1] != ids[i])]
-        for s in starts:  # rows at both ends of each image block of sequence 0
-            rows += [s, s + 1, s + w.block_len - 1, s + w.block_len]
-        rows = sorted(set(rows))
+        rows = sorted(set(rows) | set(block_edge_rows(w)))
     run_case(w, seed=0, rows=rows)
 
 

@@ -13,10 +13,11 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from attention_prologue_b200 import g4attn as G
 from attention_prologue_b200 import workloads as W
 
-from helpers import BF16_MAX_ABS, BF16_MEAN_ABS, desc_of
+from helpers import BF16_MAX_ABS, BF16_MEAN_ABS, check, desc_of, oracle_layer
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -74,3 +75,51 @@ def test_decode_noalloc_rejects_a_batch_beyond_the_fixed_array():
     with pytest.raises(G.G4AttnError) as e:
         G.g4attn_decode_noalloc(d, cache, q, w)
     assert e.value.status == G.G4ATTN_EWORKSPACE
+
+
+def oracle_rows(L, tok, k_pre, v_pre, cap, lens, seqs):
+    """The float64 oracle's decode of the sampled sequences, from the cache
+    contents before the append and the new token's raw inputs."""
+    sel = torch.as_tensor(seqs)
+    return oracle.decode(oracle_layer(L), tok["q_raw"].cpu()[sel], tok["q_norm_w"].cpu(),
+                         k_pre, v_pre, cap, False, np.asarray(lens)[seqs],
+                         k_new=tok["k_raw"].cpu()[sel],
+                         v_new=None if tok["v_raw"] is None else tok["v_raw"].cpu()[sel],
+                         wk=tok["k_norm_w"].cpu())
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_decode_noalloc_reduced_chunk_plan_matches_the_oracle(dtype):
+    """When the usual chunk count does not fit the fixed array the keys are
+    cut into fewer, longer chunks: check that plan against the float64
+    oracle on sampled sequences.  bf16: the K=V global layer of the 26B-A4B
+    shape (64 sequences, 16 heads on 2 KV heads, 7 chunks of 4976 keys in
+    place of 17 of 2048; tensor-core split kernel).  fp32: 64 query heads on
+    one KV head, head_dim 64 (15 chunks of 2336 keys in place of 17; the
+    CUDA-core split kernel)."""
+    rng = np.random.default_rng(23)
+    if dtype == torch.bfloat16:
+        L, cap = W.global_(16, 2, 512), 32768
+    else:
+        L, cap = W.global_(64, 1, 64), 32768
+    B = 64
+    lens = rng.integers(1000, cap - 1, size=B).astype(np.int32)
+    lens[:2] = (cap - 1, 1)  # the longest span the plan must cover, and a single key
+    g = torch.Generator(device=DEV)
+    g.manual_seed(24)
+    tok = W.decode_token_inputs(L, B, g, DEV, dtype)
+    cache = G.KVCache.allocate(B, L.num_kv_heads, cap, L.head_dim, dtype=dtype, device=DEV)
+    W.fill_cache(cache.k, cache.v, lens, False, g)
+    cache.len.copy_(torch.as_tensor(lens, dtype=torch.int32))
+    seqs = [0, 1, 2, 17, 40, 63]
+    sel = torch.as_tensor(seqs, device=DEV)
+    k_pre, v_pre = cache.k[sel].cpu(), cache.v[sel].cpu()
+    d = desc_of(L, dtype)
+    G.g4attn_cache_append(d, cache, tok["k_raw"], tok["v_raw"], tok["k_norm_w"])
+    out = G.g4attn_decode_noalloc(d, cache, tok["q_raw"], tok["q_norm_w"])
+    again = G.g4attn_decode_noalloc(d, cache, tok["q_raw"], tok["q_norm_w"])
+    torch.cuda.synchronize()
+    assert G.g4attn_get_device_status() == G.G4ATTN_OK
+    assert torch.equal(out, again)
+    ref = oracle_rows(L, tok, k_pre, v_pre, cap, lens, seqs)
+    check(out[sel, 0], ref, dtype, f"decode_noalloc reduced plan {dtype}")
