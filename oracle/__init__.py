@@ -71,7 +71,8 @@ def _load():
         lib.or_prefill_chunk_rows.argtypes = [LP, I, I, I, P, P, I, I, P, P, P, P, I, P, I]
         lib.or_prefill_chunk_rows_masked.argtypes = [LP, I, I, I, P, P, I, I, P, P, P, P, P, I,
                                                      P, I]
-        lib.or_decode.argtypes = [LP, LP, P, P, I, I, P, P, I, I, I, P, P, P, P, P, I, P, I]
+        lib.or_decode.argtypes = [LP, LP, P, P, I, I, P, P, I, I, I, P, P, P, P, P, I, P, I, P,
+                                  I]
         lib.or_decode.restype = I
         lib.or_partial.argtypes = [P, P, P, L, I, I, I, D, P, P, P]
         lib.or_combine.argtypes = [I, P, P, P, I, P]
@@ -302,14 +303,16 @@ def prefill_chunk(layer: Layer, q_raw, k_raw, v_raw, wq, wk, khat_cache, vhat_ca
 
 def decode(layer_q: Layer, q_raw, wq, cache_k, cache_v, capacity: int, rolling: bool, lens,
            k_new=None, v_new=None, wk=None, layer_kv: Layer | None = None, seqs=None,
-           nthreads: int | None = None) -> np.ndarray:
+           nthreads: int | None = None, attention_mask=None) -> np.ndarray:
     """One decode step ("Gemma4ConditionalGenerate": decoding over the
     per-layer KV cache; "KV Cache": rolling sliding caches; "Shared KV
     Cache": a later layer reads an earlier layer's K/V).
 
     cache_k/cache_v [B, Hkv, C, d] hold positions 0..lens[b]-1.  With k_new the
     new token is appended at position lens[b]; without it (KV-shared layer) the
-    cache already holds it at lens[b]-1.  Returns float64 [n_seqs, Hq, d]."""
+    cache already holds it at lens[b]-1.  attention_mask [B, mask_len] (1 = keep,
+    0 = padding) drops the padding keys among positions 0..mask_len-1; later
+    positions are kept.  Returns float64 [n_seqs, Hq, d]."""
     q, dt = _raw(q_raw)
     w, wdt = _raw(wq)
     ck, cdt = _raw(cache_k)
@@ -322,11 +325,17 @@ def decode(layer_q: Layer, q_raw, wq, cache_k, cache_v, capacity: int, rolling: 
     B = lens.size
     n = B if seqs_a is None else seqs_a.size
     out = np.empty((n, layer_q.num_heads, layer_q.head_dim), np.float64)
+    keep, mask_len = None, 0
+    if attention_mask is not None:
+        keep = np.ascontiguousarray(np.asarray(attention_mask) != 0, np.uint8)
+        if keep.ndim != 2 or keep.shape[0] != B:
+            raise ValueError("attention_mask must be [B, mask_len]")
+        mask_len = keep.shape[1]
     lq = layer_q._c()
     lkv = (layer_kv or layer_q)._c()
     rc = _load().or_decode(ctypes.byref(lq), ctypes.byref(lkv), _p(q), _p(w), dt, wdt, _p(ck),
                            _p(cv), cdt, int(capacity), int(bool(rolling)), _p(lens), _p(kn),
-                           _p(vn), _p(wkk), _p(seqs_a), n, _p(out),
+                           _p(vn), _p(wkk), _p(keep), int(mask_len), _p(seqs_a), n, _p(out),
                            nthreads or default_threads())
     if rc != 0:
         raise ValueError("oracle decode: a key the query needs is not in the cache")

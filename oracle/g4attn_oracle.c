@@ -411,8 +411,12 @@ void or_prefill_rows(const or_layer *L, int B, int T, const void *q_raw,
  * layer reading a cache that already holds the new token) P = len[b] - 1.
  * The query (q_raw [B][Hq][d], prologue of Lq at position P) attends over
  * the interval of row P: decode is the last row of a prefill over P + 1
- * tokens.  out is [n_seqs][Hq][d].  Returns 0, or -1 if a key the query
- * needs is not in the cache. */
+ * tokens.  keep, when given, is the padding mask of the prompt positions,
+ * [B][mask_len] ("Gemma4ConditionalGenerate" arguments: attention_mask,
+ * 1 = keep, 0 = padding): position p < mask_len is dropped when its entry
+ * is 0; later positions (the generated tokens) are kept.  out is
+ * [n_seqs][Hq][d].  Returns 0, or -1 if a key the query needs is not in the
+ * cache. */
 typedef struct {
   const or_layer *Lq, *Lkv;
   const void *q_raw, *wq;
@@ -421,6 +425,8 @@ typedef struct {
   int cache_dtype, C, rolling;
   const int *len;
   const void *k_new, *v_new, *wk;
+  const unsigned char *keep; /* [B][mask_len] or NULL */
+  int mask_len;
   const int *seqs;
   int n_seqs;
   double *out;
@@ -465,8 +471,12 @@ static void *or_decode_worker(void *arg) {
     double *kk = (double *)malloc(sizeof(double) * n * d);
     double *vv = (double *)malloc(sizeof(double) * n * d);
     double *s = (double *)malloc(sizeof(double) * n);
+    unsigned char *kp = (unsigned char *)malloc(n); /* padding mask of lo..P */
     for (long p = lo; p <= P; ++p) {
       double *kd = kk + (p - lo) * d, *vd = vv + (p - lo) * d;
+      kp[p - lo] = (J->keep && p < J->mask_len)
+                       ? (J->keep[(long)b * J->mask_len + p] != 0)
+                       : 1;
       if (append && p == P) {
         memcpy(kd, kn, sizeof(double) * d);
         memcpy(vd, vn, sizeof(double) * d);
@@ -480,11 +490,11 @@ static void *or_decode_worker(void *arg) {
       }
     }
     or_attend(q, kk, vv, d, 0, (int)(n - 1), d, Lq->softmax_scale,
-              Lq->logit_softcap, NULL, s,
-              J->out + ((long)si * Hq + h) * d);
+              Lq->logit_softcap, kp, s, J->out + ((long)si * Hq + h) * d);
     free(kk);
     free(vv);
     free(s);
+    free(kp);
   }
   free(q);
   free(kn);
@@ -496,16 +506,16 @@ int or_decode(const or_layer *Lq, const or_layer *Lkv, const void *q_raw,
               const void *wq, int dtype, int w_dtype, const void *cache_k,
               const void *cache_v, int cache_dtype, int C, int rolling,
               const int *len, const void *k_new, const void *v_new,
-              const void *wk, const int *seqs, int n_seqs, double *out,
-              int nthreads) {
+              const void *wk, const unsigned char *keep, int mask_len,
+              const int *seqs, int n_seqs, double *out, int nthreads) {
   if (nthreads < 1) nthreads = 1;
   or_decode_job *jobs =
       (or_decode_job *)calloc(nthreads, sizeof(or_decode_job));
   for (int t = 0; t < nthreads; ++t) {
-    or_decode_job j = {Lq,      Lkv,   q_raw,       wq,    dtype,   w_dtype,
-                       cache_k, cache_v, cache_dtype, C,   rolling, len,
-                       k_new,   v_new, wk,          seqs,  n_seqs,  out,
-                       t,       nthreads, 0};
+    or_decode_job j = {Lq,      Lkv,     q_raw,       wq,    dtype,   w_dtype,
+                       cache_k, cache_v, cache_dtype, C,     rolling, len,
+                       k_new,   v_new,   wk,          keep,  mask_len, seqs,
+                       n_seqs,  out,     t,           nthreads, 0};
     jobs[t] = j;
   }
   or_run(or_decode_worker, jobs, sizeof(or_decode_job), nthreads);

@@ -672,3 +672,44 @@ def test_all_ones_padding_mask_changes_nothing():
     plain = oracle.prefill(L, q, k, v, wq, wk)
     masked = oracle.prefill(L, q, k, v, wq, wk, attention_mask=np.ones((2, 21), np.int32))
     np.testing.assert_array_equal(masked, plain)
+
+
+@pytest.mark.parametrize("case", ["sliding_left_pad", "global_holes_softcap", "rolling"])
+def test_masked_decode_equals_last_row_of_the_masked_prefill(case):
+    """Decode with the prompt's padding mask (positions past the mask are
+    generated tokens, always kept) is the last row of the masked prefill over
+    the prompt plus the new token."""
+    rng = np.random.default_rng(41)
+    T = 37  # cached positions; the new token sits at T
+    if case == "global_holes_softcap":
+        L = global_layer(logit_softcap=3.0)
+    else:
+        L = sliding_layer(window=12)
+    B = 2
+    q, k, v, wq, wk = inputs(L, B, T + 1, rng)
+    keep = np.ones((B, T), np.int32)
+    if case == "global_holes_softcap":
+        keep[0] = (rng.random(T) > 0.4)
+        keep[1, :20] = 0
+    else:
+        keep[0, :30] = 0  # left padding reaching into the last window
+        keep[1, 26:29] = 0
+    full = np.concatenate([keep, np.ones((B, 1), np.int32)], axis=1)
+    ref = oracle.prefill(L, q, k, v, wq, wk, attention_mask=full)[:, T]
+    kh, vh = oracle.prefill_kv(L, k[:, :T], None if v is None else v[:, :T], wk)
+    rolling = case == "rolling"
+    C = L.window if rolling else 64
+    out = oracle.decode(L, q[:, T:T + 1], wq, _cache_from(kh, C, rolling),
+                        _cache_from(vh, C, rolling), C, rolling, [T, T],
+                        k_new=k[:, T:T + 1], v_new=None if v is None else v[:, T:T + 1], wk=wk,
+                        attention_mask=keep)
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    # an all-ones mask is the unmasked decode, bit for bit
+    plain = oracle.decode(L, q[:, T:T + 1], wq, _cache_from(kh, C, rolling),
+                          _cache_from(vh, C, rolling), C, rolling, [T, T],
+                          k_new=k[:, T:T + 1], v_new=None if v is None else v[:, T:T + 1], wk=wk)
+    ones = oracle.decode(L, q[:, T:T + 1], wq, _cache_from(kh, C, rolling),
+                         _cache_from(vh, C, rolling), C, rolling, [T, T],
+                         k_new=k[:, T:T + 1], v_new=None if v is None else v[:, T:T + 1], wk=wk,
+                         attention_mask=np.ones((B, T), np.int32))
+    np.testing.assert_array_equal(ones, plain)
