@@ -73,6 +73,8 @@ def _load():
                                                      P, I]
         lib.or_decode.argtypes = [LP, LP, P, P, I, I, P, P, I, I, I, P, P, P, P, P, I, P, I, P,
                                   I]
+        lib.or_attend_rows.argtypes = [LP, I, I, I, P, P, P, P, P, P, I, P, I]
+        lib.or_prologue_q_all.argtypes = [LP, I, I, I, P, P, I, I, P]
         lib.or_decode.restype = I
         lib.or_partial.argtypes = [P, P, P, L, I, I, I, D, P, P, P]
         lib.or_combine.argtypes = [I, P, P, P, I, P]
@@ -284,6 +286,46 @@ def prefill_chunk_rows(layer: Layer, q_raw, wq, khat, vhat, p0: int, block_ids=N
     _load().or_prefill_chunk_rows_masked(ctypes.byref(c), B, T, int(p0), _p(q), _p(w), dt, wdt,
                                          _p(ids), _p(keep), _p(khat), _p(vhat), _p(rows_a),
                                          n_rows, _p(out), nthreads or default_threads())
+    return out
+
+
+def prologue_q_all(layer: Layer, q_raw, wq, p0: int = 0) -> np.ndarray:
+    """Post-prologue queries of every token, float64 [B, T, Hq, d], the
+    tokens at positions p0 .. p0 + T - 1 ("What changed": plain-weight
+    RMSNorm, zero-pad partial rope)."""
+    q, dt = _raw(q_raw)
+    w, wdt = _raw(wq)
+    B, T, Hq, d = q_raw.shape
+    out = np.empty((B, T, Hq, d), np.float64)
+    c = layer._c()
+    _load().or_prologue_q_all(ctypes.byref(c), B, T, int(p0), _p(q), _p(w), dt, wdt, _p(out))
+    return out
+
+
+def attend_rows(layer: Layer, qhat, khat, vhat, p0: int = 0, block_ids=None, rows=None,
+                nthreads: int | None = None, attention_mask=None) -> np.ndarray:
+    """The attention of prefill_chunk_rows from given post-prologue queries
+    qhat [B, T, Hq, d] (float64), keys/values khat/vhat [B, p0 + T, Hkv, d]:
+    the same intervals, padding, soft-cap and softmax.  For modelling a
+    storage format of the post-prologue vectors (round them, then attend).
+    Returns float64 [B, n_rows, Hq, d]."""
+    qhat = np.ascontiguousarray(qhat, np.float64)
+    B, T, Hq, d = qhat.shape
+    khat = np.ascontiguousarray(khat, np.float64)
+    vhat = np.ascontiguousarray(vhat, np.float64)
+    if khat.shape[1] != p0 + T or vhat.shape[1] != p0 + T:
+        raise ValueError("khat/vhat must hold positions 0 .. p0 + T - 1")
+    ids = _i32(block_ids)
+    rows_a = _i32(rows)
+    n_rows = T if rows_a is None else rows_a.size
+    keep = None
+    if attention_mask is not None:
+        keep = np.ascontiguousarray(np.asarray(attention_mask) != 0, np.uint8)
+    out = np.empty((B, n_rows, Hq, d), np.float64)
+    c = layer._c()
+    _load().or_attend_rows(ctypes.byref(c), B, T, int(p0), _p(qhat), _p(ids), _p(keep),
+                           _p(khat), _p(vhat), _p(rows_a), n_rows, _p(out),
+                           nthreads or default_threads())
     return out
 
 

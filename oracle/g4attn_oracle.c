@@ -253,6 +253,7 @@ typedef struct {
   const double *khat, *vhat; /* [B][p0 + T][Hkv][d] */
   double *out;               /* [B][n_rows][Hq][d] */
   int tid, nthreads;
+  const double *qhat;        /* [B][T][Hq][d] post-prologue queries, or NULL */
 } or_prefill_job;
 
 static void *or_prefill_worker(void *arg) {
@@ -271,7 +272,10 @@ static void *or_prefill_worker(void *arg) {
     int i = J->rows ? J->rows[r] : r; /* row of the chunk */
     int pos = J->p0 + i;
     long qoff = (((long)b * J->T + i) * Hq + h) * d;
-    or_prologue_q(L, J->q_raw, qoff, J->dtype, J->wq, J->w_dtype, pos, q);
+    if (J->qhat)
+      memcpy(q, J->qhat + qoff, sizeof(double) * d);
+    else
+      or_prologue_q(L, J->q_raw, qoff, J->dtype, J->wq, J->w_dtype, pos, q);
     int lo, hi;
     or_interval(L, J->block_ids ? J->block_ids + (long)b * Tk : NULL, Tk, pos,
                 &lo, &hi);
@@ -367,11 +371,44 @@ void or_prefill_chunk_rows_masked(const or_layer *L, int B, int T, int p0,
   for (int t = 0; t < nthreads; ++t) {
     or_prefill_job j = {L,     B,       T,         p0,   q_raw,  wq,
                         dtype, w_dtype, block_ids, keep, rows,   n_rows,
-                        khat,  vhat,    out,       t,    nthreads};
+                        khat,  vhat,    out,       t,    nthreads, NULL};
     jobs[t] = j;
   }
   or_run(or_prefill_worker, jobs, sizeof(or_prefill_job), nthreads);
   free(jobs);
+}
+
+/* The attention of or_prefill_chunk_rows_masked from given post-prologue
+ * queries qhat [B][T][Hq][d] (float64) instead of raw ones: the same row
+ * intervals, padding and soft-cap, the same loop.  Lets a caller model a
+ * storage format of q_hat, k_hat, v_hat (values rounded before they are
+ * attended), with every step after the prologue unchanged. */
+void or_attend_rows(const or_layer *L, int B, int T, int p0, const double *qhat,
+                    const int *block_ids, const unsigned char *keep,
+                    const double *khat, const double *vhat, const int *rows,
+                    int n_rows, double *out, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  or_prefill_job *jobs =
+      (or_prefill_job *)calloc(nthreads, sizeof(or_prefill_job));
+  for (int t = 0; t < nthreads; ++t) {
+    or_prefill_job j = {L,      B,    T,         p0,   NULL,   NULL,
+                        OR_FP64, OR_FP64, block_ids, keep, rows, n_rows,
+                        khat,   vhat, out,       t,    nthreads, qhat};
+    jobs[t] = j;
+  }
+  or_run(or_prefill_worker, jobs, sizeof(or_prefill_job), nthreads);
+  free(jobs);
+}
+
+/* Post-prologue queries RoPE_pos(RMSNorm(q) * w_q) of every token, float64
+ * [B][T][Hq][d], the tokens at positions p0 .. p0 + T - 1. */
+void or_prologue_q_all(const or_layer *L, int B, int T, int p0, const void *q_raw,
+                       const void *wq, int dtype, int w_dtype, double *out) {
+  int d = L->head_dim, Hq = L->num_heads;
+  for (long it = 0; it < (long)B * T * Hq; ++it) {
+    long t = (it / Hq) % T;
+    or_prologue_q(L, q_raw, it * d, dtype, wq, w_dtype, p0 + t, out + it * d);
+  }
 }
 
 /* The same with every key kept. */

@@ -713,3 +713,35 @@ def test_masked_decode_equals_last_row_of_the_masked_prefill(case):
                          k_new=k[:, T:T + 1], v_new=None if v is None else v[:, T:T + 1], wk=wk,
                          attention_mask=np.ones((B, T), np.int32))
     np.testing.assert_array_equal(ones, plain)
+
+
+@pytest.mark.parametrize("case", ["sliding_blocks_mask_softcap", "global_chunk"])
+def test_attend_rows_from_the_oracles_own_prologue_is_prefill(case):
+    """Attention from given post-prologue vectors, fed the oracle's own
+    q_hat / k_hat / v_hat, is the oracle's prefill bit for bit: the same
+    intervals, padding, soft-cap and softmax (so it inherits every pin of
+    the prefill path)."""
+    rng = np.random.default_rng(51)
+    if case == "sliding_blocks_mask_softcap":
+        L = sliding_layer(window=6, logit_softcap=1.5, num_heads=4, num_kv_heads=2)
+        T, p0 = 33, 0
+        ids = ids_with_blocks(2, T, [(4, 15), (20, 24)])
+        keep = (rng.random((2, T)) > 0.25).astype(np.int32)
+    else:
+        L = global_layer()
+        T, p0 = 17, 20
+        ids, keep = None, None
+    B = 2
+    q, k, v, wq, wk = inputs(L, B, p0 + T, rng)
+    kh, vh = oracle.prefill_kv(L, k, v, wk)
+    rows = [0, 3, T - 1]
+    want = oracle.prefill_chunk_rows(L, q[:, p0:], wq, kh, vh, p0, block_ids=ids, rows=rows,
+                                     attention_mask=keep)
+    qh = oracle.prologue_q_all(L, q[:, p0:], wq, p0)
+    got = oracle.attend_rows(L, qh, kh, vh, p0, block_ids=ids, rows=rows, attention_mask=keep)
+    np.testing.assert_array_equal(got, want)
+    # and each q_hat is the single-vector prologue at its position
+    for t in (0, T - 1):
+        np.testing.assert_array_equal(qh[1, t, 2 % L.num_heads],
+                                      oracle.prologue_q(L, q[1, p0 + t, 2 % L.num_heads], wq,
+                                                        p0 + t))
