@@ -82,6 +82,7 @@ static int make_cfg(const g4attn_layer_desc* d, LayerCfg* L) {
   if (!(d->rope_theta > 0.0) || !std::isfinite(d->rope_theta)) return G4ATTN_EINVAL;
   if (!(d->softmax_scale > 0.f) || !std::isfinite(d->softmax_scale)) return G4ATTN_EINVAL;
   if (!(d->rms_eps >= 0.f) || !std::isfinite(d->rms_eps)) return G4ATTN_EINVAL;
+  if (!(d->logit_softcap >= 0.f) || !std::isfinite(d->logit_softcap)) return G4ATTN_EINVAL;
   if (d->k_eq_v != 0 && d->k_eq_v != 1) return G4ATTN_EINVAL;
   // a valid layer without a kernel: head sizes other than 64/128/256/512, or
   // more than 32 KV heads (the cache append runs one warp per KV head in a
@@ -98,6 +99,7 @@ static int make_cfg(const g4attn_layer_desc* d, LayerCfg* L) {
   L->dtype = d->dtype;
   L->scale = d->softmax_scale;
   L->eps = d->rms_eps;
+  L->softcap = d->logit_softcap;
   std::memset(&L->rope, 0, sizeof(L->rope));
   L->rope.rotated_pairs = (int)(R2 / 2);
   for (int k = 0; k < L->rope.rotated_pairs; ++k)
@@ -112,16 +114,24 @@ static int check_cache(const LayerCfg& L, const g4attn_cache* c, int B) {
   if (c->capacity < 1 || (c->rolling != 0 && c->rolling != 1)) return G4ATTN_EINVAL;
   if (c->rolling && (L.layer_type != G4ATTN_SLIDING || c->capacity < L.window))
     return G4ATTN_EINVAL;
+  if (c->key_mask && c->mask_len < 0) return G4ATTN_EINVAL;
   return G4ATTN_OK;
+}
+
+static KeyMask cache_mask(const g4attn_cache* c) {
+  return c->key_mask ? KeyMask{c->key_mask, c->mask_len} : KeyMask{nullptr, 0};
 }
 
 // Workspace of one prefill call.
 struct PrefillWs {
-  size_t q_hat, kv, intervals, total;  // byte offsets / sizes
-  bool need_kv;                        // keys go to scratch (no usable cache)
+  size_t q_hat, kv, intervals, bits, total;  // byte offsets / sizes
+  bool need_kv;                              // keys go to scratch (no usable cache)
+  int words;                                 // 64-key words of the padding bits
 };
 
-static PrefillWs prefill_ws(const LayerCfg& L, int B, int T, bool need_kv, bool intervals) {
+// Tk: key positions the call's rows may see (T, or p0 + T for a chunk).
+static PrefillWs prefill_ws(const LayerCfg& L, int B, int T, bool need_kv, bool intervals,
+                            bool mask, int Tk) {
   PrefillWs w;
   const size_t es = elem_size(L.dtype);
   size_t off = 0;
@@ -131,9 +141,22 @@ static PrefillWs prefill_ws(const LayerCfg& L, int B, int T, bool need_kv, bool 
   if (need_kv) off += 2 * align256((size_t)B * T * L.Hkv * L.d * es);
   w.intervals = off;
   if (intervals) off += 2 * align256((size_t)B * T * sizeof(int32_t));
+  w.words = (Tk + 63) / 64;
+  w.bits = off;
+  if (mask) off += align256((size_t)B * w.words * sizeof(uint64_t));
   w.total = off;
   w.need_kv = need_kv;
   return w;
+}
+
+// The padding bits of a prefill call, or none.
+static cudaError_t padding_bits(const PrefillWs& w, char* ws, int B, int Tk, const uint8_t* mask,
+                                KeyBits* kb, cudaStream_t s) {
+  *kb = KeyBits{nullptr, 0};
+  if (!mask) return cudaSuccess;
+  uint64_t* bits = reinterpret_cast<uint64_t*>(ws + w.bits);
+  *kb = KeyBits{bits, w.words};
+  return launch_mask_bits(B, Tk, mask, bits, w.words, s);
 }
 
 }  // namespace g4
@@ -145,7 +168,7 @@ extern "C" {
 size_t g4attn_prefill_workspace_size(const g4attn_layer_desc* desc, int B, int T) {
   LayerCfg L;
   if (make_cfg(desc, &L) != G4ATTN_OK || B < 0 || T < 0) return 0;
-  return prefill_ws(L, B, T, true, L.layer_type == G4ATTN_SLIDING).total;
+  return prefill_ws(L, B, T, true, L.layer_type == G4ATTN_SLIDING, true, T).total;
 }
 
 size_t g4attn_decode_workspace_size(const g4attn_layer_desc* desc, const g4attn_cache* cache) {
@@ -157,8 +180,9 @@ size_t g4attn_decode_workspace_size(const g4attn_layer_desc* desc, const g4attn_
 
 int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_raw,
                    const void* k_raw, const void* v_raw, const void* q_norm_w,
-                   const void* k_norm_w, const int32_t* image_block_ids, g4attn_cache* cache,
-                   void* out, void* workspace, size_t ws_bytes, void* stream) {
+                   const void* k_norm_w, const int32_t* image_block_ids,
+                   const uint8_t* attention_mask, g4attn_cache* cache, void* out,
+                   void* workspace, size_t ws_bytes, void* stream) {
   LayerCfg L;
   int st = make_cfg(desc, &L);
   if (st != G4ATTN_OK) return st;
@@ -182,7 +206,7 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
   // slots 0..T-1, otherwise from scratch
   const bool cache_is_src = cache && cache->capacity >= T;
   const bool intervals = L.layer_type == G4ATTN_SLIDING && image_block_ids != nullptr;
-  PrefillWs w = prefill_ws(L, B, T, !cache_is_src, intervals);
+  PrefillWs w = prefill_ws(L, B, T, !cache_is_src, intervals, attention_mask != nullptr, T);
   if (!workspace || ws_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return G4ATTN_EWORKSPACE;
   char* ws = static_cast<char*>(workspace);
@@ -191,11 +215,11 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
 
   KVSrc src;
   if (cache_is_src) {
-    src = {cache->k, cache->v, cache->capacity};
+    src = {cache->k, cache->v, cache->capacity, T};
   } else {
     char* kbuf = ws + w.kv;
     char* vbuf = kbuf + align256((size_t)B * T * L.Hkv * L.d * es);
-    src = {kbuf, vbuf, T};
+    src = {kbuf, vbuf, T, T};
   }
   cudaError_t e = cudaSuccess;
   KVDst d0{nullptr, nullptr, 1, 0, 0}, d1{nullptr, nullptr, 1, 0, 0};
@@ -205,7 +229,7 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
       d1 = {cache->k, cache->v, cache->capacity, 1, T - cache->capacity};
   }
   void* q_hat = ws + w.q_hat;
-  e = launch_token_prologue(L, B, T, q_raw, q_norm_w, q_hat, shared ? nullptr : k_raw, v_raw,
+  e = launch_token_prologue(L, B, T, 0, q_raw, q_norm_w, q_hat, shared ? nullptr : k_raw, v_raw,
                             k_norm_w, d0, d1, (cache && !shared) ? cache->len : nullptr, s);
   if (e != cudaSuccess) return G4ATTN_ECUDA;
   RowIntervals rows{nullptr, nullptr};
@@ -217,12 +241,76 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
       return G4ATTN_ECUDA;
     rows = {lo, hi};
   }
+  KeyBits kb;
+  if (padding_bits(w, ws, B, T, attention_mask, &kb, s) != cudaSuccess) return G4ATTN_ECUDA;
   cudaEvent_t ev0, ev1;
   take_timing(&ev0, &ev1);
   if (ev0) cudaEventRecord(ev0, s);
   e = attention_sm100_supported(L)
-          ? launch_attention_sm100(L, B, T, q_hat, src, rows, out, status_ptr(), s)
-          : launch_attention_simt(L, B, T, q_hat, src, rows, out, s);
+          ? launch_attention_sm100(L, B, T, q_hat, src, rows, kb, out, status_ptr(), s)
+          : launch_attention_simt(L, B, T, q_hat, src, rows, kb, out, s);
+  if (ev1) cudaEventRecord(ev1, s);
+  return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
+}
+
+size_t g4attn_prefill_chunk_workspace_size(const g4attn_layer_desc* desc, int B, int T, int p0) {
+  LayerCfg L;
+  if (make_cfg(desc, &L) != G4ATTN_OK || B < 0 || T < 0 || p0 < 0) return 0;
+  return prefill_ws(L, B, T, false, true, true, p0 + T).total;
+}
+
+int g4attn_prefill_chunk(const g4attn_layer_desc* desc, int B, int T, int p0, const void* q_raw,
+                         const void* k_raw, const void* v_raw, const void* q_norm_w,
+                         const void* k_norm_w, const int32_t* image_block_ids,
+                         const uint8_t* attention_mask, g4attn_cache* cache, void* out,
+                         void* workspace, size_t ws_bytes, void* stream) {
+  LayerCfg L;
+  int st = make_cfg(desc, &L);
+  if (st != G4ATTN_OK) return st;
+  if (B < 0 || T < 0 || p0 < 0) return G4ATTN_EINVAL;
+  if (!q_raw || !q_norm_w || !out || !cache) return G4ATTN_EINVAL;
+  const bool shared = k_raw == nullptr;  // KV-shared layer: the chunk's keys are in the cache
+  if (shared) {
+    if (v_raw) return G4ATTN_EINVAL;
+  } else {
+    if (!k_norm_w) return G4ATTN_EINVAL;
+    if ((v_raw == nullptr) != (L.k_eq_v == 1)) return G4ATTN_EINVAL;
+  }
+  if ((st = check_cache(L, cache, B)) != G4ATTN_OK) return st;
+  if ((long)p0 + T > cache->capacity)  // every position must stay readable
+    return cache->rolling || shared ? G4ATTN_EINVAL : G4ATTN_ECACHE_OVERFLOW;
+  if (B == 0 || T == 0) return G4ATTN_OK;
+
+  PrefillWs w = prefill_ws(L, B, T, false, true, attention_mask != nullptr, p0 + T);
+  if (!workspace || ws_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return G4ATTN_EWORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* q_hat = ws + w.q_hat;
+  KVDst d0{nullptr, nullptr, 1, 0, 0}, d1{nullptr, nullptr, 1, 0, 0};
+  if (!shared) d0 = {cache->k, cache->v, cache->capacity, cache->rolling, 0};
+  cudaError_t e = launch_token_prologue(L, B, T, p0, q_raw, q_norm_w, q_hat,
+                                        shared ? nullptr : k_raw, v_raw, k_norm_w, d0, d1,
+                                        shared ? nullptr : cache->len, s);
+  if (e != cudaSuccess) return G4ATTN_ECUDA;
+  int32_t* lo = reinterpret_cast<int32_t*>(ws + w.intervals);
+  int32_t* hi =
+      reinterpret_cast<int32_t*>(ws + w.intervals + align256((size_t)B * T * sizeof(int32_t)));
+  e = launch_chunk_intervals(L, B, T, p0,
+                             L.layer_type == G4ATTN_SLIDING ? image_block_ids : nullptr, lo, hi,
+                             s);
+  if (e != cudaSuccess) return G4ATTN_ECUDA;
+  const KVSrc src{cache->k, cache->v, cache->capacity, p0 + T};
+  const RowIntervals rows{lo, hi};
+  KeyBits kb;
+  if (padding_bits(w, ws, B, p0 + T, attention_mask, &kb, s) != cudaSuccess)
+    return G4ATTN_ECUDA;
+  cudaEvent_t ev0, ev1;
+  take_timing(&ev0, &ev1);
+  if (ev0) cudaEventRecord(ev0, s);
+  e = attention_sm100_supported(L)
+          ? launch_attention_sm100(L, B, T, q_hat, src, rows, kb, out, status_ptr(), s)
+          : launch_attention_simt(L, B, T, q_hat, src, rows, kb, out, s);
   if (ev1) cudaEventRecord(ev1, s);
   return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
 }
@@ -258,7 +346,7 @@ int g4attn_decode(const g4attn_layer_desc* desc, const g4attn_cache* cache, cons
   cudaEvent_t ev0, ev1;
   take_timing(&ev0, &ev1);
   cudaError_t e = launch_decode(L, cache->batch, q_raw, q_norm_w, cache->k, cache->v, cache->len,
-                                cache->capacity, cache->rolling, plan,
+                                cache->capacity, cache->rolling, cache_mask(cache), plan,
                                 static_cast<float*>(workspace), out, status_ptr(),
                                 static_cast<cudaStream_t>(stream), ev0, ev1);
   return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
@@ -273,8 +361,8 @@ int g4attn_decode_noalloc(const g4attn_layer_desc* desc, const g4attn_cache* cac
   if ((st = check_cache(L, cache, cache->batch)) != G4ATTN_OK) return st;
   if (cache->batch == 0) return G4ATTN_OK;
   return launch_decode_noalloc(L, cache->batch, q_raw, q_norm_w, cache->k, cache->v, cache->len,
-                               cache->capacity, cache->rolling, out, status_ptr(),
-                               static_cast<cudaStream_t>(stream));
+                               cache->capacity, cache->rolling, cache_mask(cache), out,
+                               status_ptr(), static_cast<cudaStream_t>(stream));
 }
 
 int g4attn_get_device_status(void* stream) {

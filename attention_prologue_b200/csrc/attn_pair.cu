@@ -13,15 +13,17 @@
 //
 // DSMEM moves ~21 GB/s per direction and SM (about 0.8 us per 16 KB), so
 // the swap is the cost to minimise and to hide:
-//  - each partial goes as fp16, already in log2 units (times scale * log2 e)
-//    and clamped to the fp16 range: 16 KB per tile and direction.  A CTA
-//    adds the peer's fp16 partial to its own fp32 one, so the logits of the
-//    two CTAs differ by the fp16 rounding of one partial (at most 2^-11 of
-//    it, below the bf16 rounding of P); each CTA normalises its half of O
-//    with its own row sums, so each half is exactly consistent with its P.
-//    The fp16 values are decoded with integer and FMA instructions, not
-//    conversions: the transcendental/conversion pipe (16 per clock per SM)
-//    already carries exp2 and the bf16 packing of P.
+//  - each partial goes as a 16-bit integer, already in log2 units (times
+//    scale * log2 e), with one fp32 step per row and tile: q = round(y /
+//    step), step = max |y| / 32766 over the row's 64 keys -- 16 KB + 512 B
+//    per tile and direction.  A CTA adds the peer's decoded partial to its
+//    own fp32 one, so the logits of the two CTAs differ by at most step / 2
+//    (~1e-3 log2 units at softmax scale 1, ~1e-4 at 1/sqrt(d): at scale 1 an
+//    fp16 partial was 20x coarser and moved outputs by ~0.02).  Each CTA
+//    normalises its half of O with its own row sums, so each half is exactly
+//    consistent with its P.  Encoding and decoding use FMA and byte-permute
+//    instructions, no conversions: the transcendental/conversion pipe (16
+//    per clock per SM) already carries exp2 and the bf16 packing of P.
 //  - sender warps read and send each partial as soon as its MMA is done,
 //    while the softmax warps work on earlier tiles; the inbox has two slots.
 //  - the sends are st.async: the bytes complete the receiver's mbarrier, no
@@ -39,7 +41,7 @@
 //                  S_j  = Q K_j^T   (M 128, N 64, K 256; A half TMEM, half smem)
 //                  O   += P_j V_j   (M 128, N 256, K 64; P from TMEM)
 //                with S up to two tiles ahead of PV (three S buffers)
-//   warps 8..11  senders: own partial of S_j -> fp16 -> the peer's inbox
+//   warps 8..11  senders: own partial of S_j -> int16 + step -> the peer's inbox
 //   warps 4..7   softmax (lazy rescale when a row max grows by more than
 //                2^16): copy the TMEM half of Q in at the start; then per
 //                tile the own partial of S_j + the peer's,
@@ -81,9 +83,10 @@ constexpr uint32_t kQ = 0;                       // Q chunks 2, 3 (dims 128..255
 constexpr uint32_t kK = kQ + (kChunks - kQTmemChunks) * kQChunk;
 constexpr uint32_t kV = kK + kStagesK * kChunks * kKVChunk;  // also stages Q chunks 0, 1
 constexpr uint32_t kX = kV + kStagesV * kChunks * kKVChunk;  // inbox: the peer's partials
-constexpr uint32_t kXSlot = BM * BN * 2;                     // one tile of fp16 partials
-constexpr uint32_t kXWarp = kXSlot / 4;                      // the 32 rows of one warp
-constexpr uint32_t kBars = kX + kSlots * kXSlot;
+constexpr uint32_t kXSlot = BM * BN * 2;                     // one tile of int16 partials
+constexpr uint32_t kXS = kX + kSlots * kXSlot;               // inbox: the fp32 step of each row
+constexpr uint32_t kXWarp = kXSlot / 4 + 32 * 4;             // bytes of the 32 rows of one warp
+constexpr uint32_t kBars = kXS + kSlots * BM * 4;
 static_assert(kQTmemChunks * kQChunk <= kStagesV * kChunks * kKVChunk, "Q staging fits the V ring");
 constexpr uint32_t kAlloc = kBars + 512;
 static_assert(kAlloc <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
@@ -119,26 +122,39 @@ struct Scalars {
   int klo, khi;
 };
 
-// 64 fp32 partial scores -> 32 packed fp16 pairs in log2 units, clamped to
-// the finite fp16 range.
-__device__ __forceinline__ void pack_partial(const uint32_t* sr, float scale_log2, uint32_t* h) {
+// 64 fp32 partial scores -> log2 units y -> 32 packed pairs of 16-bit
+// integers q = round(y / step); returns step = max |y| / 32766.  The
+// rounding adds 1.5 * 2^23 in one FMA: the sum lies in [2^23, 2^24), where
+// the float's unit is 1, so its low 16 bits are q in two's complement.
+// (|y / step| <= 32766 (1 + 2^-22) also with the approximate reciprocal.)
+__device__ __forceinline__ float pack_partial(const uint32_t* sr, float scale_log2, uint32_t* h) {
+  float y[BN];
+  float amax = 1e-30f;
+#pragma unroll
+  for (int c = 0; c < BN; ++c) {
+    y[c] = __uint_as_float(sr[c]) * scale_log2;
+    amax = fmaxf(amax, fabsf(y[c]));
+  }
+  const float inv = 32766.f * rcp_approx(amax);
 #pragma unroll
   for (int e = 0; e < BN / 2; ++e) {
-    const float a = fminf(fmaxf(__uint_as_float(sr[2 * e]) * scale_log2, -65504.f), 65504.f);
-    const float c = fminf(fmaxf(__uint_as_float(sr[2 * e + 1]) * scale_log2, -65504.f), 65504.f);
-    __half2 v = __floats2half2_rn(a, c);
-    h[e] = *reinterpret_cast<uint32_t*>(&v);
+    const float f0 = fmaf(y[2 * e], inv, 12582912.f);
+    const float f1 = fmaf(y[2 * e + 1], inv, 12582912.f);
+    h[e] = __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x5410);
   }
+  return amax * (1.f / 32766.f);
 }
 
 }  // namespace
 
+// kExtras: the padding mask and the logit soft-cap are compiled in.
+template <bool kExtras>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v, RowIntervals rows,
+                     const __grid_constant__ CUtensorMap tm_v, RowIntervals rows, KeyBits kb,
                      __nv_bfloat16* __restrict__ out, int T_, int Hq, int Hkv, int layer_type,
-                     int window, float scale_log2, int gp_log2, int* status) {
+                     int window, float scale_log2, float cap2, int gp_log2, int* status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {  // the 128-byte-swizzle atoms need a 1024-byte base
     if (threadIdx.x == 0) record_status(status, G4ATTN_EDEVICE);
@@ -352,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       tc_fence_after();
       uint32_t h[BN / 2];
+      float step;
       {
         uint32_t sr[BN];
         tmem_ld32(tmem + lane_off + (j % kNS) * BN, sr);
@@ -359,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(Bars::s_read + j % kNS));
-        pack_partial(sr, scale_log2, h);
+        step = pack_partial(sr, scale_log2, h);
       }
       // the peer has consumed this warp's rows of tile j - kSlots from the slot
       const int sl = j % kSlots;
@@ -373,6 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; q < BN / 8; ++q)
         st_async_v4(map_peer(slot + ((q ^ (r & 7)) << 4), peer), rbar, h[4 * q], h[4 * q + 1],
                     h[4 * q + 2], h[4 * q + 3]);
+      st_async_b32(map_peer(base + kXS + ((uint32_t)sl * BM + r) * 4, peer), rbar,
+                   __float_as_uint(step));
     }
     // the peer's last accesses to this CTA are its acknowledgements of the
     // last tiles: wait for them (bounded) before the shared memory goes
@@ -408,6 +427,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int j = 0; j < n_tiles; ++j) {
       const int sb = j % kNS;
+      // the padding bits of this key tile (all kept without a mask), read
+      // before the wait so the load overlaps it
+      const uint64_t keep =
+          (kExtras && kb.bits) ? kb.bits[(long)b * kb.words + kt0 + j] : ~0ull;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::s_full + sb), (j / kNS) & 1, abort));
       if (!ok) break;
       tc_fence_after();
@@ -417,26 +440,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_off + sb * BN, sr);
         tmem_ld32(tmem + lane_off + sb * BN + 32, sr + 32);
         tmem_wait_ld();
-        // + the peer's partial of S_j (fp16 pairs, already in log2 units)
+        // + the peer's partial of S_j (int16 pairs and a step, in log2 units)
         ok = __all_sync(0xffffffffu, mbar_wait_cluster(bar(Bars::rx_full + 4 * (j % kSlots) + sw),
                                                         (j / kSlots) & 1, abort));
         if (!ok) break;
         const uint4* in = reinterpret_cast<const uint4*>(smem_raw + kX + (j % kSlots) * kXSlot +
                                                          r * (BN * 2));
+        const float step =
+            *reinterpret_cast<const float*>(smem_raw + kXS + ((j % kSlots) * BM + r) * 4);
 #pragma unroll
         for (int q = 0; q < BN / 8; ++q) {
           const uint4 v = in[q ^ (r & 7)];
           const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            // fp16 -> fp32 exactly (subnormals too): move sign, exponent and
-            // mantissa into fp32 position and rescale the exponent by 2^112
-            const uint32_t lo = ((w[e] & 0x7fffu) << 13) | ((w[e] & 0x8000u) << 16);
-            const uint32_t hi = ((w[e] >> 3) & 0x0fffe000u) | (w[e] & 0x80000000u);
+            // int16 q -> float exactly: flip the sign bits (q + 32768 in
+            // [0, 65535]), place each half below the exponent of 2^23, then
+            // subtract 2^23 + 32768
+            const uint32_t u = w[e] ^ 0x80008000u;
+            const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7610)) - 8421376.f;
+            const float f1 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7632)) - 8421376.f;
             const int c = 8 * q + 2 * e;
-            x[c] = fmaf(__uint_as_float(lo), 0x1p112f, __uint_as_float(sr[c]) * scale_log2);
-            x[c + 1] =
-                fmaf(__uint_as_float(hi), 0x1p112f, __uint_as_float(sr[c + 1]) * scale_log2);
+            x[c] = fmaf(f0, step, __uint_as_float(sr[c]) * scale_log2);
+            x[c + 1] = fmaf(f1, step, __uint_as_float(sr[c + 1]) * scale_log2);
           }
         }
       }
@@ -448,16 +474,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(bar(Bars::rx_full + 4 * (j % kSlots) + sw), kXWarp);
         mbar_arrive_remote(peer_tx + 32u * (uint32_t)(j % kSlots));
       }
-      // x: logits of S_j in log2 units
+      // x: logits of S_j in log2 units (soft-capped there when asked)
+      if (kExtras && cap2 > 0.f) {
+        const float k = 1.f / cap2;
+#pragma unroll
+        for (int c = 0; c < BN; ++c) x[c] = cap2 * tanh_fast(x[c] * k);
+      }
       const int key0 = (kt0 + j) * BN;
       float mt = -INFINITY;
-      if (key0 >= lo && key0 + BN - 1 <= hi) {
+      if (key0 >= lo && key0 + BN - 1 <= hi && (!kExtras || keep == ~0ull)) {
 #pragma unroll
         for (int c = 0; c < BN; ++c) mt = fmaxf(mt, x[c]);
       } else {
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
-          x[c] = (key0 + c >= lo && key0 + c <= hi) ? x[c] : -INFINITY;
+          x[c] = (key0 + c >= lo && key0 + c <= hi && (!kExtras || ((keep >> c) & 1))) ? x[c]
+                                                                                     : -INFINITY;
           mt = fmaxf(mt, x[c]);
         }
       }
@@ -495,9 +527,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int e = 0; e < BN / 2; ++e) {
         const float e0 = ex2_approx(x[2 * e] + neg_m);
         const float e1 = ex2_approx(x[2 * e + 1] + neg_m);
-        rs += e0 + e1;
         __nv_bfloat162 bb = __floats2bfloat162_rn(e0, e1);
         pk[e] = *reinterpret_cast<uint32_t*>(&bb);
+        // the row sum adds the P values the PV product multiplies (bf16)
+        rs += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
       }
       // P_j overwrites S_j: the senders must have read it
       ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::s_read + sb), (j / kNS) & 1, abort));
@@ -547,7 +580,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 cudaError_t launch_attention_pair(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
-                                  RowIntervals rows, void* out, int* status, cudaStream_t s) {
+                                  RowIntervals rows, KeyBits kb, void* out, int* status,
+                                  cudaStream_t s) {
   if (L.d != 2 * DH) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
   const int gp_log2 = gqa_pack_log2(L.Hq, L.Hkv);
@@ -558,15 +592,16 @@ cudaError_t launch_attention_pair(const LayerCfg& L, int B, int T, const void* q
     const uint32_t box[4] = {64, (uint32_t)(1 << gp_log2), (uint32_t)(BM >> gp_log2), 1};
     if (!make_bf16_map(&tq, q_hat, 4, dims, str, box)) return cudaErrorInvalidValue;
   }
-  {  // K, V [B * Hkv, cap, 512]; rows at positions >= T read as zero
-    const uint64_t dims[3] = {D, (uint64_t)T, (uint64_t)B * L.Hkv};
+  {  // K, V [B * Hkv, cap, 512]; rows at positions >= kv.len read as zero
+    const uint64_t dims[3] = {D, (uint64_t)kv.len, (uint64_t)B * L.Hkv};
     const uint64_t str[2] = {D * es, (uint64_t)kv.cap * D * es};
     const uint32_t box[3] = {64, BN, 1};
     if (!make_bf16_map(&tk, kv.k, 3, dims, str, box)) return cudaErrorInvalidValue;
     if (!make_bf16_map(&tv, kv.v, 3, dims, str, box)) return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(attn_pair_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kAlloc);
+  const bool extras = kb.bits != nullptr || L.softcap > 0.f;
+  auto kern = extras ? attn_pair_kernel<true> : attn_pair_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kAlloc);
   if (e != cudaSuccess) return e;
   const float scale_log2 = L.scale * 1.4426950408889634f;
   const int bp = BM >> gp_log2;
@@ -582,9 +617,9 @@ cudaError_t launch_attention_pair(const LayerCfg& L, int B, int T, const void* q
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, attn_pair_kernel, tq, tk, tv, rows,
+  e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, rows, kb,
                          static_cast<__nv_bfloat16*>(out), T, L.Hq, L.Hkv, L.layer_type,
-                         L.window, scale_log2, gp_log2, status);
+                         L.window, scale_log2, softcap_log2(L), gp_log2, status);
   if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();

@@ -6,6 +6,10 @@
 //                                       "Sliding-window attention")
 //   image blocks  window U block        ("Gemma 4" Keras docs, "What changed")
 //   global rows   [0, i]                (overview blog, "Global attention layers")
+//   padding keys  dropped               ("Gemma 4" Keras docs,
+//                                        "Gemma4ConditionalGenerate": attention_mask)
+// with an optional logit soft-cap s -> c tanh(s / c) ("gemma4-pt-claude"
+// README, "Attention Backend Notes").  A row left without any key outputs 0.
 // Key tiles outside the union of a CTA's row intervals are never visited.
 //
 // CTA = (32 query rows, one query head, one sequence); 8 warps x 4 rows.
@@ -26,8 +30,9 @@ constexpr size_t simt_smem_bytes() {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
-    attn_simt_kernel(const T* __restrict__ q_hat, KVSrc kv, RowIntervals rows, T* __restrict__ out,
-                     int T_, int Hq, int Hkv, int layer_type, int window, float scale) {
+    attn_simt_kernel(const T* __restrict__ q_hat, KVSrc kv, RowIntervals rows, KeyBits kb,
+                     T* __restrict__ out, int T_, int Hq, int Hkv, int layer_type, int window,
+                     float scale, float cap) {
   extern __shared__ float smem[];
   float* sq = smem;                      // [rows][D]
   float* sk = sq + kSimtRows * D;        // [keys][D + 1] (padded: lane j reads row j)
@@ -104,7 +109,8 @@ __global__ void __launch_bounds__(256)
       const int lo = s_lo[r], hi = s_hi[r];
       if (lo > hi || hi < t0 || lo >= t0 + kSimtKeys) continue;  // warp-uniform
       const int key = t0 + lane;
-      const bool ok = key >= lo && key <= hi;
+      const bool ok = key >= lo && key <= hi &&
+                      (!kb.bits || ((kb.bits[(long)b * kb.words + (key >> 6)] >> (key & 63)) & 1));
       float s = -INFINITY;
       if (ok) {
         const float* qr = sq + r * D;
@@ -113,10 +119,12 @@ __global__ void __launch_bounds__(256)
 #pragma unroll 8
         for (int c = 0; c < D; ++c) dot = fmaf(qr[c], kr[c], dot);
         s = dot * scale;
+        if (cap > 0.f) s = cap * tanhf(s / cap);
       }
       const float mn = fmaxf(m[rr], warp_max(s));
+      if (mn == -INFINITY) continue;  // no key of this row so far (warp-uniform)
       const float p = ok ? expf(s - mn) : 0.f;
-      const float corr = expf(m[rr] - mn);
+      const float corr = m[rr] == -INFINITY ? 0.f : expf(m[rr] - mn);
       l[rr] = l[rr] * corr + warp_sum(p);
       m[rr] = mn;
 #pragma unroll
@@ -133,8 +141,8 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
   for (int rr = 0; rr < kSimtRowsPerWarp; ++rr) {
     const int r = warp * kSimtRowsPerWarp + rr, i = r0 + r;
-    if (i >= T_ || s_lo[r] > s_hi[r]) continue;
-    const float inv = 1.f / l[rr];
+    if (i >= T_) continue;
+    const float inv = l[rr] > 0.f ? 1.f / l[rr] : 0.f;  // no key: a zero row
     T* dst = out + (((long)b * T_ + i) * Hq + h) * D;
 #pragma unroll
     for (int c = 0; c < C; ++c) dst[lane + 32 * c] = from_f<T>(o[rr][c] * inv);
@@ -143,31 +151,31 @@ __global__ void __launch_bounds__(256)
 
 template <typename E, int D>
 static cudaError_t run_simt(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
-                            RowIntervals rows, void* out, cudaStream_t s) {
+                            RowIntervals rows, KeyBits kb, void* out, cudaStream_t s) {
   constexpr size_t smem = simt_smem_bytes<D>();
   cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<E, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((T + kSimtRows - 1) / kSimtRows, L.Hq, B);
-  attn_simt_kernel<E, D><<<grid, 256, smem, s>>>(static_cast<const E*>(q_hat), kv, rows,
+  attn_simt_kernel<E, D><<<grid, 256, smem, s>>>(static_cast<const E*>(q_hat), kv, rows, kb,
                                                   static_cast<E*>(out), T, L.Hq, L.Hkv,
-                                                  L.layer_type, L.window, L.scale);
+                                                  L.layer_type, L.window, L.scale, L.softcap);
   count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_attention_simt(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
-                                  RowIntervals rows, void* out, cudaStream_t s) {
+                                  RowIntervals rows, KeyBits kb, void* out, cudaStream_t s) {
   const bool f32 = L.dtype == 1;
   switch (L.d) {
-    case 64: return f32 ? run_simt<float, 64>(L, B, T, q_hat, kv, rows, out, s)
-                        : run_simt<__nv_bfloat16, 64>(L, B, T, q_hat, kv, rows, out, s);
-    case 128: return f32 ? run_simt<float, 128>(L, B, T, q_hat, kv, rows, out, s)
-                         : run_simt<__nv_bfloat16, 128>(L, B, T, q_hat, kv, rows, out, s);
-    case 256: return f32 ? run_simt<float, 256>(L, B, T, q_hat, kv, rows, out, s)
-                         : run_simt<__nv_bfloat16, 256>(L, B, T, q_hat, kv, rows, out, s);
-    case 512: return f32 ? run_simt<float, 512>(L, B, T, q_hat, kv, rows, out, s)
-                         : run_simt<__nv_bfloat16, 512>(L, B, T, q_hat, kv, rows, out, s);
+    case 64: return f32 ? run_simt<float, 64>(L, B, T, q_hat, kv, rows, kb, out, s)
+                        : run_simt<__nv_bfloat16, 64>(L, B, T, q_hat, kv, rows, kb, out, s);
+    case 128: return f32 ? run_simt<float, 128>(L, B, T, q_hat, kv, rows, kb, out, s)
+                         : run_simt<__nv_bfloat16, 128>(L, B, T, q_hat, kv, rows, kb, out, s);
+    case 256: return f32 ? run_simt<float, 256>(L, B, T, q_hat, kv, rows, kb, out, s)
+                         : run_simt<__nv_bfloat16, 256>(L, B, T, q_hat, kv, rows, kb, out, s);
+    case 512: return f32 ? run_simt<float, 512>(L, B, T, q_hat, kv, rows, kb, out, s)
+                         : run_simt<__nv_bfloat16, 512>(L, B, T, q_hat, kv, rows, kb, out, s);
   }
   return cudaErrorInvalidValue;
 }

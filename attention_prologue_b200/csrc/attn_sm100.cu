@@ -25,9 +25,8 @@
 //               edge tiles, lazy O rescale, P_j = exp2(S_j - m) as bf16 into
 //               TMEM over S_j; hands the row sums to the epilogue warps
 //   warps 8..11 Q and epilogue: after the last S of a tile, load the next
-//               tile's Q by TMA; then normalise the previous tile's O
-//               and write it out (each thread its row) while the next tile
-//               runs
+//               tile's Q by TMA; then normalise the previous tile's O and
+//               write it out (each thread its row) while the next tile runs
 // TMEM columns: NS = 4 S buffers of 64, O at 256.
 //
 // The tensor core's issue queue is short and a tcgen05.mma blocks while it
@@ -85,21 +84,22 @@ struct Layout {
 
 struct Bars {  // offsets (in 8-byte words) of the mbarriers from Layout::kBars
   enum {
-    q_full = 0,   // Q of the current tile in smem
-    q_empty = 2,  // the last S of a tile is done: Q may be replaced
-    o_last = 3,   // the last PV of a tile is done
-    o_free = 4,   // the epilogue warps have read O out of TMEM (128 arrivals)
-    l_ready = 5,  // [2] row sums of tiles k with k % 2 = i written (128 arrivals)
-    drain = 7,    // (S issuer)
-    drain2 = 8,   // (PV issuer)
-    k_full = 9,   // [4]
-    k_empty = 13,  // [4]
-    v_full = 17,   // [2]
-    v_empty = 19,  // [2]
-    s_full = 21,   // [NS]
-    p_full = 25,   // [NS]
-    o_done = 29,   // [NS] PV_j done (one per S buffer: rescale waits stay in one phase)
-    count = 33
+    q_full = 0,    // Q of the current tile in smem
+    q_empty = 1,   // the last S of a tile is done: Q may be replaced
+    o_last = 2,    // the last PV of a tile is done
+    o_free = 3,    // the epilogue warps have read O out of TMEM (128 arrivals)
+    l_ready = 4,   // [2] row sums of tiles k with k % 2 = i written (128 arrivals)
+    l_free = 6,    // [2] the epilogue warps have read those row sums (128 arrivals)
+    drain = 8,     // (S issuer)
+    drain2 = 9,    // (PV issuer)
+    k_full = 10,   // [4]
+    k_empty = 14,  // [4]
+    v_full = 18,   // [2]
+    v_empty = 20,  // [2]
+    s_full = 22,   // [NS]
+    p_full = 26,   // [NS]
+    o_done = 30,   // [NS] PV_j done (one per S buffer: rescale waits stay in one phase)
+    count = 34
   };
 };
 
@@ -147,14 +147,16 @@ __device__ __forceinline__ TileInfo tile_info(int t, int n_rt, int n_hg, int gp_
 
 }  // namespace
 
-template <int D>
+// kExtras: the padding mask and the logit soft-cap are compiled in (the
+// plain instantiation carries none of their code in the softmax loop).
+template <int D, bool kExtras>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
-                      RowIntervals rows, __nv_bfloat16* __restrict__ out, int T_,
-                      int Hq, int Hkv, int layer_type, int window, float scale_log2, int gp_log2,
-                      int n_work, int* status) {
+                      RowIntervals rows, KeyBits kb, __nv_bfloat16* __restrict__ out, int T_,
+                      int Hq, int Hkv, int layer_type, int window, float scale_log2,
+                      float cap2, int gp_log2, int n_work, int* status) {
   using Ly = Layout<D>;
   constexpr int kStagesK = Ly::kStagesK;
   static_assert(8 * Bars::count + (int)sizeof(Scalars) <= 512, "barrier area");
@@ -187,8 +189,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar(Bars::q_empty), 1);
     mbar_init(bar(Bars::o_last), 1);
     mbar_init(bar(Bars::o_free), 4 * 32);
-    mbar_init(bar(Bars::l_ready), 4 * 32);
-    mbar_init(bar(Bars::l_ready + 1), 4 * 32);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(Bars::l_ready + i), 4 * 32);
+      mbar_init(bar(Bars::l_free + i), 4 * 32);
+    }
     mbar_init(bar(Bars::drain), 1);
     mbar_init(bar(Bars::drain2), 1);
     for (int s = 0; s < kStagesK; ++s) {
@@ -354,8 +358,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       float m_used = -INFINITY, l = 0.f;
+      // with a soft-cap the scores are capped in log2 units first, then the
+      // scale is 1
+      const float sl2 = (kExtras && cap2 > 0.f) ? 1.f : scale_log2;
       for (int j = 0; j < ti.n; ++j, ++g) {
         const int sb = g % kNS;
+        // the padding bits of this key tile (all kept without a mask), read
+        // before the wait so the load overlaps it
+        const uint64_t keep =
+            (kExtras && kb.bits) ? kb.bits[(long)ti.b * kb.words + ti.kt0 + j] : ~0ull;
         ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::s_full + sb), (g / kNS) & 1, abort));
         if (!ok) break;
         tc_fence_after();
@@ -365,21 +376,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         const int key0 = (ti.kt0 + j) * BN;
         float x[BN];
-        float mt = -INFINITY;
-        if (key0 >= lo && key0 + BN - 1 <= hi) {  // interior tile: no mask
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            x[c] = __uint_as_float(sr[c]);
-            mt = fmaxf(mt, x[c]);
-          }
+        for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(sr[c]);
+        if (kExtras && cap2 > 0.f) {
+          const float k = scale_log2 / cap2;
+#pragma unroll
+          for (int c = 0; c < BN; ++c) x[c] = cap2 * tanh_fast(x[c] * k);
+        }
+        float mt = -INFINITY;
+        if (key0 >= lo && key0 + BN - 1 <= hi && (!kExtras || keep == ~0ull)) {  // no mask
+#pragma unroll
+          for (int c = 0; c < BN; ++c) mt = fmaxf(mt, x[c]);
         } else {
 #pragma unroll
           for (int c = 0; c < BN; ++c) {
-            x[c] = (key0 + c >= lo && key0 + c <= hi) ? __uint_as_float(sr[c]) : -INFINITY;
+            const bool in =
+                key0 + c >= lo && key0 + c <= hi && (!kExtras || ((keep >> c) & 1));
+            x[c] = in ? x[c] : -INFINITY;
             mt = fmaxf(mt, x[c]);
           }
         }
-        mt *= scale_log2;  // scale > 0: the max of the scaled scores
+        mt *= sl2;  // sl2 > 0: the max of the scaled scores
         // lazy rescale: only when the row max grows by more than 2^16
         const bool first = m_used == -INFINITY;
         const bool grow = !first && mt > m_used + 16.f;
@@ -415,11 +432,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[BN / 2];
 #pragma unroll
         for (int e = 0; e < BN / 2; ++e) {
-          const float p0 = ex2_approx(fmaf(x[2 * e], scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(x[2 * e + 1], scale_log2, neg_m));
-          rs += p0 + p1;
+          const float p0 = ex2_approx(fmaf(x[2 * e], sl2, neg_m));
+          const float p1 = ex2_approx(fmaf(x[2 * e + 1], sl2, neg_m));
           __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
           pk[e] = *reinterpret_cast<uint32_t*>(&bb);
+          // the row sum adds the P values the PV product multiplies (bf16),
+          // so a row's normalisation matches its weights exactly
+          rs += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
         }
         tmem_st32(tmem + lane_off + sb * BN, pk);
         tmem_wait_st();
@@ -434,6 +453,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // epilogue has yet to wait for tile k - 1 (one barrier for both would
       // then be two phases ahead of that wait); it cannot finish tile k + 1,
       // whose Q is loaded only after the epilogue of tile k - 1
+      // (the epilogue warps have read the row sums of tile k - 2 from this
+      // buffer: they arrive on l_free right after reading them)
+      if (k >= 2 && !(ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::l_free + (k & 1)),
+                                                             ((k - 2) >> 1) & 1, abort))))
+        break;
       lbuf[(k & 1) * BM + r] = l;
       mbar_arrive(bar(Bars::l_ready + (k & 1)));
     }
@@ -442,8 +466,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ew = warp - kEpiWarp0;
     const int r = threadIdx.x - kEpiWarp0 * 32;  // row (TMEM lane) of this thread
     const uint32_t lane_off = (uint32_t)(ew * 32) << 16;
-    const bool leader = ew == 0 && lane == 0;
     bool ok = true;
+    int q_issued = 0;  // tiles whose Q chunks the leader (warp 8, lane 0) has loaded
     TileInfo prev{};
     for (int k = 0; ok; ++k) {
       const int t = tile_of(k);
@@ -451,16 +475,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       TileInfo ti{};
       if (has) {
         ti = info(t);
-        // Q of tile k replaces tile k - 1's once the last S of tile k - 1 is done
+        // Q of tile k replaces tile k - 1's once the last S of tile k - 1 is
+        // done (all four warps wait: the epilogue of tile k - 1 follows it)
         if (k > 0)
           ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::q_empty), (k - 1) & 1, abort));
         if (!ok) break;
-        if (leader) {
+        if (ew == 0 && lane == 0) {
           mbar_arrive_expect_tx(bar(Bars::q_full), Ly::kChunks * BM * 128);
           for (int c = 0; c < Ly::kChunks; ++c)
-            tma_load_4d(base + Ly::kQ + c * Ly::kQChunk, &tm_q, bar(Bars::q_full), c * 64, ti.h0,
-                        ti.p0, ti.b);
+            tma_load_4d(base + Ly::kQ + c * Ly::kQChunk, &tm_q, bar(Bars::q_full), c * 64,
+                        ti.h0, ti.p0, ti.b);
         }
+        q_issued = k + 1;
       }
       if (k > 0) {
         // ---- epilogue of tile k - 1: O / l as bf16, each thread its row
@@ -470,6 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const float lsum = lbuf[((k - 1) & 1) * BM + r];
+        mbar_arrive(bar(Bars::l_free + ((k - 1) & 1)));  // the buffer may take tile k + 1's sums
         const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
         uint32_t ob[D / 2];
 #pragma unroll
@@ -502,6 +529,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!has) break;
       prev = ti;
     }
+    if (ew == 0 && lane == 0 && *abort && q_issued > 0)  // the last Q load lands before exit
+      mbar_wait(bar(Bars::q_full), (q_issued - 1) & 1, nullptr);
   }
 
   tc_fence_before();
@@ -567,7 +596,7 @@ bool make_map(CUtensorMap* m, const void* ptr, int rank, const uint64_t* dims,
 
 template <int D>
 cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
-                      RowIntervals rows, void* out, int* status, cudaStream_t s) {
+                      RowIntervals rows, KeyBits kb, void* out, int* status, cudaStream_t s) {
   CUtensorMap tq, tk, tv;
   const int gp_log2 = gqa_pack_log2(L.Hq, L.Hkv);
   constexpr int DF = D;
@@ -578,16 +607,18 @@ cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc 
     const uint32_t box[4] = {64, (uint32_t)(1 << gp_log2), (uint32_t)(BM >> gp_log2), 1};
     if (!make_map(&tq, q_hat, 4, dims, str, box)) return cudaErrorInvalidValue;
   }
-  {  // K, V [B * Hkv, cap, D]; only positions < T exist (rows past T read as 0)
-    const uint64_t dims[3] = {(uint64_t)DF, (uint64_t)T, (uint64_t)B * L.Hkv};
+  {  // K, V [B * Hkv, cap, D]; only positions < kv.len exist (rows past it read as 0)
+    const uint64_t dims[3] = {(uint64_t)DF, (uint64_t)kv.len, (uint64_t)B * L.Hkv};
     const uint64_t str[2] = {DF * es, (uint64_t)kv.cap * DF * es};
     const uint32_t box[3] = {64, BN, 1};
     if (!make_map(&tk, kv.k, 3, dims, str, box)) return cudaErrorInvalidValue;
     if (!make_map(&tv, kv.v, 3, dims, str, box)) return cudaErrorInvalidValue;
   }
   using Ly = Layout<D>;
-  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
+  const bool extras = kb.bits != nullptr || L.softcap > 0.f;
+  auto kern = extras ? attn_sm100_kernel<D, true> : attn_sm100_kernel<D, false>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
   if (e != cudaSuccess) return e;
   const float scale_log2 = L.scale * 1.4426950408889634f;
   const int bp = BM >> gp_log2;  // positions per tile
@@ -603,9 +634,9 @@ cudaError_t run_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc 
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = Ly::kAlloc;
   cfg.stream = s;
-  e = cudaLaunchKernelEx(&cfg, attn_sm100_kernel<D>, tq, tk, tv, rows,
+  e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, rows, kb,
                          static_cast<__nv_bfloat16*>(out), T, L.Hq, L.Hkv, L.layer_type, L.window,
-                         scale_log2, gp_log2, n_work, status);
+                         scale_log2, softcap_log2(L), gp_log2, n_work, status);
   if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();
@@ -618,12 +649,13 @@ bool attention_sm100_supported(const LayerCfg& L) {
 }
 
 cudaError_t launch_attention_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
-                                   RowIntervals rows, void* out, int* status, cudaStream_t s) {
+                                   RowIntervals rows, KeyBits kb, void* out, int* status,
+                                   cudaStream_t s) {
   switch (L.d) {
-    case 64: return run_sm100<64>(L, B, T, q_hat, kv, rows, out, status, s);
-    case 128: return run_sm100<128>(L, B, T, q_hat, kv, rows, out, status, s);
-    case 256: return run_sm100<256>(L, B, T, q_hat, kv, rows, out, status, s);
-    case 512: return launch_attention_pair(L, B, T, q_hat, kv, rows, out, status, s);
+    case 64: return run_sm100<64>(L, B, T, q_hat, kv, rows, kb, out, status, s);
+    case 128: return run_sm100<128>(L, B, T, q_hat, kv, rows, kb, out, status, s);
+    case 256: return run_sm100<256>(L, B, T, q_hat, kv, rows, kb, out, status, s);
+    case 512: return launch_attention_pair(L, B, T, q_hat, kv, rows, kb, out, status, s);
   }
   return cudaErrorInvalidValue;
 }

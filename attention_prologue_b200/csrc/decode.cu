@@ -13,6 +13,10 @@
 // and the combine kernel merges the chunks with
 //   o = sum_c e^{m_c - M} o~_c / sum_c e^{m_c - M} l_c,  M = max_c m_c.
 // The query prologue (RMSNorm * w_q, RoPE at P) runs inside the split kernel.
+// Padding keys of the prompt ("Gemma 4" Keras docs, "Gemma4ConditionalGenerate":
+// attention_mask) are skipped, and scores take the optional logit soft-cap
+// s -> c tanh(s / c) ("gemma4-pt-claude" README, "Attention Backend Notes");
+// a chunk without a kept key yields m = -inf, l = 0, which the combine ignores.
 #include "common.cuh"
 #include "g4attn.h"
 
@@ -42,8 +46,9 @@ __global__ void __launch_bounds__(kDecWarps * 32)
     decode_split_kernel(const T* __restrict__ q_raw, const T* __restrict__ wq,
                         const T* __restrict__ ck, const T* __restrict__ cv,
                         const int32_t* __restrict__ len, int cap, int rolling, int Hq, int Hkv,
-                        int layer_type, int window, float scale, float eps, int chunk, int nc,
-                        float* __restrict__ part_ml, float* __restrict__ part_o, int* status,
+                        int layer_type, int window, float scale, float softcap, KeyMask km,
+                        float eps, int chunk, int nc, float* __restrict__ part_ml,
+                        float* __restrict__ part_o, int* status,
                         const __grid_constant__ RopeParams rope) {
   constexpr int E = D / 32;  // contiguous elements per lane
   __shared__ float sq[kDecHeads][D];
@@ -92,6 +97,7 @@ __global__ void __launch_bounds__(kDecWarps * 32)
       }
     }
     for (int key = k_begin + warp; key < k_end; key += kDecWarps) {
+      if (km.keep && key < km.len && km.keep[(long)b * km.len + key] == 0) continue;  // padding
       const long slot = rolling ? key % cap : key;
       float kf[E], vf[E];
       Vec<T, E>::load(ck + (kv_base + slot) * D + lane * E, kf);
@@ -102,7 +108,8 @@ __global__ void __launch_bounds__(kDecWarps * 32)
         float dot = 0.f;
 #pragma unroll
         for (int e = 0; e < E; ++e) dot = fmaf(q[hh][e], kf[e], dot);
-        const float s = warp_sum(dot) * scale;
+        float s = warp_sum(dot) * scale;
+        if (softcap > 0.f) s = softcap * tanhf(s / softcap);
         const float mn = fmaxf(m[hh], s);
         const float corr = expf(m[hh] - mn);
         const float p = expf(s - mn);
@@ -184,22 +191,23 @@ __global__ void __launch_bounds__(128)
 template <typename T, int D>
 static cudaError_t run_decode(const LayerCfg& L, int B, const void* q_raw, const void* wq,
                               const void* cache_k, const void* cache_v, const int32_t* len,
-                              int cap, int rolling, const DecodePlan& plan, float* partials,
-                              void* out, int* status, cudaStream_t s, cudaEvent_t ev0,
-                              cudaEvent_t ev1) {
+                              int cap, int rolling, KeyMask km, const DecodePlan& plan,
+                              float* partials, void* out, int* status, cudaStream_t s,
+                              cudaEvent_t ev0, cudaEvent_t ev1) {
   float* part_ml = partials;
   float* part_o = partials + 2 * (size_t)B * L.Hq * plan.n_chunks;
   dim3 grid(plan.n_chunks, L.Hkv, B);
   if (ev0) cudaEventRecord(ev0, s);
   cudaError_t e;
   if (decode_mma_supported(L, cap, rolling)) {
-    e = launch_decode_mma(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, plan, part_ml,
-                          part_o, status, s);
+    e = launch_decode_mma(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, plan,
+                          part_ml, part_o, status, s);
   } else {
     decode_split_kernel<T, D><<<grid, kDecWarps * 32, 0, s>>>(
         static_cast<const T*>(q_raw), static_cast<const T*>(wq), static_cast<const T*>(cache_k),
         static_cast<const T*>(cache_v), len, cap, rolling, L.Hq, L.Hkv, L.layer_type, L.window,
-        L.scale, L.eps, plan.chunk, plan.n_chunks, part_ml, part_o, status, L.rope);
+        L.scale, L.softcap, km, L.eps, plan.chunk, plan.n_chunks, part_ml, part_o, status,
+        L.rope);
     count_launch();
     e = cudaGetLastError();
   }
@@ -215,14 +223,16 @@ static cudaError_t run_decode(const LayerCfg& L, int B, const void* q_raw, const
 
 cudaError_t launch_decode(const LayerCfg& L, int B, const void* q_raw, const void* wq,
                           const void* cache_k, const void* cache_v, const int32_t* len, int cap,
-                          int rolling, const DecodePlan& plan, float* partials, void* out,
-                          int* status, cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1) {
+                          int rolling, KeyMask km, const DecodePlan& plan, float* partials,
+                          void* out, int* status, cudaStream_t s, cudaEvent_t ev0,
+                          cudaEvent_t ev1) {
   const bool f32 = L.dtype == 1;
-#define G4_DEC(D)                                                                               \
-  return f32 ? run_decode<float, D>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, plan, \
-                                    partials, out, status, s, ev0, ev1)                          \
-             : run_decode<__nv_bfloat16, D>(L, B, q_raw, wq, cache_k, cache_v, len, cap,       \
-                                            rolling, plan, partials, out, status, s, ev0, ev1)
+#define G4_DEC(D)                                                                              \
+  return f32 ? run_decode<float, D>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, \
+                                    plan, partials, out, status, s, ev0, ev1)                   \
+             : run_decode<__nv_bfloat16, D>(L, B, q_raw, wq, cache_k, cache_v, len, cap,      \
+                                            rolling, km, plan, partials, out, status, s, ev0,  \
+                                            ev1)
   switch (L.d) {
     case 64: G4_DEC(64);
     case 128: G4_DEC(128);

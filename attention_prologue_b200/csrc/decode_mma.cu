@@ -96,8 +96,9 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
                       const __grid_constant__ CUtensorMap tm_v,
                       const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __restrict__ wq,
                       const int32_t* __restrict__ len, int cap, int rolling, int Hq, int Hkv,
-                      int layer_type, int window, float scale_log2, float eps, int chunk, int nc,
-                      float* __restrict__ part_ml, float* __restrict__ part_o, int* status,
+                      int layer_type, int window, float scale_log2, float cap2, KeyMask km,
+                      float eps, int chunk, int nc, float* __restrict__ part_ml,
+                      float* __restrict__ part_o, int* status,
                       const __grid_constant__ RopeParams rope) {
   using Ly = DmLayout<D>;
   constexpr int NS = Ly::kStages;
@@ -220,13 +221,24 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
           mma16816(sc, a, qb[kk][0], qb[kk][1]);
         }
       }
-      // masked scores in log2 units: rows = keys pos0 + lane/4 (+8), cols = heads
+      // masked scores in log2 units: rows = keys pos0 + lane/4 (+8), cols = heads;
+      // a padding key of the prompt (km) is masked like one outside [lo, P]
       const int kA = pos0 + (lane >> 2), kB = kA + 8;
-      const bool vA = kA >= lo && kA <= P, vB = kB >= lo && kB <= P;
-      const float x0 = vA ? sc[0] * scale_log2 : -INFINITY;  // (kA, head hA)
-      const float x1 = vA ? sc[1] * scale_log2 : -INFINITY;  // (kA, head hB)
-      const float x2 = vB ? sc[2] * scale_log2 : -INFINITY;  // (kB, head hA)
-      const float x3 = vB ? sc[3] * scale_log2 : -INFINITY;  // (kB, head hB)
+      auto kept = [&](int k) {
+        return !km.keep || k >= km.len || km.keep[(long)b * km.len + k] != 0;
+      };
+      const bool vA = kA >= lo && kA <= P && kept(kA), vB = kB >= lo && kB <= P && kept(kB);
+      float r[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) r[e] = sc[e] * scale_log2;
+      if (cap2 > 0.f) {  // soft-cap in log2 units
+#pragma unroll
+        for (int e = 0; e < 4; ++e) r[e] = cap2 * tanh_fast(r[e] * (1.f / cap2));
+      }
+      const float x0 = vA ? r[0] : -INFINITY;  // (kA, head hA)
+      const float x1 = vA ? r[1] : -INFINITY;  // (kA, head hB)
+      const float x2 = vB ? r[2] : -INFINITY;  // (kB, head hA)
+      const float x3 = vB ? r[3] : -INFINITY;  // (kB, head hB)
       float tA = fmaxf(x0, x2), tB = fmaxf(x1, x3);
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
@@ -336,8 +348,8 @@ bool decode_mma_supported(const LayerCfg& L, int cap, int rolling) {
 template <int D>
 static cudaError_t run_mma(const LayerCfg& L, int B, const void* q_raw, const void* wq,
                            const void* cache_k, const void* cache_v, const int32_t* len, int cap,
-                           int rolling, const DecodePlan& plan, float* part_ml, float* part_o,
-                           int* status, cudaStream_t s) {
+                           int rolling, KeyMask km, const DecodePlan& plan, float* part_ml,
+                           float* part_o, int* status, cudaStream_t s) {
   using Ly = DmLayout<D>;
   CUtensorMap tk, tv;
   const uint64_t dims[3] = {(uint64_t)D, (uint64_t)cap, (uint64_t)B * L.Hkv};
@@ -351,21 +363,21 @@ static cudaError_t run_mma(const LayerCfg& L, int B, const void* q_raw, const vo
   dim3 grid(plan.n_chunks, L.Hkv, B);
   decode_mma_kernel<D><<<grid, kThreadsDm, Ly::kAlloc, s>>>(
       tk, tv, static_cast<const __nv_bfloat16*>(q_raw), static_cast<const __nv_bfloat16*>(wq), len,
-      cap, rolling, L.Hq, L.Hkv, L.layer_type, L.window, L.scale * 1.4426950408889634f, L.eps,
-      plan.chunk, plan.n_chunks, part_ml, part_o, status, L.rope);
+      cap, rolling, L.Hq, L.Hkv, L.layer_type, L.window, L.scale * 1.4426950408889634f,
+      softcap_log2(L), km, L.eps, plan.chunk, plan.n_chunks, part_ml, part_o, status, L.rope);
   count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_mma(const LayerCfg& L, int B, const void* q_raw, const void* wq,
                               const void* cache_k, const void* cache_v, const int32_t* len,
-                              int cap, int rolling, const DecodePlan& plan, float* part_ml,
-                              float* part_o, int* status, cudaStream_t s) {
+                              int cap, int rolling, KeyMask km, const DecodePlan& plan,
+                              float* part_ml, float* part_o, int* status, cudaStream_t s) {
   switch (L.d) {
-    case 64: return run_mma<64>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, plan, part_ml, part_o, status, s);
-    case 128: return run_mma<128>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, plan, part_ml, part_o, status, s);
-    case 256: return run_mma<256>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, plan, part_ml, part_o, status, s);
-    case 512: return run_mma<512>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, plan, part_ml, part_o, status, s);
+    case 64: return run_mma<64>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, plan, part_ml, part_o, status, s);
+    case 128: return run_mma<128>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, plan, part_ml, part_o, status, s);
+    case 256: return run_mma<256>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, plan, part_ml, part_o, status, s);
+    case 512: return run_mma<512>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, plan, part_ml, part_o, status, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -24,8 +24,16 @@ struct LayerCfg {
   int Hq, Hkv, d;
   int dtype;  // 0 bf16, 1 fp32
   float scale, eps;
+  float softcap;  // logit soft-cap c (0: none)
   RopeParams rope;
 };
+
+// Soft-cap of a score already in log2 units: with C2 = c * log2(e),
+// x -> C2 * tanh(x / C2) (the cap c * tanh(s / c) of the natural-log score
+// s = x / log2(e)).  C2 == 0: no cap.
+inline float softcap_log2(const LayerCfg& L) {
+  return L.softcap > 0.f ? L.softcap * 1.4426950408889634f : 0.f;
+}
 
 // Where the key/value prologue writes: [B, Hkv, cap, d]; positions t >= first
 // go to slot (rolling ? t % cap : t).  k == nullptr: no destination.
@@ -37,11 +45,13 @@ struct KVDst {
   int first;
 };
 
-// Keys of one attention source: [B, Hkv, cap, d], position t at slot t.
+// Keys of one attention source: [B, Hkv, cap, d], position t at slot t;
+// positions 0 .. len-1 exist (a cached prefill reads len = p0 + T of them).
 struct KVSrc {
   const void* k;
   const void* v;
   int cap;
+  int len;
 };
 
 // Per-row key interval [lo[b*T+i], hi[b*T+i]] (image blocks), or nullptr
@@ -51,23 +61,40 @@ struct RowIntervals {
   const int32_t* hi;
 };
 
-// Q, K and V prologue of a prompt in one launch (one warp per token);
-// k_raw == nullptr: queries only (KV-shared layer).
-cudaError_t launch_token_prologue(const LayerCfg& L, int B, int T, const void* q_raw,
+// Padding mask of the keys as bits: bit k of bits[b * words + t] is 1 when
+// key position 64 t + k of sequence b is kept.  bits == nullptr: every key.
+struct KeyBits {
+  const uint64_t* bits;
+  int words;
+};
+
+// bits [B][words] of a byte mask [B][Tk] (non-zero = keep); words = ceil(Tk / 64).
+cudaError_t launch_mask_bits(int B, int Tk, const uint8_t* mask, uint64_t* bits, int words,
+                             cudaStream_t s);
+
+// Q, K and V prologue of T tokens at positions p0 .. p0+T-1 in one launch
+// (one warp per token); k_raw == nullptr: queries only (KV-shared layer).
+cudaError_t launch_token_prologue(const LayerCfg& L, int B, int T, int p0, const void* q_raw,
                                   const void* wq, void* q_hat, const void* k_raw,
                                   const void* v_raw, const void* wk, KVDst d0, KVDst d1,
                                   int32_t* len_out, cudaStream_t s);
 cudaError_t launch_block_intervals(const LayerCfg& L, int B, int T, const int32_t* ids,
                                    int32_t* lo, int32_t* hi, cudaStream_t s);
+// Per-row key intervals of a cached-prefill chunk (positions p0 .. p0+T-1);
+// ids [B][p0 + T] or nullptr.
+cudaError_t launch_chunk_intervals(const LayerCfg& L, int B, int T, int p0, const int32_t* ids,
+                                   int32_t* lo, int32_t* hi, cudaStream_t s);
 cudaError_t launch_attention_simt(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
-                                  RowIntervals rows, void* out, cudaStream_t s);
+                                  RowIntervals rows, KeyBits kb, void* out, cudaStream_t s);
 // tcgen05 prefill attention (bf16, head_dim 64/128/256/512); q_hat [B, T, Hq, d].
 bool attention_sm100_supported(const LayerCfg& L);
 cudaError_t launch_attention_sm100(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
-                                   RowIntervals rows, void* out, int* status, cudaStream_t s);
+                                   RowIntervals rows, KeyBits kb, void* out, int* status,
+                                   cudaStream_t s);
 // head_dim 512 on 2-CTA clusters (called by launch_attention_sm100).
 cudaError_t launch_attention_pair(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
-                                  RowIntervals rows, void* out, int* status, cudaStream_t s);
+                                  RowIntervals rows, KeyBits kb, void* out, int* status,
+                                  cudaStream_t s);
 
 // Query heads packed into one 128-row prefill tile, as a power of two: the
 // largest 2^g <= 8 dividing Hq / Hkv (every head of a tile reads the same KV
@@ -89,10 +116,18 @@ struct DecodePlan {
 };
 DecodePlan decode_plan(const LayerCfg& L, int cap);
 size_t decode_partials_bytes(const LayerCfg& L, int B, const DecodePlan& p);
+// Padding mask of a cache's prompt positions: position p < len of sequence
+// b is a padding key when keep[b * len + p] == 0 (keep == nullptr: none).
+struct KeyMask {
+  const uint8_t* keep;
+  int len;
+};
+
 cudaError_t launch_decode(const LayerCfg& L, int B, const void* q_raw, const void* wq,
                           const void* cache_k, const void* cache_v, const int32_t* len, int cap,
-                          int rolling, const DecodePlan& plan, float* partials, void* out,
-                          int* status, cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1);
+                          int rolling, KeyMask km, const DecodePlan& plan, float* partials,
+                          void* out, int* status, cudaStream_t s, cudaEvent_t ev0,
+                          cudaEvent_t ev1);
 
 // Tensor-core split kernel of g4attn_decode (bf16, <= 8 query heads per KV
 // head, rolling caches with capacity % 16 == 0); writes the same partials
@@ -100,14 +135,14 @@ cudaError_t launch_decode(const LayerCfg& L, int B, const void* q_raw, const voi
 bool decode_mma_supported(const LayerCfg& L, int cap, int rolling);
 cudaError_t launch_decode_mma(const LayerCfg& L, int B, const void* q_raw, const void* wq,
                               const void* cache_k, const void* cache_v, const int32_t* len,
-                              int cap, int rolling, const DecodePlan& plan, float* part_ml,
-                              float* part_o, int* status, cudaStream_t s);
+                              int cap, int rolling, KeyMask km, const DecodePlan& plan,
+                              float* part_ml, float* part_o, int* status, cudaStream_t s);
 
 // g4attn_decode with the split-KV partials in the library's fixed device
 // array instead of a workspace; returns a g4attn_status code.
 int launch_decode_noalloc(const LayerCfg& L, int B, const void* q_raw, const void* wq,
                           const void* cache_k, const void* cache_v, const int32_t* len, int cap,
-                          int rolling, void* out, int* status, cudaStream_t s);
+                          int rolling, KeyMask km, void* out, int* status, cudaStream_t s);
 
 // Tensor map of a bf16 tensor with a 128-byte-swizzled box (dims[0]
 // contiguous, strides in bytes for dims 1..rank-1); false on failure.

@@ -62,8 +62,9 @@ __global__ void __launch_bounds__(kWarps * 32)
     token_prologue_kernel(const T* __restrict__ q_raw, const T* __restrict__ wq,
                           T* __restrict__ q_hat, const T* __restrict__ k_raw,
                           const T* __restrict__ v_raw, const T* __restrict__ wk, int B, int T_,
-                          int Hq, int Hkv, KVDst d0, KVDst d1, int32_t* __restrict__ len_out,
-                          const __grid_constant__ RopeParams rope, float eps) {
+                          int p0, int Hq, int Hkv, KVDst d0, KVDst d1,
+                          int32_t* __restrict__ len_out, const __grid_constant__ RopeParams rope,
+                          float eps) {
   constexpr int E = D / 64, NB = 4;
   __shared__ double inv_freq[D / 2];
   for (int k = threadIdx.x; k < D / 2; k += blockDim.x) inv_freq[k] = rope.inv_freq[k];
@@ -71,7 +72,8 @@ __global__ void __launch_bounds__(kWarps * 32)
   const long tok = (long)blockIdx.x * kWarps + (threadIdx.x >> 5);
   if (tok >= (long)B * T_) return;
   const int lane = threadIdx.x & 31;
-  const long t = tok % T_, b = tok / T_;
+  const long b = tok / T_;
+  const long t = p0 + tok % T_;  // position of the token
   // the loads of the first batch of query heads and of the first K/V head
   // go out together, and the RoPE factors (fp64 angle reduction) are
   // computed while they are in flight
@@ -133,7 +135,131 @@ __global__ void __launch_bounds__(kWarps * 32)
     put_kv<T, D>(d0, Hkv, b, h, t, x0[0], x1[0], x0[1], x1[1]);
     put_kv<T, D>(d1, Hkv, b, h, t, x0[0], x1[0], x0[1], x1[1]);
   }
-  if (len_out && t == 0 && lane == 0) len_out[b] = T_;
+  if (len_out && t == p0 && lane == 0) len_out[b] = p0 + T_;
+}
+
+// Raw bf16 values kept packed (two per 32-bit word) between their load and
+// their use: the E = D/64 elements a lane holds of one half of a head.
+template <int E>
+struct PackedHalf {
+  static constexpr int W = E / 2;
+  uint32_t w[W];
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+    if constexpr (W == 4) {
+      const uint4 v = *reinterpret_cast<const uint4*>(p);
+      w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else if constexpr (W == 2) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p);
+      w[0] = v.x; w[1] = v.y;
+    } else {
+      w[0] = *reinterpret_cast<const uint32_t*>(p);
+    }
+  }
+  // bf16 -> fp32 is exact: the bits move into the high half of the word
+  __device__ __forceinline__ void unpack(float* x) const {
+#pragma unroll
+    for (int i = 0; i < W; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+
+// Prologue of a whole prompt for bf16 heads of 128/256/512: as
+// token_prologue_kernel, but the raw vectors of up to NQ query heads and NKV
+// key/value heads are loaded together, kept packed, before any arithmetic,
+// so a warp has ~2-5 KB of loads in flight at once (the kernel is bound by
+// memory latency: bytes in flight per SM set its rate).  Heads are then
+// normalised and rotated two at a time (the two norms' shuffles interleave).
+template <int D, int NQ, int NKV>
+__global__ void __launch_bounds__(kWarps * 32)
+    token_prologue_packed_kernel(const __nv_bfloat16* __restrict__ q_raw,
+                                 const __nv_bfloat16* __restrict__ wq,
+                                 __nv_bfloat16* __restrict__ q_hat,
+                                 const __nv_bfloat16* __restrict__ k_raw,
+                                 const __nv_bfloat16* __restrict__ v_raw,
+                                 const __nv_bfloat16* __restrict__ wk, int B, int T_, int p0,
+                                 int Hq, int Hkv, KVDst d0, KVDst d1,
+                                 int32_t* __restrict__ len_out,
+                                 const __grid_constant__ RopeParams rope, float eps) {
+  using bf16 = __nv_bfloat16;
+  constexpr int E = D / 64;
+  static_assert(E % 2 == 0 && NQ % 2 == 0, "packed pairs, heads two at a time");
+  __shared__ double inv_freq[D / 2];
+  for (int k = threadIdx.x; k < D / 2; k += blockDim.x) inv_freq[k] = rope.inv_freq[k];
+  __syncthreads();
+  const long tok = (long)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  if (tok >= (long)B * T_) return;
+  const int lane = threadIdx.x & 31;
+  const long b = tok / T_;
+  const long t = p0 + tok % T_;  // position of the token
+  PackedHalf<E> q[NQ][2];
+  auto load_q = [&](int h0) {
+#pragma unroll
+    for (int j = 0; j < NQ; ++j) {
+      const int h = min(h0 + j, Hq - 1);  // tail: reload the last head, store it once
+      const bf16* src = q_raw + (tok * Hq + h) * D + lane * E;
+      q[j][0].load(src);
+      q[j][1].load(src + D / 2);
+    }
+  };
+  PackedHalf<E> kv[NKV][2][2];  // [head][K or V][half]
+  const bf16* vsrc = v_raw ? v_raw : k_raw;
+  auto load_kv = [&](int h0) {
+#pragma unroll
+    for (int j = 0; j < NKV; ++j) {
+      const long off = (tok * Hkv + min(h0 + j, Hkv - 1)) * D + lane * E;
+      kv[j][0][0].load(k_raw + off);
+      kv[j][0][1].load(k_raw + off + D / 2);
+      kv[j][1][0].load(vsrc + off);
+      kv[j][1][1].load(vsrc + off + D / 2);
+    }
+  };
+  load_q(0);
+  if (k_raw) load_kv(0);
+  float w0[E], w1[E];
+  Vec<bf16, E>::load(wq + lane * E, w0);
+  Vec<bf16, E>::load(wq + D / 2 + lane * E, w1);
+  float c[E], s[E];
+  bool rot[E];
+  rope_factors<D>(t, inv_freq, rope.rotated_pairs, c, s, rot);
+  for (int h0 = 0; h0 < Hq; h0 += NQ) {
+    if (h0 > 0) load_q(h0);
+#pragma unroll
+    for (int j = 0; j < NQ; j += 2) {
+      float x0[2][E], x1[2][E];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        q[j + u][0].unpack(x0[u]);
+        q[j + u][1].unpack(x1[u]);
+      }
+      norm_rope<D, 2>(x0, x1, w0, w1, c, s, rot, true, eps);
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (h0 + j + u < Hq) store_vec<bf16, D>(q_hat + (tok * Hq + h0 + j + u) * D, x0[u], x1[u]);
+    }
+  }
+  if (!k_raw) return;
+  Vec<bf16, E>::load(wk + lane * E, w0);
+  Vec<bf16, E>::load(wk + D / 2 + lane * E, w1);
+  for (int h0 = 0; h0 < Hkv; h0 += NKV) {
+    if (h0 > 0) load_kv(h0);
+#pragma unroll
+    for (int j = 0; j < NKV; ++j) {
+      if (h0 + j >= Hkv) break;
+      float x0[2][E], x1[2][E];  // [K, V]
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        kv[j][u][0].unpack(x0[u]);
+        kv[j][u][1].unpack(x1[u]);
+      }
+      norm_rope<D, 1>(x0, x1, w0, w1, c, s, rot, true, eps);
+      norm_rope<D, 1>(x0 + 1, x1 + 1, nullptr, nullptr, c, s, rot, false, eps);
+      put_kv<bf16, D>(d0, Hkv, b, h0 + j, t, x0[0], x1[0], x0[1], x1[1]);
+      put_kv<bf16, D>(d1, Hkv, b, h0 + j, t, x0[0], x1[0], x0[1], x1[1]);
+    }
+  }
+  if (len_out && t == p0 && lane == 0) len_out[b] = p0 + T_;
 }
 
 // lo/hi of every row of a sliding layer with image blocks: the window
@@ -199,17 +325,34 @@ static cudaError_t dispatch(const LayerCfg& L, F&& f) {
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_token_prologue(const LayerCfg& L, int B, int T, const void* q_raw,
+cudaError_t launch_token_prologue(const LayerCfg& L, int B, int T, int p0, const void* q_raw,
                                   const void* wq, void* q_hat, const void* k_raw,
                                   const void* v_raw, const void* wk, KVDst d0, KVDst d1,
                                   int32_t* len_out, cudaStream_t s) {
   const long n_tok = (long)B * T;
   const unsigned grid = (unsigned)((n_tok + kWarps - 1) / kWarps);
+  using bf16 = __nv_bfloat16;
+  if (L.dtype == 0 && L.d >= 128) {  // bf16: the packed-load kernel
+    auto go = [&](auto kern) {
+      kern<<<grid, kWarps * 32, 0, s>>>(
+          static_cast<const bf16*>(q_raw), static_cast<const bf16*>(wq),
+          static_cast<bf16*>(q_hat), static_cast<const bf16*>(k_raw),
+          static_cast<const bf16*>(v_raw), static_cast<const bf16*>(wk), B, T, p0, L.Hq, L.Hkv,
+          d0, d1, len_out, L.rope, L.eps);
+      count_launch();
+      return cudaGetLastError();
+    };
+    switch (L.d) {
+      case 128: return go(token_prologue_packed_kernel<128, 8, 2>);
+      case 256: return go(token_prologue_packed_kernel<256, 8, 1>);
+      case 512: return go(token_prologue_packed_kernel<512, 4, 1>);
+    }
+  }
   return dispatch(L, [&]<typename E, int D>() {
     token_prologue_kernel<E, D><<<grid, kWarps * 32, 0, s>>>(
         static_cast<const E*>(q_raw), static_cast<const E*>(wq), static_cast<E*>(q_hat),
         static_cast<const E*>(k_raw), static_cast<const E*>(v_raw), static_cast<const E*>(wk), B,
-        T, L.Hq, L.Hkv, d0, d1, len_out, L.rope, L.eps);
+        T, p0, L.Hq, L.Hkv, d0, d1, len_out, L.rope, L.eps);
     count_launch();
     return cudaGetLastError();
   });
@@ -219,6 +362,75 @@ cudaError_t launch_block_intervals(const LayerCfg& L, int B, int T, const int32_
                                    int32_t* lo, int32_t* hi, cudaStream_t s) {
   const long n = (long)B * T;
   block_interval_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(ids, B, T, L.window, lo, hi);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// lo/hi of every row of a chunk at positions p0 .. p0+T-1 of a prompt of
+// p0 + T tokens (cached prefill): a global row sees [0, pos]; a sliding row
+// its window [max(0, pos-w+1), pos] united with the maximal run of equal
+// non-negative ids (ids [B][p0 + T], or nullptr) that contains pos, seen up
+// to the chunk's last position.
+__global__ void chunk_interval_kernel(const int32_t* __restrict__ ids, int B, int T_, int p0,
+                                      int layer_type, int window, int32_t* __restrict__ lo,
+                                      int32_t* __restrict__ hi) {
+  const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long)B * T_) return;
+  const int i = (int)(idx % T_);
+  const long b = idx / T_;
+  const int Tk = p0 + T_;
+  const int pos = p0 + i;
+  int a = 0, e = pos;
+  if (layer_type != 1) {
+    a = pos - window + 1;
+    if (a < 0) a = 0;
+    if (ids) {
+      const int32_t* row = ids + b * Tk;
+      const int id = row[pos];
+      if (id >= 0) {
+        int s = pos;
+        while (s > 0 && row[s - 1] == id) --s;
+        while (e + 1 < Tk && row[e + 1] == id) ++e;
+        if (s < a) a = s;
+      }
+    }
+  }
+  lo[idx] = a;
+  hi[idx] = e;
+}
+
+cudaError_t launch_chunk_intervals(const LayerCfg& L, int B, int T, int p0, const int32_t* ids,
+                                   int32_t* lo, int32_t* hi, cudaStream_t s) {
+  const long n = (long)B * T;
+  chunk_interval_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+      ids, B, T, p0, L.layer_type, L.window, lo, hi);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// Padding mask as bits, one thread per 64-key word: bit k of word t of
+// sequence b is 1 when key 64 t + k is kept (mask byte non-zero); keys past
+// the mask's end (the last word's tail) read as kept, and no row sees them.
+__global__ void mask_bits_kernel(const uint8_t* __restrict__ mask, int B, int Tk, int words,
+                                 uint64_t* __restrict__ bits) {
+  const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long)B * words) return;
+  const long b = idx / words;
+  const int t = (int)(idx % words);
+  const uint8_t* row = mask + b * Tk;
+  const int k0 = t * 64;
+  const int n = min(64, Tk - k0);
+  uint64_t v = ~0ull;
+  for (int k = 0; k < n; ++k)
+    if (row[k0 + k] == 0) v &= ~(1ull << k);
+  bits[idx] = v;
+}
+
+cudaError_t launch_mask_bits(int B, int Tk, const uint8_t* mask, uint64_t* bits, int words,
+                             cudaStream_t s) {
+  const long n = (long)B * words;
+  if (n == 0) return cudaSuccess;
+  mask_bits_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(mask, B, Tk, words, bits);
   count_launch();
   return cudaGetLastError();
 }

@@ -124,6 +124,14 @@ __device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t clus
       : "memory");
 }
 
+// 4-byte form of st_async_v4.
+__device__ __forceinline__ void st_async_b32(uint32_t cluster_addr, uint32_t cluster_bar,
+                                             uint32_t a) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+               ::"r"(cluster_addr), "r"(a), "r"(cluster_bar)
+               : "memory");
+}
+
 // try_wait with cluster-scope acquire (sees the peer's released writes).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -310,6 +318,21 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 1/x with the hardware approximation (MUFU.RCP, at most 1 ulp off).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// tanh(y) = 1 - 2 / (1 + e^{2y}) from the two approximations above: its
+// absolute error is a few 1e-7 (no cancellation problem: the result is
+// needed to an absolute, not relative, accuracy), and +-inf give +-1.
+__device__ __forceinline__ float tanh_fast(float y) {
+  const float e = ex2_approx(y * 2.8853900817779268f);  // e^{2y} = 2^{2y log2(e)}
+  return 1.f - 2.f * rcp_approx(1.f + e);
 }
 
 // ---------------------------------------------------------------- descriptors

@@ -21,6 +21,7 @@ G4ATTN_SLIDING, G4ATTN_GLOBAL = 0, 1
 G4ATTN_BF16, G4ATTN_FP32 = 0, 1
 
 EXPORTED = ("g4attn_prefill_workspace_size", "g4attn_decode_workspace_size", "g4attn_prefill",
+            "g4attn_prefill_chunk_workspace_size", "g4attn_prefill_chunk",
             "g4attn_cache_append", "g4attn_decode", "g4attn_decode_noalloc",
             "g4attn_get_device_status", "g4attn_time_next_attention", "g4attn_launch_count",
             "g4attn_status_string")
@@ -39,7 +40,7 @@ class LayerDesc(ctypes.Structure):
                 ("k_eq_v", ctypes.c_int), ("num_heads", ctypes.c_int),
                 ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
                 ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("logit_softcap", ctypes.c_float)]
 
 
 class _CCache(ctypes.Structure):
@@ -47,7 +48,8 @@ class _CCache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("len", ctypes.c_void_p),
                 ("capacity", ctypes.c_int), ("rolling", ctypes.c_int), ("batch", ctypes.c_int),
                 ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("key_mask", ctypes.c_void_p),
+                ("mask_len", ctypes.c_int)]
 
 
 _lib = None
@@ -66,8 +68,12 @@ def lib() -> ctypes.CDLL:
         L.g4attn_prefill_workspace_size.restype = S
         L.g4attn_decode_workspace_size.argtypes = [DP, CP]
         L.g4attn_decode_workspace_size.restype = S
-        L.g4attn_prefill.argtypes = [DP, I, I, P, P, P, P, P, P, CP, P, P, S, P]
+        L.g4attn_prefill.argtypes = [DP, I, I, P, P, P, P, P, P, P, CP, P, P, S, P]
         L.g4attn_prefill.restype = I
+        L.g4attn_prefill_chunk_workspace_size.argtypes = [DP, I, I, I]
+        L.g4attn_prefill_chunk_workspace_size.restype = S
+        L.g4attn_prefill_chunk.argtypes = [DP, I, I, I, P, P, P, P, P, P, P, CP, P, P, S, P]
+        L.g4attn_prefill_chunk.restype = I
         L.g4attn_cache_append.argtypes = [DP, CP, P, P, P, P]
         L.g4attn_cache_append.restype = I
         L.g4attn_decode.argtypes = [DP, CP, P, P, P, P, S, P]
@@ -97,11 +103,11 @@ def _dtype_code(dt: torch.dtype) -> int:
 def make_desc(layer_type: int, num_heads: int, num_kv_heads: int, head_dim: int, *,
               window: int = 0, rotary_fraction: float = 1.0, rope_theta: float = 1e4,
               k_eq_v: bool = False, softmax_scale: float | None = None, rms_eps: float = 1e-6,
-              dtype: torch.dtype = torch.bfloat16) -> LayerDesc:
+              dtype: torch.dtype = torch.bfloat16, logit_softcap: float = 0.0) -> LayerDesc:
     scale = head_dim ** -0.5 if softmax_scale is None else softmax_scale
     return LayerDesc(int(layer_type), int(window), float(rotary_fraction), float(rope_theta),
                      int(bool(k_eq_v)), int(num_heads), int(num_kv_heads), int(head_dim),
-                     float(scale), float(rms_eps), _dtype_code(dtype))
+                     float(scale), float(rms_eps), _dtype_code(dtype), float(logit_softcap))
 
 
 def _ptr(t: torch.Tensor | None, name: str, device: torch.device | None = None):
@@ -132,11 +138,14 @@ def cache_bytes(batch: int, num_kv_heads: int, capacity: int, head_dim: int,
 
 @dataclass
 class KVCache:
-    """A layer's KV cache in device memory owned by torch."""
+    """A layer's KV cache in device memory owned by torch.  key_mask (uint8
+    [batch, mask_len], optional) marks the padding positions of the prompt it
+    holds (0 = padding); later positions are kept."""
     k: torch.Tensor
     v: torch.Tensor
     len: torch.Tensor
     rolling: bool = False
+    key_mask: torch.Tensor | None = None
 
     @classmethod
     def allocate(cls, batch: int, num_kv_heads: int, capacity: int, head_dim: int, *,
@@ -157,9 +166,15 @@ class KVCache:
             raise ValueError("cache k and v differ in shape or dtype")
         if self.len.dtype != torch.int32 or self.len.numel() != B:
             raise ValueError("cache len must be int32 [batch]")
+        km, mlen = None, 0
+        if self.key_mask is not None:
+            if self.key_mask.dtype != torch.uint8 or self.key_mask.dim() != 2 \
+                    or self.key_mask.shape[0] != B:
+                raise ValueError("cache key_mask must be uint8 [batch, mask_len]")
+            km, mlen = _ptr(self.key_mask, "cache.key_mask"), self.key_mask.shape[1]
         return _CCache(_ptr(self.k, "cache.k"), _ptr(self.v, "cache.v"),
                        _ptr(self.len, "cache.len"), C, int(self.rolling), B, Hkv, d,
-                       _dtype_code(self.k.dtype))
+                       _dtype_code(self.k.dtype), km, mlen)
 
 
 def _check(rc: int, where: str):
@@ -180,12 +195,22 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
+def _mask(m: torch.Tensor | None, shape, name: str):
+    if m is None:
+        return None
+    if m.dtype != torch.uint8 or tuple(m.shape) != tuple(shape):
+        raise ValueError(f"{name} must be uint8 {list(shape)}")
+    return m
+
+
 def g4attn_prefill(desc: LayerDesc, q_raw: torch.Tensor, k_raw: torch.Tensor | None,
                    v_raw: torch.Tensor | None, q_norm_w: torch.Tensor,
                    k_norm_w: torch.Tensor | None, image_block_ids: torch.Tensor | None = None,
                    cache: KVCache | None = None, out: torch.Tensor | None = None,
-                   workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Prefill of q_raw [B, T, Hq, d] (see g4attn_prefill in g4attn.h)."""
+                   workspace: torch.Tensor | None = None, stream=None,
+                   attention_mask: torch.Tensor | None = None) -> torch.Tensor:
+    """Prefill of q_raw [B, T, Hq, d] (see g4attn_prefill in g4attn.h);
+    attention_mask uint8 [B, T], 0 = padding key."""
     B, T = q_raw.shape[0], q_raw.shape[1]
     dev = q_raw.device
     if out is None:
@@ -194,14 +219,49 @@ def g4attn_prefill(desc: LayerDesc, q_raw: torch.Tensor, k_raw: torch.Tensor | N
         workspace = _workspace(g4attn_prefill_workspace_size(desc, B, T), dev)
     if image_block_ids is not None and image_block_ids.dtype != torch.int32:
         raise ValueError("image_block_ids must be int32")
+    am = _mask(attention_mask, (B, T), "attention_mask")
     cc = cache.c() if cache is not None else None
     rc = lib().g4attn_prefill(
         ctypes.byref(desc), B, T, _ptr(q_raw, "q_raw", dev), _ptr(k_raw, "k_raw", dev),
         _ptr(v_raw, "v_raw", dev), _ptr(q_norm_w, "q_norm_w", dev),
         _ptr(k_norm_w, "k_norm_w", dev), _ptr(image_block_ids, "image_block_ids", dev),
+        _ptr(am, "attention_mask", dev),
         ctypes.byref(cc) if cc is not None else None, _ptr(out, "out", dev),
         _ptr(workspace, "workspace", dev), workspace.numel(), _stream(stream))
     _check(rc, "g4attn_prefill")
+    return out
+
+
+def g4attn_prefill_chunk_workspace_size(desc: LayerDesc, B: int, T: int, p0: int) -> int:
+    return int(lib().g4attn_prefill_chunk_workspace_size(ctypes.byref(desc), B, T, p0))
+
+
+def g4attn_prefill_chunk(desc: LayerDesc, p0: int, q_raw: torch.Tensor,
+                         k_raw: torch.Tensor | None, v_raw: torch.Tensor | None,
+                         q_norm_w: torch.Tensor, k_norm_w: torch.Tensor | None,
+                         image_block_ids: torch.Tensor | None, cache: KVCache,
+                         out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                         stream=None, attention_mask: torch.Tensor | None = None) -> torch.Tensor:
+    """Cached prefill of a chunk q_raw [B, T, Hq, d] at positions p0 .. p0+T-1
+    (see g4attn_prefill_chunk in g4attn.h); image_block_ids and
+    attention_mask (uint8, 0 = padding key) [B, p0 + T]."""
+    B, T = q_raw.shape[0], q_raw.shape[1]
+    dev = q_raw.device
+    if out is None:
+        out = torch.empty_like(q_raw)
+    if workspace is None:
+        workspace = _workspace(g4attn_prefill_chunk_workspace_size(desc, B, T, p0), dev)
+    if image_block_ids is not None and image_block_ids.dtype != torch.int32:
+        raise ValueError("image_block_ids must be int32")
+    am = _mask(attention_mask, (B, p0 + T), "attention_mask")
+    cc = cache.c()
+    rc = lib().g4attn_prefill_chunk(
+        ctypes.byref(desc), B, T, p0, _ptr(q_raw, "q_raw", dev), _ptr(k_raw, "k_raw", dev),
+        _ptr(v_raw, "v_raw", dev), _ptr(q_norm_w, "q_norm_w", dev),
+        _ptr(k_norm_w, "k_norm_w", dev), _ptr(image_block_ids, "image_block_ids", dev),
+        _ptr(am, "attention_mask", dev), ctypes.byref(cc), _ptr(out, "out", dev), _ptr(workspace, "workspace", dev),
+        workspace.numel(), _stream(stream))
+    _check(rc, "g4attn_prefill_chunk")
     return out
 
 

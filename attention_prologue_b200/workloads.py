@@ -39,6 +39,7 @@ class LayerShape:
     k_eq_v: bool = False
     softmax_scale: float | None = None  # None: 1/sqrt(head_dim)
     rms_eps: float = 1e-6
+    logit_softcap: float = 0.0          # 0: none
 
     @property
     def scale(self) -> float:

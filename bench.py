@@ -268,7 +268,8 @@ def job_rate(world: int, units_per_step: float, steps: int, max_ms: float) -> fl
 def desc_of(L: W.LayerShape, dtype=torch.bfloat16) -> G.LayerDesc:
     return G.make_desc(L.layer_type, L.num_heads, L.num_kv_heads, L.head_dim, window=L.window,
                        rotary_fraction=L.rotary_fraction, rope_theta=L.rope_theta,
-                       k_eq_v=L.k_eq_v, softmax_scale=L.scale, rms_eps=L.rms_eps, dtype=dtype)
+                       k_eq_v=L.k_eq_v, softmax_scale=L.scale, rms_eps=L.rms_eps, dtype=dtype,
+                       logit_softcap=L.logit_softcap)
 
 
 def made_events(n):

@@ -39,6 +39,12 @@
  *  [V3] "Gemma 4" overview blog, "Shared KV Cache": later layers reuse the
  *       K/V of the most recent earlier layer of the same type and compute
  *       only their own queries.
+ *  [K4] "Gemma 4" (Keras port docs), "Gemma4ConditionalGenerate" argument
+ *       table: attention_mask (batch, seq), 1 = keep, 0 = padding.
+ *  [P3] "gemma4-pt-claude" README, "Attention Backend Notes": an attention
+ *       logit soft-cap (attn_logits_soft_cap) exists as a layer option; the
+ *       page prints no formula, the reading is the tanh cap the Keras docs'
+ *       argument table names for the final logits.
  *
  * Definitions used throughout (readings of the pages, stated once):
  *  - RMSNorm over the d values of one head: x / sqrt(mean(x^2) + eps) * w,
@@ -57,7 +63,10 @@
  *    whole block, [min(max(0, i - window + 1), s), e - 1]  [K1][V1].
  *    An image block is a maximal run of equal non-negative ids in
  *    image_block_ids; -1 marks text.
- *  - o_i = sum_j softmax_j(softmax_scale * q_i . k_j) v_j over those keys.
+ *  - o_i = sum_j softmax_j(s_ij) v_j over those keys, with the score
+ *    s_ij = softmax_scale * q_i . k_j, or c * tanh(softmax_scale * q_i . k_j / c)
+ *    with a logit soft-cap c > 0 [P3].  A padding key (mask entry 0) is never
+ *    attended [K4]; a query left without any key outputs 0.
  */
 #ifndef G4ATTN_H
 #define G4ATTN_H
@@ -105,6 +114,8 @@ typedef struct {
   float softmax_scale;
   float rms_eps;
   int dtype;             /* G4ATTN_BF16 or G4ATTN_FP32 */
+  float logit_softcap;   /* c > 0: scores become c * tanh(score / c) [P3];
+                            0: no cap */
 } g4attn_layer_desc;
 
 /* A per-layer KV cache [P2], caller-owned device memory.  K and V are stored
@@ -114,7 +125,13 @@ typedef struct {
  * sequence b written so far.  A rolling cache keeps position p at slot
  * p % capacity and needs capacity >= window; it is only valid on sliding
  * layers.  A non-rolling cache keeps position p at slot p and rejects
- * p >= capacity. */
+ * p >= capacity.
+ * key_mask (device uint8 [batch, mask_len], or NULL) is the padding mask of
+ * the prompt the cache holds [K4]: position p < mask_len of sequence b is a
+ * padding key when key_mask[b * mask_len + p] == 0; positions >= mask_len
+ * (tokens appended later) are kept.  g4attn_decode reads it; the prefill
+ * calls take their mask as an argument.  mask_len is ignored when key_mask
+ * is NULL. */
 typedef struct {
   void *k;
   void *v;
@@ -125,6 +142,8 @@ typedef struct {
   int num_kv_heads;
   int head_dim;
   int dtype;
+  const uint8_t *key_mask;
+  int mask_len;
 } g4attn_cache;
 
 /* Bytes of device workspace g4attn_prefill needs for this layer and size.
@@ -151,6 +170,10 @@ size_t g4attn_decode_workspace_size(const g4attn_layer_desc *desc,
  *                  is NULL).
  *  image_block_ids device int32 [B, T] or NULL: -1 text, a block is a maximal
  *                  run of one non-negative id.  Ignored on global layers.
+ *  attention_mask  device uint8 [B, T] or NULL [K4]: a key at a position
+ *                  whose entry is 0 is padding and never attended (RoPE
+ *                  positions stay the token indices); a row left without any
+ *                  key outputs 0.  NULL: no padding.
  *  cache           NULL, or a cache of this layer: with k_raw the post-prologue
  *                  K/V of positions 0..T-1 are written to it (a rolling cache
  *                  keeps the last `capacity` of them) and len[b] is set to T;
@@ -173,8 +196,45 @@ size_t g4attn_decode_workspace_size(const g4attn_layer_desc *desc,
 int g4attn_prefill(const g4attn_layer_desc *desc, int B, int T,
                    const void *q_raw, const void *k_raw, const void *v_raw,
                    const void *q_norm_w, const void *k_norm_w,
-                   const int32_t *image_block_ids, g4attn_cache *cache,
+                   const int32_t *image_block_ids,
+                   const uint8_t *attention_mask, g4attn_cache *cache,
                    void *out, void *workspace, size_t ws_bytes, void *stream);
+
+/* Bytes of device workspace g4attn_prefill_chunk needs.  Returns 0 if the
+ * arguments are invalid. */
+size_t g4attn_prefill_chunk_workspace_size(const g4attn_layer_desc *desc,
+                                           int B, int T, int p0);
+
+/* Cached (chunked) prefill ("gemma4-pt-claude" README, "Tests": a cached
+ * path reproduces the uncached forward pass, image spans included): a chunk
+ * of T tokens per sequence at positions p0 .. p0+T-1 after the p0 tokens
+ * `cache` already holds (len[b] == p0 for every sequence: the caller's
+ * contract).  The chunk's keys/values go through the prologue into slots
+ * p0 .. p0+T-1 and len[b] becomes p0 + T; each query row then attends over
+ * the interval of its position in a prompt of p0 + T tokens (image blocks
+ * seen up to position p0 + T - 1: cut chunks between blocks to reproduce a
+ * whole prompt).
+ *
+ *  q_raw, k_raw, v_raw, q_norm_w, k_norm_w, out: as g4attn_prefill, [B, T,
+ *                  ...] for the chunk; k_raw NULL: a KV-shared layer reading
+ *                  `cache`, which must hold positions 0 .. p0+T-1.
+ *  image_block_ids device int32 [B, p0 + T] or NULL (ignored on global layers).
+ *  attention_mask  device uint8 [B, p0 + T] or NULL: the padding mask of every
+ *                  position up to the chunk's last (as g4attn_prefill); the
+ *                  cache's key_mask is not read.
+ *  cache           required; capacity >= p0 + T (a rolling cache only before
+ *                  it wraps).
+ *  workspace       g4attn_prefill_chunk_workspace_size bytes, 256-byte aligned.
+ *
+ * Errors: as g4attn_prefill; G4ATTN_ECACHE_OVERFLOW for a non-rolling cache
+ * with capacity < p0 + T; G4ATTN_EINVAL for a rolling or KV-shared one. */
+int g4attn_prefill_chunk(const g4attn_layer_desc *desc, int B, int T, int p0,
+                         const void *q_raw, const void *k_raw,
+                         const void *v_raw, const void *q_norm_w,
+                         const void *k_norm_w, const int32_t *image_block_ids,
+                         const uint8_t *attention_mask, g4attn_cache *cache,
+                         void *out, void *workspace, size_t ws_bytes,
+                         void *stream);
 
 /* Append one token per sequence to a layer's cache [P2][K3]: the key/value
  * prologue of k_raw/v_raw (device [B, 1, num_kv_heads, d]; v_raw NULL with
@@ -190,8 +250,9 @@ int g4attn_cache_append(const g4attn_layer_desc *desc, g4attn_cache *cache,
 /* Single-token decode [K3][V1][V3]: for every sequence b the query of the
  * token at position P = len[b] - 1 (the last one appended) attends over the
  * keys of row P of a prefill -- [max(0, P - window + 1), P] on a sliding
- * layer, [0, P] on a global one -- read from `cache`.  A KV-shared layer
- * passes the cache of the layer it reads and skips the append.
+ * layer, [0, P] on a global one -- read from `cache`, minus the padding keys
+ * the cache's key_mask marks [K4].  A KV-shared layer passes the cache of
+ * the layer it reads and skips the append.
  *
  *  q_raw     device [B, 1, num_heads, d];  q_norm_w device [d].
  *  out       device [B, 1, num_heads, d].

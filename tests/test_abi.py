@@ -44,7 +44,7 @@ def desc(**kw):
 
 
 def prefill_rc(d, B=1, T=16, k=FAKE, v=FAKE, ids=None, cache=None, ws=FAKE, ws_bytes=1 << 40):
-    return G.lib().g4attn_prefill(ctypes.byref(d), B, T, FAKE, k, v, FAKE, FAKE, ids,
+    return G.lib().g4attn_prefill(ctypes.byref(d), B, T, FAKE, k, v, FAKE, FAKE, ids, None,
                                   ctypes.byref(cache) if cache is not None else None, FAKE, ws,
                                   ws_bytes, None)
 
@@ -62,7 +62,8 @@ def ccache(d, B=1, C=64, rolling=0, **kw):
     dict(num_kv_heads=0), dict(window=0),
     dict(rotary_fraction=0.3), dict(rotary_fraction=1.5), dict(rope_theta=-1.0),
     dict(rms_eps=-1.0), dict(softmax_scale=float("inf")), dict(softmax_scale=0.0),
-    dict(softmax_scale=-0.5), dict(layer_type=2),
+    dict(softmax_scale=-0.5), dict(layer_type=2), dict(logit_softcap=-1.0),
+    dict(logit_softcap=float("inf")), dict(logit_softcap=float("nan")),
 ])
 def test_bad_descriptors_are_rejected(bad):
     d = desc(**bad)
@@ -147,8 +148,10 @@ def test_workspace_sizes():
     d = desc(num_heads=8, num_kv_heads=1, head_dim=256, window=512)
     B, T = 1, 8192
     ws = G.lib().g4attn_prefill_workspace_size(ctypes.byref(d), B, T)
-    # q_hat + K/V scratch + two int32 interval arrays, 256-aligned pieces
-    assert ws == B * T * 8 * 256 * 2 + 2 * B * T * 1 * 256 * 2 + 2 * B * T * 4
+    # q_hat + K/V scratch + two int32 interval arrays + the padding bits (one
+    # 64-bit word per 64 keys, 256-byte aligned), 256-aligned pieces
+    bits = -(-(B * (T // 64) * 8) // 256) * 256
+    assert ws == B * T * 8 * 256 * 2 + 2 * B * T * 1 * 256 * 2 + 2 * B * T * 4 + bits
     c = ccache(d, B=64, C=1024, rolling=1)
     dws = G.lib().g4attn_decode_workspace_size(ctypes.byref(d), ctypes.byref(c))
     assert dws > 0 and dws % 256 == 0
@@ -177,3 +180,53 @@ def test_cache_layout_reproduces_the_printed_kv_table():
         win_b = n_sliding * G.cache_bytes(1, skv, window, hd, torch.bfloat16) + glob
         assert round(full_b / 1e9, 1) == float(full), model
         assert round(win_b / 1e9, 1) == float(windowed), model
+
+
+def chunk_rc(d, B=1, T=16, p0=32, k=FAKE, v=FAKE, cache=None, ws=FAKE, ws_bytes=1 << 40):
+    return G.lib().g4attn_prefill_chunk(ctypes.byref(d), B, T, p0, FAKE, k, v, FAKE, FAKE, None,
+                                        None,
+                                        ctypes.byref(cache) if cache is not None else None, FAKE,
+                                        ws, ws_bytes, None)
+
+
+def test_chunked_prefill_validation():
+    lib = G.lib()
+    d = desc()
+    assert chunk_rc(d) == G.G4ATTN_EINVAL  # a cached prefill needs its cache
+    assert chunk_rc(d, p0=-1, cache=ccache(d, C=64)) == G.G4ATTN_EINVAL
+    assert chunk_rc(d, p0=56, T=16, cache=ccache(d, C=64)) == G.G4ATTN_ECACHE_OVERFLOW
+    dr = desc(window=8)
+    assert chunk_rc(dr, p0=56, T=16, cache=ccache(dr, C=64, rolling=1)) == G.G4ATTN_EINVAL
+    assert chunk_rc(d, k=None, v=None, p0=56, T=16, cache=ccache(d, C=64)) == G.G4ATTN_EINVAL
+    assert chunk_rc(desc(k_eq_v=True), cache=ccache(d, C=64)) == G.G4ATTN_EINVAL
+    assert chunk_rc(d, cache=ccache(d, C=64), ws=None, ws_bytes=0) == G.G4ATTN_EWORKSPACE
+    assert chunk_rc(d, T=0, cache=ccache(d, C=64)) == G.G4ATTN_OK
+    assert lib.g4attn_prefill_chunk_workspace_size(ctypes.byref(d), 1, 16, -1) == 0
+    assert lib.g4attn_prefill_chunk_workspace_size(ctypes.byref(d), 2, 16, 48) >= \
+        2 * 16 * 8 * 256 * 2 + 2 * 2 * 16 * 4
+
+
+def test_cache_key_mask_length_is_checked():
+    """A cache's padding mask needs a length >= 0 (decode reads it)."""
+    d = desc()
+    c = ccache(d, C=64)
+    c.key_mask = FAKE
+    c.mask_len = -1
+    assert G.lib().g4attn_decode_workspace_size(ctypes.byref(d), ctypes.byref(c)) == 0
+    assert G.lib().g4attn_decode(ctypes.byref(d), ctypes.byref(c), FAKE, FAKE, FAKE, FAKE,
+                                 1 << 40, None) == G.G4ATTN_EINVAL
+    c.mask_len = 0  # an empty mask: every position is kept
+    assert G.lib().g4attn_decode_workspace_size(ctypes.byref(d), ctypes.byref(c)) > 0
+
+
+def test_prefill_workspace_covers_the_padding_bits():
+    """The workspace size covers the padding bits of the largest call (one
+    64-bit word per 64 key positions and sequence)."""
+    lib = G.lib()
+    d = desc(layer_type=G.G4ATTN_GLOBAL)
+    base = lib.g4attn_prefill_workspace_size(ctypes.byref(d), 2, 1000)
+    q_hat = 2 * 1000 * 8 * 256 * 2
+    kv = 2 * 2 * 1000 * 2 * 256 * 2
+    assert base >= q_hat + kv + 2 * 16 * 8
+    assert lib.g4attn_prefill_chunk_workspace_size(ctypes.byref(d), 2, 100, 900) >= \
+        2 * 100 * 8 * 256 * 2 + 2 * 16 * 8

@@ -13,7 +13,8 @@ import oracle
 from attention_prologue_b200 import g4attn as G
 from attention_prologue_b200 import workloads as W
 
-from helpers import (check, desc_of, gpu_prefill, oracle_layer, oracle_prefill, sample_rows)
+from helpers import (check, check_beyond_output_rounding, desc_of, gpu_prefill, oracle_layer,
+                     oracle_prefill, record, sample_rows, stored_reference, value_bound)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -137,9 +138,28 @@ def test_kv_shared_prefill_reads_the_source_cache():
 
 # -- softmax scale 1.0 on the tensor-core kernels -----------------------------
 # The README's reading ("QK-norm replaces 1/sqrt(d)") gives logits sqrt(d)
-# times larger than the 1/sqrt(d) scale: the exponentials are far more
-# sensitive to absolute score errors (the head_dim-512 kernel exchanges
-# partial scores between the two CTAs of a pair).
+# times larger than the 1/sqrt(d) scale, and the exponentials are that much
+# more sensitive to absolute score errors.  There the bf16 storage of q_hat
+# and k_hat alone (the KV cache's format) moves the output by up to ~0.18 at
+# d 256 and ~0.3 at d 512 against the unrounded oracle (a CPU computation
+# with nothing but that rounding gives the same), more than any kernel error.
+# So these cases assert the kernels against the oracle's attention of the
+# bf16-stored q_hat, k_hat, v_hat -- which still covers every step of the
+# kernels' arithmetic: fp32 accumulation, exp2, P in bf16, the int16 exchange
+# of partial scores at d 512 -- and record the distance to the unrounded
+# oracle in the run's summary.  The bar is the usual 2e-2 / 2e-3 on what the
+# kernel adds beyond the bf16 rounding of its own output, which at this
+# scale alone reaches 0.0156 (|o| up to ~5), plus the effect of rounding the
+# softmax weights to bf16 for the PV product, which this reference does not
+# model (<= 2^-9 max |v_hat|, ~0.01; helpers.check_beyond_output_rounding).
+
+def run_stored(w, inp, rows=None):
+    out = gpu_prefill(w, inp)
+    got = out if rows is None else out[:, rows]
+    check_beyond_output_rounding(got, stored_reference(w, inp, rows),
+                                 f"{w.name} (bf16-stored q,k,v)",
+                                 p_bound=2.0 ** -9 * value_bound(w, inp))
+    record(got, stored_reference(w, inp, rows, store=False), f"{w.name} (unrounded oracle)")
 
 SCALE_ONE = [
     W.scaled_down(W.E2B_SLIDING, T=1000, softmax_scale=1.0),                 # d 256 sliding
@@ -151,7 +171,7 @@ SCALE_ONE = [
 
 @pytest.mark.parametrize("w", SCALE_ONE, ids=lambda w: w.name)
 def test_tensor_cores_at_scale_one(w):
-    run_case(w, seed=21)
+    run_stored(w, W.prefill_inputs(w, DEV, 21))
 
 
 @pytest.mark.parametrize("hd,layer", [(256, "sliding"), (512, "global")])
@@ -177,8 +197,7 @@ def test_tensor_cores_with_large_correlated_logits(hd, layer, mix):
             j = torch.maximum(j, (t - L.window + 1).clamp(min=0))
         noise = torch.randn(T, L.head_dim, generator=g, device=DEV) * mix
         inp["q_raw"][0, :, h] = (inp["k_raw"][0, j, h // grp].float() + noise).bfloat16()
-    out = gpu_prefill(w, inp)
-    check(out, oracle_prefill(w, inp), w.dtype, w.name)
+    run_stored(w, inp)
 
 
 # -- full-size workloads, sampled rows ----------------------------------------
