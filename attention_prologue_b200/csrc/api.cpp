@@ -107,8 +107,13 @@ static int make_cfg(const g4attn_layer_desc* d, LayerCfg* L) {
   return G4ATTN_OK;
 }
 
+// A single-tensor cache (v == NULL) stores V = RMSNorm(k_raw) of a K=V layer
+// in `k`; a reader rebuilds K with the owning layer's k_norm_w and RoPE.
+static bool single_tensor(const g4attn_cache* c) { return c->v == nullptr; }
+
 static int check_cache(const LayerCfg& L, const g4attn_cache* c, int B) {
-  if (!c->k || !c->v || !c->len) return G4ATTN_EINVAL;
+  if (!c->k || !c->len) return G4ATTN_EINVAL;
+  if (single_tensor(c) && (!L.k_eq_v || !c->k_norm_w || c->rolling)) return G4ATTN_EINVAL;
   if (c->batch != B || c->num_kv_heads != L.Hkv || c->head_dim != L.d || c->dtype != L.dtype)
     return G4ATTN_EINVAL;
   if (c->capacity < 1 || (c->rolling != 0 && c->rolling != 1)) return G4ATTN_EINVAL;
@@ -199,12 +204,13 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
     if ((st = check_cache(L, cache, B)) != G4ATTN_OK) return st;
     if (!cache->rolling && cache->capacity < T) return G4ATTN_ECACHE_OVERFLOW;
     if (shared && cache->capacity < T) return G4ATTN_EINVAL;  // evicted keys cannot be read
+    if (shared && single_tensor(cache)) return G4ATTN_EUNSUPPORTED;  // no K to read
   }
   if (B == 0 || T == 0) return G4ATTN_OK;
 
-  // attention reads keys from the cache when it holds positions 0..T-1 at
-  // slots 0..T-1, otherwise from scratch
-  const bool cache_is_src = cache && cache->capacity >= T;
+  // attention reads keys from the cache when it holds K and V of positions
+  // 0..T-1 at slots 0..T-1, otherwise from scratch
+  const bool cache_is_src = cache && cache->capacity >= T && !single_tensor(cache);
   const bool intervals = L.layer_type == G4ATTN_SLIDING && image_block_ids != nullptr;
   PrefillWs w = prefill_ws(L, B, T, !cache_is_src, intervals, attention_mask != nullptr, T);
   if (!workspace || ws_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
@@ -225,7 +231,9 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
   KVDst d0{nullptr, nullptr, 1, 0, 0}, d1{nullptr, nullptr, 1, 0, 0};
   if (!shared) {
     d0 = {const_cast<void*>(src.k), const_cast<void*>(src.v), src.cap, 0, 0};
-    if (cache && !cache_is_src)  // rolling cache smaller than the prompt: last `cap` positions
+    if (cache && single_tensor(cache))  // V alone (put_kv with v == nullptr)
+      d1 = {cache->k, nullptr, cache->capacity, 0, 0};
+    else if (cache && !cache_is_src)  // rolling cache smaller than the prompt: the last `cap`
       d1 = {cache->k, cache->v, cache->capacity, 1, T - cache->capacity};
   }
   void* q_hat = ws + w.q_hat;
@@ -277,6 +285,7 @@ int g4attn_prefill_chunk(const g4attn_layer_desc* desc, int B, int T, int p0, co
     if ((v_raw == nullptr) != (L.k_eq_v == 1)) return G4ATTN_EINVAL;
   }
   if ((st = check_cache(L, cache, B)) != G4ATTN_OK) return st;
+  if (single_tensor(cache)) return G4ATTN_EUNSUPPORTED;  // the chunk reads K from the cache
   if ((long)p0 + T > cache->capacity)  // every position must stay readable
     return cache->rolling || shared ? G4ATTN_EINVAL : G4ATTN_ECACHE_OVERFLOW;
   if (B == 0 || T == 0) return G4ATTN_OK;
@@ -338,6 +347,8 @@ int g4attn_decode(const g4attn_layer_desc* desc, const g4attn_cache* cache, cons
   if (st != G4ATTN_OK) return st;
   if (!cache || !q_raw || !q_norm_w || !out) return G4ATTN_EINVAL;
   if ((st = check_cache(L, cache, cache->batch)) != G4ATTN_OK) return st;
+  if (single_tensor(cache) && !decode_mma_supported(L, cache->capacity, 0))
+    return G4ATTN_EUNSUPPORTED;  // K is rebuilt only by the tensor-core split kernel
   if (cache->batch == 0) return G4ATTN_OK;
   const DecodePlan plan = decode_plan(L, cache->capacity);
   const size_t need = decode_partials_bytes(L, cache->batch, plan);
@@ -345,7 +356,8 @@ int g4attn_decode(const g4attn_layer_desc* desc, const g4attn_cache* cache, cons
     return G4ATTN_EWORKSPACE;
   cudaEvent_t ev0, ev1;
   take_timing(&ev0, &ev1);
-  cudaError_t e = launch_decode(L, cache->batch, q_raw, q_norm_w, cache->k, cache->v, cache->len,
+  cudaError_t e = launch_decode(L, cache->batch, q_raw, q_norm_w, cache->k, cache->v,
+                                single_tensor(cache) ? cache->k_norm_w : nullptr, cache->len,
                                 cache->capacity, cache->rolling, cache_mask(cache), plan,
                                 static_cast<float*>(workspace), out, status_ptr(),
                                 static_cast<cudaStream_t>(stream), ev0, ev1);
@@ -359,8 +371,11 @@ int g4attn_decode_noalloc(const g4attn_layer_desc* desc, const g4attn_cache* cac
   if (st != G4ATTN_OK) return st;
   if (!cache || !q_raw || !q_norm_w || !out) return G4ATTN_EINVAL;
   if ((st = check_cache(L, cache, cache->batch)) != G4ATTN_OK) return st;
+  if (single_tensor(cache) && !decode_mma_supported(L, cache->capacity, 0))
+    return G4ATTN_EUNSUPPORTED;
   if (cache->batch == 0) return G4ATTN_OK;
-  return launch_decode_noalloc(L, cache->batch, q_raw, q_norm_w, cache->k, cache->v, cache->len,
+  return launch_decode_noalloc(L, cache->batch, q_raw, q_norm_w, cache->k, cache->v,
+                               single_tensor(cache) ? cache->k_norm_w : nullptr, cache->len,
                                cache->capacity, cache->rolling, cache_mask(cache), out,
                                status_ptr(), static_cast<cudaStream_t>(stream));
 }

@@ -190,18 +190,20 @@ __global__ void __launch_bounds__(128)
 
 template <typename T, int D>
 static cudaError_t run_decode(const LayerCfg& L, int B, const void* q_raw, const void* wq,
-                              const void* cache_k, const void* cache_v, const int32_t* len,
-                              int cap, int rolling, KeyMask km, const DecodePlan& plan,
-                              float* partials, void* out, int* status, cudaStream_t s,
-                              cudaEvent_t ev0, cudaEvent_t ev1) {
+                              const void* cache_k, const void* cache_v, const void* wk_single,
+                              const int32_t* len, int cap, int rolling, KeyMask km,
+                              const DecodePlan& plan, float* partials, void* out, int* status,
+                              cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1) {
   float* part_ml = partials;
   float* part_o = partials + 2 * (size_t)B * L.Hq * plan.n_chunks;
   dim3 grid(plan.n_chunks, L.Hkv, B);
   if (ev0) cudaEventRecord(ev0, s);
   cudaError_t e;
   if (decode_mma_supported(L, cap, rolling)) {
-    e = launch_decode_mma(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, plan,
-                          part_ml, part_o, status, s);
+    e = launch_decode_mma(L, B, q_raw, wq, cache_k, cache_v, wk_single, len, cap, rolling, km,
+                          plan, part_ml, part_o, status, s);
+  } else if (!cache_v) {  // a single-tensor cache needs the tensor-core kernel (host-checked)
+    return cudaErrorInvalidValue;
   } else {
     decode_split_kernel<T, D><<<grid, kDecWarps * 32, 0, s>>>(
         static_cast<const T*>(q_raw), static_cast<const T*>(wq), static_cast<const T*>(cache_k),
@@ -222,17 +224,17 @@ static cudaError_t run_decode(const LayerCfg& L, int B, const void* q_raw, const
 }
 
 cudaError_t launch_decode(const LayerCfg& L, int B, const void* q_raw, const void* wq,
-                          const void* cache_k, const void* cache_v, const int32_t* len, int cap,
-                          int rolling, KeyMask km, const DecodePlan& plan, float* partials,
-                          void* out, int* status, cudaStream_t s, cudaEvent_t ev0,
-                          cudaEvent_t ev1) {
+                          const void* cache_k, const void* cache_v, const void* wk_single,
+                          const int32_t* len, int cap, int rolling, KeyMask km,
+                          const DecodePlan& plan, float* partials, void* out, int* status,
+                          cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1) {
   const bool f32 = L.dtype == 1;
-#define G4_DEC(D)                                                                              \
-  return f32 ? run_decode<float, D>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, \
-                                    plan, partials, out, status, s, ev0, ev1)                   \
-             : run_decode<__nv_bfloat16, D>(L, B, q_raw, wq, cache_k, cache_v, len, cap,      \
-                                            rolling, km, plan, partials, out, status, s, ev0,  \
-                                            ev1)
+#define G4_DEC(D)                                                                             \
+  return f32 ? run_decode<float, D>(L, B, q_raw, wq, cache_k, cache_v, wk_single, len, cap,  \
+                                    rolling, km, plan, partials, out, status, s, ev0, ev1)     \
+             : run_decode<__nv_bfloat16, D>(L, B, q_raw, wq, cache_k, cache_v, wk_single, len, \
+                                            cap, rolling, km, plan, partials, out, status, s, \
+                                            ev0, ev1)
   switch (L.d) {
     case 64: G4_DEC(64);
     case 128: G4_DEC(128);

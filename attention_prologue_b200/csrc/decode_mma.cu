@@ -49,7 +49,10 @@ struct DmLayout {
   static_assert(kStages >= kConsumers, "at least one stage per consumer");
   static constexpr uint32_t kQ = kStages * kStage;         // q_hat [8][D] bf16
   static constexpr uint32_t kBars = kQ + 8 * D * 2;        // full[NS], empty[NS]
-  static constexpr uint32_t kAlloc = kBars + 2 * kStages * 8 + 64;
+  // single-tensor caches: per rotated pair k (< D/2) its frequency (double),
+  // cos and sin of it and the key-norm weights of dims k and k + D/2
+  static constexpr uint32_t kRot = (kBars + 2 * kStages * 8 + 15) & ~15u;
+  static constexpr uint32_t kAlloc = kRot + (D / 2) * 24 + 64;
   static_assert(kConsumers * 8 * D * 4 + kConsumers * 8 * 8 <= kQ, "merge buffer fits");
 };
 
@@ -90,7 +93,14 @@ __device__ __forceinline__ uint32_t tile_off(int key, int dim) {
 
 }  // namespace
 
-template <int D>
+// kSingle: a single-tensor cache of a K=V layer.  The cache holds V =
+// RMSNorm(k_raw) alone and K = RoPE(V * w_k) is rebuilt per tile: w_k folds
+// into the query on the unrotated dims (q.(V*w) = (q*w).V); the rotated pairs
+// of each 16-key tile are computed into the V half of the stage (which the
+// TMA no longer fills), and the S product reads those boxes from there.  The
+// cos/sin of a pair step from key to key by the angle addition formulas
+// (one fp64-reduced sincos per pair and tile).  V is the loaded tile itself.
+template <int D, bool kSingle>
 __global__ void __launch_bounds__(kThreadsDm, 1)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
@@ -99,6 +109,7 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
                       int layer_type, int window, float scale_log2, float cap2, KeyMask km,
                       float eps, int chunk, int nc, float* __restrict__ part_ml,
                       float* __restrict__ part_o, int* status,
+                      const __nv_bfloat16* __restrict__ wk_single, uint32_t rot_boxes,
                       const __grid_constant__ RopeParams rope) {
   using Ly = DmLayout<D>;
   constexpr int NS = Ly::kStages;
@@ -145,10 +156,35 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
         float y0[D / 64], y1[D / 64];
         prologue_vec<__nv_bfloat16, D>(q_raw + ((long)b * Hq + kvh * g + hh) * D, wq, P, &rope,
                                        eps, y0, y1);
+        if constexpr (kSingle) {  // w_k folds into the query on the unrotated pairs
+          float w0[D / 64], w1[D / 64];
+          Vec<__nv_bfloat16, D / 64>::load(wk_single + lane * (D / 64), w0);
+          Vec<__nv_bfloat16, D / 64>::load(wk_single + D / 2 + lane * (D / 64), w1);
+#pragma unroll
+          for (int e = 0; e < D / 64; ++e)
+            if (lane * (D / 64) + e >= rope.rotated_pairs) {
+              y0[e] *= w0[e];
+              y1[e] *= w1[e];
+            }
+        }
         store_vec<__nv_bfloat16, D>(qs + hh * D, y0, y1);
       } else {
         for (int k = lane; k < D; k += 32) qs[hh * D + k] = __float2bfloat16_rn(0.f);
       }
+    }
+  }
+  if constexpr (kSingle) {  // the rotation table of this layer's pairs
+    for (int k = threadIdx.x; k < rope.rotated_pairs; k += blockDim.x) {
+      uint8_t* e = smem + Ly::kRot + k * 24;
+      const double f = rope.inv_freq[k];
+      float sf, cf;
+      rope_sincos(1, f, &sf, &cf);
+      *reinterpret_cast<double*>(e) = f;
+      float* x = reinterpret_cast<float*>(e + 8);
+      x[0] = cf;
+      x[1] = sf;
+      x[2] = __bfloat162float(wk_single[k]);
+      x[3] = __bfloat162float(wk_single[k + D / 2]);
     }
   }
   __syncthreads();
@@ -170,12 +206,13 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
         const int pos = (t0 + i) * kKeys;
         const int slot = rolling ? pos % cap : pos;  // rolling caches: cap % 16 == 0
         const uint32_t st = base + s * Ly::kStage;
-        mbar_arrive_expect_tx(bars + 8 * s, Ly::kStage);
+        mbar_arrive_expect_tx(bars + 8 * s, kSingle ? Ly::kTile : Ly::kStage);
 #pragma unroll
         for (int bx = 0; bx < Ly::kBoxes; ++bx) {
           tma_load_3d(st + bx * Ly::kBox, &tm_k, bars + 8 * s, bx * 64, slot, b * Hkv + kvh);
-          tma_load_3d(st + Ly::kTile + bx * Ly::kBox, &tm_v, bars + 8 * s, bx * 64, slot,
-                      b * Hkv + kvh);
+          if constexpr (!kSingle)
+            tma_load_3d(st + Ly::kTile + bx * Ly::kBox, &tm_v, bars + 8 * s, bx * 64, slot,
+                        b * Hkv + kvh);
         }
         issued = i + 1;
       }
@@ -200,13 +237,49 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
       const int pos0 = (t0 + i) * kKeys;
       if (pos0 + kKeys - 1 > P) {  // last tile: zero V rows past P (never written)
         const int first = P - pos0 + 1;
-        uint8_t* vrow = smem + s * Ly::kStage + Ly::kTile;
+        uint8_t* vrow = smem + s * Ly::kStage + (kSingle ? 0 : Ly::kTile);
         for (int e = lane; e < (kKeys - first) * Ly::kBoxes * 8; e += 32) {
           const int rr = first + e / (Ly::kBoxes * 8), rest = e % (Ly::kBoxes * 8);
           *reinterpret_cast<uint4*>(vrow + (rest >> 3) * Ly::kBox + rr * 128 + (rest & 7) * 16) =
               make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();  // a later TMA refill of this stage comes after these writes
+        __syncwarp();
+      }
+      if constexpr (kSingle) {
+        // K of the rotated pairs of the 16 keys into the V half of the stage:
+        // (a, b) = (V[k] w_k, V[k + D/2] w_(k+D/2)) turned by pos * f_k; the
+        // unrotated dims that share a 64-dim box with rotated ones are copied
+        uint8_t* sk = smem + s * Ly::kStage;
+        uint8_t* sv = sk + Ly::kTile;
+        for (int k = lane; k < rope.rotated_pairs; k += 32) {
+          const uint8_t* e = smem + Ly::kRot + k * 24;
+          const float* x = reinterpret_cast<const float*>(e + 8);
+          const float cf = x[0], sf = x[1], wa = x[2], wb = x[3];
+          float sn, cs;
+          rope_sincos(pos0, *reinterpret_cast<const double*>(e), &sn, &cs);
+          const int da = k, db = k + D / 2;
+#pragma unroll 4
+          for (int j = 0; j < kKeys; ++j) {
+            const uint32_t oa = tile_off(j, da) + (da & 7) * 2, ob = tile_off(j, db) + (db & 7) * 2;
+            const float a = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sk + oa)) * wa;
+            const float bb = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sk + ob)) * wb;
+            *reinterpret_cast<__nv_bfloat16*>(sv + oa) = __float2bfloat16_rn(a * cs - bb * sn);
+            *reinterpret_cast<__nv_bfloat16*>(sv + ob) = __float2bfloat16_rn(a * sn + bb * cs);
+            const float c2 = cs * cf - sn * sf;  // the angle of the next position
+            sn = sn * cf + cs * sf;
+            cs = c2;
+          }
+        }
+        for (uint32_t m = rot_boxes; m; m &= m - 1) {
+          const int bx = __ffs(m) - 1;
+          for (int e = lane; e < kKeys * 64; e += 32) {
+            const int j = e >> 6, dim = bx * 64 + (e & 63);
+            if ((dim % (D / 2)) < rope.rotated_pairs) continue;
+            const uint32_t o = tile_off(j, dim) + (dim & 7) * 2;
+            *reinterpret_cast<__nv_bfloat16*>(sv + o) = *reinterpret_cast<const __nv_bfloat16*>(sk + o);
+          }
+        }
         __syncwarp();
       }
       // S^T (16 keys x 8 heads)
@@ -217,7 +290,9 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           uint32_t a[4];
-          ldsm_x4(kb + tile_off(key, kk * 16 + (mi >> 1) * 8), a);
+          // single-tensor cache: the boxes with rotated dims come from the V half
+          const uint32_t src = (kSingle && ((rot_boxes >> (kk >> 2)) & 1u)) ? vb : kb;
+          ldsm_x4(src + tile_off(key, kk * 16 + (mi >> 1) * 8), a);
           mma16816(sc, a, qb[kk][0], qb[kk][1]);
         }
       }
@@ -273,7 +348,7 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
           acc[mt][2] *= cA;
           acc[mt][3] *= cB;
           uint32_t a[4];
-          ldsm_x4_t(vb + tile_off(key, mt * 16 + (mi & 1) * 8), a);
+          ldsm_x4_t((kSingle ? kb : vb) + tile_off(key, mt * 16 + (mi & 1) * 8), a);
           mma16816(acc[mt], a, pb0, pb1);
         }
       }
@@ -347,38 +422,52 @@ bool decode_mma_supported(const LayerCfg& L, int cap, int rolling) {
 
 template <int D>
 static cudaError_t run_mma(const LayerCfg& L, int B, const void* q_raw, const void* wq,
-                           const void* cache_k, const void* cache_v, const int32_t* len, int cap,
-                           int rolling, KeyMask km, const DecodePlan& plan, float* part_ml,
-                           float* part_o, int* status, cudaStream_t s) {
+                           const void* cache_k, const void* cache_v, const void* wk_single,
+                           const int32_t* len, int cap, int rolling, KeyMask km,
+                           const DecodePlan& plan, float* part_ml, float* part_o, int* status,
+                           cudaStream_t s) {
   using Ly = DmLayout<D>;
+  const bool single = cache_v == nullptr;  // single-tensor cache of a K=V layer
   CUtensorMap tk, tv;
   const uint64_t dims[3] = {(uint64_t)D, (uint64_t)cap, (uint64_t)B * L.Hkv};
   const uint64_t str[2] = {(uint64_t)D * 2, (uint64_t)cap * D * 2};
   const uint32_t box[3] = {64, kKeys, 1};
   if (!make_bf16_map(&tk, cache_k, 3, dims, str, box)) return cudaErrorInvalidValue;
-  if (!make_bf16_map(&tv, cache_v, 3, dims, str, box)) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
+  if (!make_bf16_map(&tv, single ? cache_k : cache_v, 3, dims, str, box))
+    return cudaErrorInvalidValue;
+  // the 64-dim boxes that hold rotated dims (pairs k < R: dims k and k + D/2)
+  uint32_t rot_boxes = 0;
+  for (int k = 0; k < L.rope.rotated_pairs; ++k)
+    rot_boxes |= (1u << (k / 64)) | (1u << ((k + D / 2) / 64));
+  auto kern = single ? decode_mma_kernel<D, true> : decode_mma_kernel<D, false>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.n_chunks, L.Hkv, B);
-  decode_mma_kernel<D><<<grid, kThreadsDm, Ly::kAlloc, s>>>(
+  kern<<<grid, kThreadsDm, Ly::kAlloc, s>>>(
       tk, tv, static_cast<const __nv_bfloat16*>(q_raw), static_cast<const __nv_bfloat16*>(wq), len,
       cap, rolling, L.Hq, L.Hkv, L.layer_type, L.window, L.scale * 1.4426950408889634f,
-      softcap_log2(L), km, L.eps, plan.chunk, plan.n_chunks, part_ml, part_o, status, L.rope);
+      softcap_log2(L), km, L.eps, plan.chunk, plan.n_chunks, part_ml, part_o, status,
+      static_cast<const __nv_bfloat16*>(wk_single), rot_boxes, L.rope);
   count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode_mma(const LayerCfg& L, int B, const void* q_raw, const void* wq,
-                              const void* cache_k, const void* cache_v, const int32_t* len,
-                              int cap, int rolling, KeyMask km, const DecodePlan& plan,
-                              float* part_ml, float* part_o, int* status, cudaStream_t s) {
+                              const void* cache_k, const void* cache_v, const void* wk_single,
+                              const int32_t* len, int cap, int rolling, KeyMask km,
+                              const DecodePlan& plan, float* part_ml, float* part_o,
+                              int* status, cudaStream_t s) {
+#define G4_MMA(D)                                                                          \
+  return run_mma<D>(L, B, q_raw, wq, cache_k, cache_v, wk_single, len, cap, rolling, km, \
+                    plan, part_ml, part_o, status, s)
   switch (L.d) {
-    case 64: return run_mma<64>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, plan, part_ml, part_o, status, s);
-    case 128: return run_mma<128>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, plan, part_ml, part_o, status, s);
-    case 256: return run_mma<256>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, plan, part_ml, part_o, status, s);
-    case 512: return run_mma<512>(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, plan, part_ml, part_o, status, s);
+    case 64: G4_MMA(64);
+    case 128: G4_MMA(128);
+    case 256: G4_MMA(256);
+    case 512: G4_MMA(512);
   }
+#undef G4_MMA
   return cudaErrorInvalidValue;
 }
 

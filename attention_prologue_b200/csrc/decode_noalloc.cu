@@ -49,8 +49,9 @@ static float* decode_scratch_ptr() {
 }
 
 int launch_decode_noalloc(const LayerCfg& L, int B, const void* q_raw, const void* wq,
-                          const void* cache_k, const void* cache_v, const int32_t* len, int cap,
-                          int rolling, KeyMask km, void* out, int* status, cudaStream_t s) {
+                          const void* cache_k, const void* cache_v, const void* wk_single,
+                          const int32_t* len, int cap, int rolling, KeyMask km, void* out,
+                          int* status, cudaStream_t s) {
   DecodePlan plan = decode_plan(L, cap);
   const size_t per_chunk = decode_partials_bytes(L, B, DecodePlan{plan.chunk, 1});
   const size_t max_chunks = kDecodeScratchBytes / per_chunk;
@@ -63,8 +64,8 @@ int launch_decode_noalloc(const LayerCfg& L, int B, const void* q_raw, const voi
   }
   float* scratch = decode_scratch_ptr();
   if (!scratch) return G4ATTN_ECUDA;
-  cudaError_t e = launch_decode(L, B, q_raw, wq, cache_k, cache_v, len, cap, rolling, km, plan,
-                                scratch, out, status, s, nullptr, nullptr);
+  cudaError_t e = launch_decode(L, B, q_raw, wq, cache_k, cache_v, wk_single, len, cap, rolling,
+                                km, plan, scratch, out, status, s, nullptr, nullptr);
   return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
 }
 

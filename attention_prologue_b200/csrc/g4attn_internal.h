@@ -36,7 +36,8 @@ inline float softcap_log2(const LayerCfg& L) {
 }
 
 // Where the key/value prologue writes: [B, Hkv, cap, d]; positions t >= first
-// go to slot (rolling ? t % cap : t).  k == nullptr: no destination.
+// go to slot (rolling ? t % cap : t).  k == nullptr: no destination;
+// v == nullptr: a single-tensor cache of a K=V layer, V alone goes to k.
 struct KVDst {
   void* k;
   void* v;
@@ -123,26 +124,30 @@ struct KeyMask {
   int len;
 };
 
+// cache_v == nullptr: a single-tensor cache (cache_k holds V of a K=V layer;
+// wk_single, the owning layer's key-norm weight, rebuilds K).
 cudaError_t launch_decode(const LayerCfg& L, int B, const void* q_raw, const void* wq,
-                          const void* cache_k, const void* cache_v, const int32_t* len, int cap,
-                          int rolling, KeyMask km, const DecodePlan& plan, float* partials,
-                          void* out, int* status, cudaStream_t s, cudaEvent_t ev0,
-                          cudaEvent_t ev1);
+                          const void* cache_k, const void* cache_v, const void* wk_single,
+                          const int32_t* len, int cap, int rolling, KeyMask km,
+                          const DecodePlan& plan, float* partials, void* out, int* status,
+                          cudaStream_t s, cudaEvent_t ev0, cudaEvent_t ev1);
 
 // Tensor-core split kernel of g4attn_decode (bf16, <= 8 query heads per KV
 // head, rolling caches with capacity % 16 == 0); writes the same partials
 // as the CUDA-core split kernel.
 bool decode_mma_supported(const LayerCfg& L, int cap, int rolling);
 cudaError_t launch_decode_mma(const LayerCfg& L, int B, const void* q_raw, const void* wq,
-                              const void* cache_k, const void* cache_v, const int32_t* len,
-                              int cap, int rolling, KeyMask km, const DecodePlan& plan,
-                              float* part_ml, float* part_o, int* status, cudaStream_t s);
+                              const void* cache_k, const void* cache_v, const void* wk_single,
+                              const int32_t* len, int cap, int rolling, KeyMask km,
+                              const DecodePlan& plan, float* part_ml, float* part_o,
+                              int* status, cudaStream_t s);
 
 // g4attn_decode with the split-KV partials in the library's fixed device
 // array instead of a workspace; returns a g4attn_status code.
 int launch_decode_noalloc(const LayerCfg& L, int B, const void* q_raw, const void* wq,
-                          const void* cache_k, const void* cache_v, const int32_t* len, int cap,
-                          int rolling, KeyMask km, void* out, int* status, cudaStream_t s);
+                          const void* cache_k, const void* cache_v, const void* wk_single,
+                          const int32_t* len, int cap, int rolling, KeyMask km, void* out,
+                          int* status, cudaStream_t s);
 
 // Tensor map of a bf16 tensor with a 128-byte-swizzled box (dims[0]
 // contiguous, strides in bytes for dims 1..rank-1); false on failure.

@@ -45,6 +45,10 @@ __device__ __forceinline__ void put_kv(const KVDst& d, int Hkv, long b, int h, l
   if (!d.k || t < d.first) return;
   const long slot = d.rolling ? t % d.cap : t;
   const long off = (((long)b * Hkv + h) * d.cap + slot) * D;
+  if (!d.v) {  // single-tensor cache of a K=V layer: V alone
+    store_vec<T, D>(static_cast<T*>(d.k) + off, v0, v1);
+    return;
+  }
   store_vec<T, D>(static_cast<T*>(d.k) + off, k0, k1);
   store_vec<T, D>(static_cast<T*>(d.v) + off, v0, v1);
 }
@@ -303,10 +307,13 @@ __global__ void append_kernel(const T* __restrict__ k_raw, const T* __restrict__
   const long src = ((long)b * Hkv + h) * D;
   const long dst = (((long)b * Hkv + h) * cap + slot) * D;
   float y0[D / 64], y1[D / 64];
-  prologue_vec<T, D>(k_raw + src, wk, pos, &rope, eps, y0, y1);
-  store_vec<T, D>(cache_k + dst, y0, y1);
+  if (cache_v) {
+    prologue_vec<T, D>(k_raw + src, wk, pos, &rope, eps, y0, y1);
+    store_vec<T, D>(cache_k + dst, y0, y1);
+  }
+  // V; a single-tensor cache (cache_v == nullptr, K=V layer) keeps V alone
   prologue_vec<T, D>((v_raw ? v_raw : k_raw) + src, nullptr, pos, nullptr, eps, y0, y1);
-  store_vec<T, D>(cache_v + dst, y0, y1);
+  store_vec<T, D>(cache_v ? cache_v + dst : cache_k + dst, y0, y1);
   __syncthreads();  // every warp has read len[b]
   if (threadIdx.x == 0) len[b] = pos + 1;
 }

@@ -49,7 +49,7 @@ class _CCache(ctypes.Structure):
                 ("capacity", ctypes.c_int), ("rolling", ctypes.c_int), ("batch", ctypes.c_int),
                 ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("key_mask", ctypes.c_void_p),
-                ("mask_len", ctypes.c_int)]
+                ("mask_len", ctypes.c_int), ("k_norm_w", ctypes.c_void_p)]
 
 
 _lib = None
@@ -140,21 +140,26 @@ def cache_bytes(batch: int, num_kv_heads: int, capacity: int, head_dim: int,
 class KVCache:
     """A layer's KV cache in device memory owned by torch.  key_mask (uint8
     [batch, mask_len], optional) marks the padding positions of the prompt it
-    holds (0 = padding); later positions are kept."""
+    holds (0 = padding); later positions are kept.  v = None: a single-tensor
+    cache of a K=V layer (k holds V = RMSNorm(k_raw); k_norm_w, the owning
+    layer's key-norm weight, rebuilds K on read)."""
     k: torch.Tensor
-    v: torch.Tensor
+    v: torch.Tensor | None
     len: torch.Tensor
     rolling: bool = False
     key_mask: torch.Tensor | None = None
+    k_norm_w: torch.Tensor | None = None
 
     @classmethod
     def allocate(cls, batch: int, num_kv_heads: int, capacity: int, head_dim: int, *,
                  rolling: bool = False, dtype: torch.dtype = torch.bfloat16,
-                 device="cuda") -> "KVCache":
+                 device="cuda", single: bool = False,
+                 k_norm_w: torch.Tensor | None = None) -> "KVCache":
         shape = (batch, num_kv_heads, capacity, head_dim)
         return cls(torch.empty(shape, dtype=dtype, device=device),
-                   torch.empty(shape, dtype=dtype, device=device),
-                   torch.zeros(batch, dtype=torch.int32, device=device), rolling)
+                   None if single else torch.empty(shape, dtype=dtype, device=device),
+                   torch.zeros(batch, dtype=torch.int32, device=device), rolling,
+                   k_norm_w=k_norm_w)
 
     @property
     def capacity(self) -> int:
@@ -162,7 +167,7 @@ class KVCache:
 
     def c(self) -> _CCache:
         B, Hkv, C, d = self.k.shape
-        if self.v.shape != self.k.shape or self.v.dtype != self.k.dtype:
+        if self.v is not None and (self.v.shape != self.k.shape or self.v.dtype != self.k.dtype):
             raise ValueError("cache k and v differ in shape or dtype")
         if self.len.dtype != torch.int32 or self.len.numel() != B:
             raise ValueError("cache len must be int32 [batch]")
@@ -174,7 +179,8 @@ class KVCache:
             km, mlen = _ptr(self.key_mask, "cache.key_mask"), self.key_mask.shape[1]
         return _CCache(_ptr(self.k, "cache.k"), _ptr(self.v, "cache.v"),
                        _ptr(self.len, "cache.len"), C, int(self.rolling), B, Hkv, d,
-                       _dtype_code(self.k.dtype), km, mlen)
+                       _dtype_code(self.k.dtype), km, mlen,
+                       _ptr(self.k_norm_w, "cache.k_norm_w"))
 
 
 def _check(rc: int, where: str):

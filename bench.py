@@ -21,8 +21,8 @@ on the launching stream; L2 is flushed (a 256 MiB write) before every timed
 prefill step, outside the events; the decode step reads ~36 GB, far more than
 L2.  Barrier + synchronize on both sides; the maximum over ranks is reported.
 With N > 1 every rank runs its own instance (independent sequences, no
-collective on the data path): weak scaling.  NVML clock samples (1 ms
-period) are taken over every timed region.
+collective on the data path): weak scaling.  NVML clock samples (every
+~0.2 ms) are taken over every timed region.
 
 --impl reference times the float64 CPU oracle (the only other implementation
 of this layer) on the same workload and metric, on a bounded row sample.
@@ -86,14 +86,15 @@ def prefill_flops(w: W.PrefillWorkload, ids) -> float:
     return 4.0 * w.layer.head_dim * w.layer.num_heads * allowed_pairs(w, ids)
 
 
-def decode_bytes(L: W.LayerShape, lens, es=2) -> float:
+def decode_bytes(L: W.LayerShape, lens, es=2, tensors=2) -> float:
     """K and V bytes of the keys the new tokens attend to (P = len, after the
-    append) plus q, out and the appended K/V."""
+    append) plus q, out and the appended K/V; tensors=1: a single-tensor cache
+    of a K=V layer (V alone, K rebuilt from it)."""
     n = np.asarray(lens, np.int64) + 1
     if L.layer_type == W.SLIDING:
         n = np.minimum(n, L.window)
-    kv = float(n.sum()) * L.num_kv_heads * L.head_dim * 2 * es
-    return kv + len(lens) * L.head_dim * es * (2 * L.num_heads + 2 * L.num_kv_heads)
+    kv = float(n.sum()) * L.num_kv_heads * L.head_dim * tensors * es
+    return kv + len(lens) * L.head_dim * es * (2 * L.num_heads + tensors * L.num_kv_heads)
 
 
 # ---------------------------------------------------------------------------
@@ -147,7 +148,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.001, paused: bool = False):
+    def __init__(self, index: int, period_s: float = 0.0002, paused: bool = False):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
         self._paused = paused
@@ -510,10 +511,10 @@ def bench_decode(args, dist: Dist, pk: dict, clk: ClockSampler):
     g_split_bytes = decode_bytes(Gl, lens)
     peak = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     achieved = g_split_bytes / (g_ms * 1e-3) / 1e9
-    # DRAM traffic from a smaller capture of the same kernel, scaled by the
-    # bytes it streams (each cached byte is read once; the partials scale too)
-    ratio = profile_field("decode_mma_26b_a4b_global_b4.md", "traffic_per_algorithmic_byte")
-    traffic = None if ratio is None else ratio * g_split_bytes
+    # DRAM traffic of the global layer's split kernel, from a capture of the
+    # same kernel source on this very step (64 sequences, rank 0's lengths)
+    traffic = (profile_field("decode_mma_26b_a4b_global.md", "traffic_bytes_per_launch")
+               if w.batch == 64 and dist.rank == 0 else None)
     res = {"metric": "decode KV-cache GB/s", "value": job_rate(dist.world, nbytes, K, total_ms) / 1e9,
            "unit": "GB/s", "ms_per_step": total_ms / K, "bytes_per_step": nbytes,
            "workload": w.name if w.batch == 64 else f"{w.name}-b{w.batch}", "batch": w.batch, "len_range": [w.len_lo, w.len_hi],
@@ -528,6 +529,61 @@ def bench_decode(args, dist: Dist, pk: dict, clk: ClockSampler):
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = decode_cpu_baseline(w, lens, (S, s_tok, s_cache), (Gl, g_tok, g_cache),
                                                   (X, x_tok))
+    if not args.no_kv_single:
+        # the same step with the global layer's cache stored as V alone (the
+        # K=V single-tensor cache): the global and KV-shared layers read half
+        # the bytes; the sliding layer is unchanged
+        del g_cache
+        torch.cuda.empty_cache()
+        sg = G.KVCache.allocate(w.batch, Gl.num_kv_heads, w.global_capacity, Gl.head_dim,
+                                device=dev, single=True, k_norm_w=g_tok["k_norm_w"])
+        W.fill_cache(sg.k, sg.k, lens, False, g)
+
+        def step1(ev=None):
+            G.g4attn_cache_append(ds, s_cache, s_tok["k_raw"], s_tok["v_raw"], s_tok["k_norm_w"],
+                                  stream)
+            G.g4attn_decode(ds, s_cache, s_tok["q_raw"], s_tok["q_norm_w"], outs["s"], ws_s, stream)
+            G.g4attn_cache_append(dg, sg, g_tok["k_raw"], None, g_tok["k_norm_w"], stream)
+            if ev:
+                G.g4attn_time_next_attention(*ev)
+            G.g4attn_decode(dg, sg, g_tok["q_raw"], g_tok["q_norm_w"], outs["g"], ws_g, stream)
+            G.g4attn_decode(dx, sg, x_tok["q_raw"], x_tok["q_norm_w"], outs["x"], ws_g, stream)
+
+        for _ in range(args.warmup):
+            s_cache.len.copy_(lens_dev)
+            sg.len.copy_(lens_dev)
+            step1()
+        torch.cuda.synchronize()
+        dist.barrier()
+        clk.resume()
+        for i in range(K):
+            s_cache.len.copy_(lens_dev)
+            sg.len.copy_(lens_dev)
+            s0[i].record(stream)
+            step1((a0[i], a1[i]))
+            s1[i].record(stream)
+        torch.cuda.synchronize()
+        clk.pause()
+        dist.barrier()
+        t1 = dist.max(sum(s0[i].elapsed_time(s1[i]) for i in range(K)))
+        status = G.g4attn_get_device_status()
+        if status != G.G4ATTN_OK:
+            raise RuntimeError(f"device status after decode: {G.g4attn_status_string(status)}")
+        g1_ms = statistics.mean(a0[i].elapsed_time(a1[i]) for i in range(K))
+        g1_bytes = decode_bytes(Gl, lens, tensors=1)
+        n1 = decode_bytes(S, lens) + g1_bytes + decode_bytes(X, lens, tensors=1)
+        res["kv_single"] = {
+            "metric": "decode KV-cache GB/s", "cache": "global layer: single-tensor K=V cache",
+            "value": job_rate(dist.world, n1, K, t1) / 1e9, "unit": "GB/s",
+            "ms_per_step": t1 / K, "bytes_per_step": n1,
+            "speedup_vs_two_tensor_step": (total_ms / K) / (t1 / K),
+            "roofline": {"bound": "hbm", "kernel": "decode split-KV (global layer, K rebuilt)",
+                         "achieved": g1_bytes / (g1_ms * 1e-3) / 1e9, "peak": peak,
+                         "unit": "GB/s", "frac": g1_bytes / (g1_ms * 1e-3) / 1e9 / peak,
+                         "traffic": None, "algorithmic_per_launch": g1_bytes,
+                         "avg_launch_ms": g1_ms}}
+        del sg
+        g_cache = None
     del g_cache, s_cache
     torch.cuda.empty_cache()
     return res
@@ -726,6 +782,8 @@ def main(argv=None):
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="sequences of the decode step (default: the workload's 64)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-kv-single", action="store_true",
+                    help="skip the decode step over a single-tensor K=V cache")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls, not a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

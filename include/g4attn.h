@@ -131,7 +131,18 @@ typedef struct {
  * padding key when key_mask[b * mask_len + p] == 0; positions >= mask_len
  * (tokens appended later) are kept.  g4attn_decode reads it; the prefill
  * calls take their mask as an argument.  mask_len is ignored when key_mask
- * is NULL. */
+ * is NULL.
+ *
+ * Single-tensor cache of a K=V layer [K1]: v == NULL.  On a K=V layer both K
+ * and V derive from one raw vector, V = RMSNorm(k_raw) and K =
+ * RoPE(V * w_k), so the cache stores V alone in `k` (half the bytes of the
+ * two-tensor cache the pages' KV-cache table counts [P2]) and k_norm_w
+ * (device [head_dim], the owning layer's key-norm weight) lets a reader
+ * rebuild K.  Non-rolling caches only.  Writers: g4attn_prefill (the cache
+ * is then not the attention's source) and g4attn_cache_append.  Readers:
+ * g4attn_decode / _noalloc on bf16 layers with at most 8 query heads per KV
+ * head (also KV-shared); other readers return G4ATTN_EUNSUPPORTED.
+ * k_norm_w is ignored when v != NULL. */
 typedef struct {
   void *k;
   void *v;
@@ -144,6 +155,7 @@ typedef struct {
   int dtype;
   const uint8_t *key_mask;
   int mask_len;
+  const void *k_norm_w;
 } g4attn_cache;
 
 /* Bytes of device workspace g4attn_prefill needs for this layer and size.

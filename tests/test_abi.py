@@ -230,3 +230,36 @@ def test_prefill_workspace_covers_the_padding_bits():
     assert base >= q_hat + kv + 2 * 16 * 8
     assert lib.g4attn_prefill_chunk_workspace_size(ctypes.byref(d), 2, 100, 900) >= \
         2 * 100 * 8 * 256 * 2 + 2 * 16 * 8
+
+
+def test_single_tensor_cache_validation():
+    """A single-tensor cache (v = NULL) is for K=V layers, non-rolling, with
+    the owning layer's key-norm weight; readers without a kernel for it
+    (prefill reading K from it, a chunk, fp32 decode, more than 8 query
+    heads per KV head) say so with G4ATTN_EUNSUPPORTED."""
+    lib = G.lib()
+    g = desc(layer_type=G.G4ATTN_GLOBAL, head_dim=512, rotary_fraction=0.25, k_eq_v=True,
+             num_heads=8, num_kv_heads=2)
+    def single(d, **kw):
+        c = ccache(d, C=64, **kw)
+        c.v = None
+        c.k_norm_w = FAKE
+        return c
+    c = single(g)
+    assert lib.g4attn_decode_workspace_size(ctypes.byref(g), ctypes.byref(c)) > 0
+    c.k_norm_w = None  # no weight to rebuild K with
+    assert lib.g4attn_decode_workspace_size(ctypes.byref(g), ctypes.byref(c)) == 0
+    s = desc(num_heads=8, num_kv_heads=2)  # not a K=V layer
+    assert lib.g4attn_decode(ctypes.byref(s), ctypes.byref(single(s)), FAKE, FAKE, FAKE, FAKE,
+                             1 << 40, None) == G.G4ATTN_EINVAL
+    # readers without a kernel
+    assert prefill_rc(g, k=None, v=None, cache=single(g)) == G.G4ATTN_EUNSUPPORTED
+    assert chunk_rc(g, v=None, cache=single(g)) == G.G4ATTN_EUNSUPPORTED
+    f32 = desc(layer_type=G.G4ATTN_GLOBAL, head_dim=512, rotary_fraction=0.25, k_eq_v=True,
+               num_heads=8, num_kv_heads=2, dtype=torch.float32)
+    assert lib.g4attn_decode(ctypes.byref(f32), ctypes.byref(single(f32)), FAKE, FAKE, FAKE,
+                             FAKE, 1 << 40, None) == G.G4ATTN_EUNSUPPORTED
+    wide = desc(layer_type=G.G4ATTN_GLOBAL, head_dim=512, rotary_fraction=0.25, k_eq_v=True,
+                num_heads=32, num_kv_heads=2)
+    assert lib.g4attn_decode_noalloc(ctypes.byref(wide), ctypes.byref(single(wide)), FAKE, FAKE,
+                                     FAKE, None) == G.G4ATTN_EUNSUPPORTED
