@@ -25,7 +25,7 @@ _SRC = os.path.join(_HERE, "g4attn_oracle.c")
 _LIB = os.path.join(_HERE, "libg4attn_oracle.so")
 
 BF16, FP32, FP64 = 0, 1, 2
-SLIDING, GLOBAL = 0, 1
+SLIDING, GLOBAL, BIDIRECTIONAL = 0, 1, 2
 ROPE_ZEROPAD, ROPE_PREFIX = 0, 1
 
 
@@ -354,7 +354,10 @@ def decode(layer_q: Layer, q_raw, wq, cache_k, cache_v, capacity: int, rolling: 
     new token is appended at position lens[b]; without it (KV-shared layer) the
     cache already holds it at lens[b]-1.  attention_mask [B, mask_len] (1 = keep,
     0 = padding) drops the padding keys among positions 0..mask_len-1; later
-    positions are kept.  Returns float64 [n_seqs, Hq, d]."""
+    positions are kept.  Returns float64 [n_seqs, Hq, d].  A bidirectional
+    (vision-tower) layer has no decode step."""
+    if BIDIRECTIONAL in (layer_q.layer_type, (layer_kv or layer_q).layer_type):
+        raise ValueError("a bidirectional layer has no decode step")
     q, dt = _raw(q_raw)
     w, wdt = _raw(wq)
     ck, cdt = _raw(cache_k)

@@ -50,12 +50,13 @@
 
 #define OR_SLIDING 0
 #define OR_GLOBAL 1
+#define OR_BIDIRECTIONAL 2 /* the vision tower's attention: every key of the sequence */
 
 #define OR_ROPE_ZEROPAD 0 /* the build's reading: zero-padded frequency vector */
 #define OR_ROPE_PREFIX 1  /* alternative reading: rotate the first fraction*d dims */
 
 typedef struct {
-  int layer_type;          /* OR_SLIDING or OR_GLOBAL */
+  int layer_type;          /* OR_SLIDING, OR_GLOBAL or OR_BIDIRECTIONAL */
   int window;              /* keys a sliding query sees, itself included */
   double rotary_fraction;  /* 1.0 on sliding layers, 0.25 on global layers */
   double rope_theta;       /* 1e4 sliding, 1e6 global */
@@ -174,12 +175,20 @@ void or_prologue_kv(const or_layer *L, const void *k_raw, const void *v_raw,
  * Sliding row inside an image block [s, e): the window united with the whole
  * block (both contain i, so the union is an interval).
  * Global row: every earlier position and itself; block ids are ignored.
+ * Bidirectional row (the vision tower's ViT attention, "gemma4-pt-claude"
+ * README, "Key architectural features"): every one of the T positions; block
+ * ids are ignored.
  * ids is the row of block ids of this sequence (-1 = text) or NULL. */
 void or_interval(const or_layer *L, const int *ids, int T, int i, int *lo,
                  int *hi) {
   if (L->layer_type == OR_GLOBAL) {
     *lo = 0;
     *hi = i;
+    return;
+  }
+  if (L->layer_type == OR_BIDIRECTIONAL) {
+    *lo = 0;
+    *hi = T - 1;
     return;
   }
   int w = L->window + (L->window_plus_one ? 1 : 0);

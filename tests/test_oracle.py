@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import oracle
-from oracle import GLOBAL, ROPE_PREFIX, SLIDING, Layer
+from oracle import BIDIRECTIONAL, GLOBAL, ROPE_PREFIX, SLIDING, Layer
 
 RNG = np.random.default_rng(1234)
 
@@ -92,6 +92,8 @@ def dense_reference(L, q, k, v, wq, wk, ids, keep=None):
     for b in range(B):
         if L.layer_type == GLOBAL:
             allowed = j <= i
+        elif L.layer_type == BIDIRECTIONAL:
+            allowed = np.ones((T, T), bool)
         else:
             allowed = (j <= i) & (i - j < L.window)
             if ids is not None:
@@ -745,3 +747,80 @@ def test_attend_rows_from_the_oracles_own_prologue_is_prefill(case):
         np.testing.assert_array_equal(qh[1, t, 2 % L.num_heads],
                                       oracle.prologue_q(L, q[1, p0 + t, 2 % L.num_heads], wq,
                                                         p0 + t))
+
+
+# ---------------------------------------------------------------------------
+# the bidirectional (vision-tower) layer: every query sees every key of its
+# sequence ("gemma4-pt-claude" README, "Key architectural features": a
+# ViT-style encoder with bidirectional attention; "Attention Backend Notes":
+# the tower's softmax scale is 1.0)
+
+def bidirectional_layer(**kw):
+    base = dict(layer_type=BIDIRECTIONAL, rotary_fraction=1.0, rope_theta=1e4, num_heads=4,
+                num_kv_heads=4, head_dim=16, softmax_scale=1.0, rms_eps=1e-6)
+    base.update(kw)
+    return Layer(**base)
+
+
+@pytest.mark.parametrize("pad", [False, True])
+def test_bidirectional_matches_the_dense_reference(pad):
+    rng = np.random.default_rng(31)
+    L = bidirectional_layer(num_heads=6, num_kv_heads=2)
+    B, T = 2, 29
+    q, k, v, wq, wk = inputs(L, B, T, rng)
+    keep = (rng.random((B, T)) > 0.3).astype(np.uint8) if pad else None
+    got = oracle.prefill(L, q, k, v, wq, wk, attention_mask=keep)
+    ref = dense_reference(L, q, k, v, wq, wk, None, keep)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_bidirectional_zero_query_gives_the_mean_of_every_value():
+    """q = 0: uniform weights over all T keys, so every row -- the first one
+    included -- is the mean of all normalised values (a causal row 0 would
+    return v_0)."""
+    L = bidirectional_layer()
+    T = 17
+    q, k, v, wq, wk = inputs(L, 1, T)
+    got = oracle.prefill(L, np.zeros_like(q), k, v, wq, wk)
+    _, vh = oracle.prefill_kv(L, k, v, wk)
+    mean = vh[0].mean(axis=0)  # [Hkv, d]
+    for i in range(T):
+        np.testing.assert_allclose(got[0, i], mean, rtol=0, atol=1e-13)
+
+
+def test_bidirectional_last_row_is_the_causal_last_row_and_block_ids_are_ignored():
+    rng = np.random.default_rng(32)
+    L = bidirectional_layer(rotary_fraction=0.25, rope_theta=1e6)
+    T = 21
+    q, k, v, wq, wk = inputs(L, 1, T, rng)
+    bi = oracle.prefill(L, q, k, v, wq, wk)
+    ca = oracle.prefill(global_layer(**{f: getattr(L, f) for f in (
+        "rotary_fraction", "rope_theta", "k_eq_v", "num_heads", "num_kv_heads", "head_dim",
+        "softmax_scale")}), q, k, v, wq, wk)
+    assert np.array_equal(bi[0, T - 1], ca[0, T - 1])  # both see keys 0..T-1
+    assert not np.allclose(bi[0, 0], ca[0, 0])
+    ids = ids_with_blocks(1, T, [(3, 9)])
+    assert np.array_equal(oracle.prefill(L, q, k, v, wq, wk, block_ids=ids), bi)
+
+
+def test_bidirectional_rows_do_not_depend_on_the_key_order():
+    """From given post-prologue vectors (no RoPE), a bidirectional row is a
+    function of the key set: permuting the keys (K and V together) leaves
+    every output unchanged."""
+    rng = np.random.default_rng(33)
+    L = bidirectional_layer(num_heads=4, num_kv_heads=2)
+    B, T, d = 1, 19, L.head_dim
+    qh = rng.standard_normal((B, T, 4, d))
+    kh = rng.standard_normal((B, T, 2, d))
+    vh = rng.standard_normal((B, T, 2, d))
+    perm = rng.permutation(T)
+    a = oracle.attend_rows(L, qh, kh, vh, 0)
+    b = oracle.attend_rows(L, qh, kh[:, perm], vh[:, perm], 0)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-13)
+
+
+def test_bidirectional_layer_has_no_decode():
+    L = bidirectional_layer()
+    with pytest.raises(ValueError):
+        oracle.decode(L, np.zeros((1, 1, 4, 16), np.float32), np.ones(16, np.float32),
+                      np.zeros((1, 4, 4, 16)), np.zeros((1, 4, 4, 16)), 4, False, [1])
