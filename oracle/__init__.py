@@ -302,6 +302,50 @@ def prologue_q_all(layer: Layer, q_raw, wq, p0: int = 0) -> np.ndarray:
     return out
 
 
+def _f64(x) -> np.ndarray:
+    """The exact values of a bf16 / fp32 / fp64 tensor or array as float64."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.detach().cpu().double().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x, np.float64)
+
+
+def qkv_prologue(layer: Layer, x, w_qkv, wq, wk=None, p0: int = 0, with_kv: bool = True):
+    """The projection in front of the layer, then its prologue ("Gemma 4"
+    overview blog, "Shared KV Cache": the key and value projections produce
+    the K/V a layer stores; "Gemma 4" Keras docs, "What changed from Gemma 3":
+    the prologue).  raw = x W^T is one float64 matmul of the exact input
+    values (a library primitive standing for the projection; the products of
+    bf16 values are exact in float64), split by rows of W into the num_heads
+    query heads, then (with_kv) the num_kv_heads key heads and, unless k_eq_v,
+    the num_kv_heads value heads; then prologue_q_all and prefill_kv at
+    positions p0 .. p0 + T - 1.
+
+    x [B, T, hidden], w_qkv [n_heads * d, hidden].  Returns float64
+    (q_hat [B, T, Hq, d], k_hat, v_hat [B, T, Hkv, d]); k_hat, v_hat are None
+    without KV heads."""
+    X = _f64(x)
+    Wm = _f64(w_qkv)
+    B, T, _ = X.shape
+    Hq, Hkv, d = layer.num_heads, layer.num_kv_heads, layer.head_dim
+    n_heads = Hq + ((Hkv if layer.k_eq_v else 2 * Hkv) if with_kv else 0)
+    if Wm.shape[0] != n_heads * d or Wm.shape[1] != X.shape[2]:
+        raise ValueError("w_qkv must be [n_heads * d, hidden]")
+    raw = X @ Wm.T
+    qh = prologue_q_all(layer, np.ascontiguousarray(raw[..., :Hq * d].reshape(B, T, Hq, d)),
+                        wq, p0)
+    if not with_kv:
+        return qh, None, None
+    k_raw = np.ascontiguousarray(raw[..., Hq * d:(Hq + Hkv) * d].reshape(B, T, Hkv, d))
+    v_raw = None if layer.k_eq_v else np.ascontiguousarray(
+        raw[..., (Hq + Hkv) * d:(Hq + 2 * Hkv) * d].reshape(B, T, Hkv, d))
+    kh, vh = prefill_kv(layer, k_raw, v_raw, wk, p0=p0)
+    return qh, kh, vh
+
+
 def attend_rows(layer: Layer, qhat, khat, vhat, p0: int = 0, block_ids=None, rows=None,
                 nthreads: int | None = None, attention_mask=None) -> np.ndarray:
     """The attention of prefill_chunk_rows from given post-prologue queries

@@ -824,3 +824,50 @@ def test_bidirectional_layer_has_no_decode():
     with pytest.raises(ValueError):
         oracle.decode(L, np.zeros((1, 1, 4, 16), np.float32), np.ones(16, np.float32),
                       np.zeros((1, 4, 4, 16)), np.zeros((1, 4, 4, 16)), 4, False, [1])
+
+
+# ---------------------------------------------------------------------------
+# the QKV projection in front of the prologue
+
+@pytest.mark.parametrize("mk", [sliding_layer, global_layer, bidirectional_layer])
+def test_qkv_projection_by_a_permutation_is_the_prologue_of_permuted_inputs(mk):
+    """W a (non-symmetric) permutation matrix: raw = x W^T picks coordinate
+    perm[j] of x for output j, so the result is the prologue of those raw
+    vectors, bit for bit.  A transposed W (x W picks perm^-1) or a wrong head
+    order (Q rows, then K, then V) fails."""
+    rng = np.random.default_rng(41)
+    L = mk()
+    Hq, Hkv, d = L.num_heads, L.num_kv_heads, L.head_dim
+    n = Hq + (Hkv if L.k_eq_v else 2 * Hkv)
+    B, T, hidden = 2, 9, n * d
+    x = f32(B, T, hidden, rng=rng)
+    perm = rng.permutation(hidden)
+    Wm = np.zeros((hidden, hidden), np.float32)
+    Wm[np.arange(hidden), perm] = 1.0
+    wq, wk = f32(d, rng=rng), f32(d, rng=rng)
+    qh, kh, vh = oracle.qkv_prologue(L, x, Wm, wq, wk, p0=5)
+    raw = x[..., perm].astype(np.float64)
+    q_raw = raw[..., :Hq * d].reshape(B, T, Hq, d)
+    k_raw = raw[..., Hq * d:(Hq + Hkv) * d].reshape(B, T, Hkv, d)
+    v_raw = None if L.k_eq_v else raw[..., (Hq + Hkv) * d:].reshape(B, T, Hkv, d)
+    assert np.array_equal(qh, oracle.prologue_q_all(L, q_raw, wq, 5))
+    k2, v2 = oracle.prefill_kv(L, k_raw, v_raw, wk, p0=5)
+    assert np.array_equal(kh, k2) and np.array_equal(vh, v2)
+
+
+def test_qkv_projection_is_scale_free_and_queries_only_without_kv():
+    """RMSNorm removes a positive scale of x (eps = 0: exactly up to rounding);
+    without KV heads W holds the query rows alone."""
+    rng = np.random.default_rng(42)
+    L = global_layer(rms_eps=0.0)
+    Hq, d = L.num_heads, L.head_dim
+    hidden = 48
+    x = f32(1, 7, hidden, rng=rng)
+    Wm = f32(Hq * d, hidden, rng=rng)
+    wq = f32(d, rng=rng)
+    a, k, v = oracle.qkv_prologue(L, x, Wm, wq, with_kv=False)
+    assert k is None and v is None
+    b, _, _ = oracle.qkv_prologue(L, 3.5 * x.astype(np.float64), Wm, wq, with_kv=False)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    with pytest.raises(ValueError):
+        oracle.qkv_prologue(L, x, Wm, wq, f32(d, rng=rng))  # KV rows missing
