@@ -2,6 +2,7 @@
 // validation, workspace layout and kernel launches on the caller's stream.
 // Nothing here allocates device memory or waits for the device, except
 // g4attn_get_device_status.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -69,7 +70,9 @@ static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 // Validate a layer descriptor and derive the kernels' view of it.
 static int make_cfg(const g4attn_layer_desc* d, LayerCfg* L) {
   if (!d) return G4ATTN_EINVAL;
-  if (d->layer_type != G4ATTN_SLIDING && d->layer_type != G4ATTN_GLOBAL) return G4ATTN_EINVAL;
+  if (d->layer_type != G4ATTN_SLIDING && d->layer_type != G4ATTN_GLOBAL &&
+      d->layer_type != G4ATTN_BIDIRECTIONAL)
+    return G4ATTN_EINVAL;
   if (d->dtype != G4ATTN_BF16 && d->dtype != G4ATTN_FP32) return G4ATTN_EINVAL;
   if (d->head_dim < 2 || (d->head_dim & 1)) return G4ATTN_EINVAL;
   if (d->num_heads < 1 || d->num_kv_heads < 1) return G4ATTN_EINVAL;
@@ -136,12 +139,12 @@ struct PrefillWs {
 
 // Tk: key positions the call's rows may see (T, or p0 + T for a chunk).
 static PrefillWs prefill_ws(const LayerCfg& L, int B, int T, bool need_kv, bool intervals,
-                            bool mask, int Tk) {
+                            bool mask, int Tk, bool with_q = true) {
   PrefillWs w;
   const size_t es = elem_size(L.dtype);
   size_t off = 0;
   w.q_hat = off;
-  off += align256((size_t)B * T * L.Hq * L.d * es);
+  if (with_q) off += align256((size_t)B * T * L.Hq * L.d * es);
   w.kv = off;
   if (need_kv) off += 2 * align256((size_t)B * T * L.Hkv * L.d * es);
   w.intervals = off;
@@ -173,7 +176,7 @@ extern "C" {
 size_t g4attn_prefill_workspace_size(const g4attn_layer_desc* desc, int B, int T) {
   LayerCfg L;
   if (make_cfg(desc, &L) != G4ATTN_OK || B < 0 || T < 0) return 0;
-  return prefill_ws(L, B, T, true, L.layer_type == G4ATTN_SLIDING, true, T).total;
+  return prefill_ws(L, B, T, true, L.layer_type != G4ATTN_GLOBAL, true, T).total;
 }
 
 size_t g4attn_decode_workspace_size(const g4attn_layer_desc* desc, const g4attn_cache* cache) {
@@ -211,7 +214,8 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
   // attention reads keys from the cache when it holds K and V of positions
   // 0..T-1 at slots 0..T-1, otherwise from scratch
   const bool cache_is_src = cache && cache->capacity >= T && !single_tensor(cache);
-  const bool intervals = L.layer_type == G4ATTN_SLIDING && image_block_ids != nullptr;
+  const bool bidir = L.layer_type == G4ATTN_BIDIRECTIONAL;
+  const bool intervals = (L.layer_type == G4ATTN_SLIDING && image_block_ids != nullptr) || bidir;
   PrefillWs w = prefill_ws(L, B, T, !cache_is_src, intervals, attention_mask != nullptr, T);
   if (!workspace || ws_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return G4ATTN_EWORKSPACE;
@@ -245,8 +249,9 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
     int32_t* lo = reinterpret_cast<int32_t*>(ws + w.intervals);
     int32_t* hi = reinterpret_cast<int32_t*>(ws + w.intervals +
                                              align256((size_t)B * T * sizeof(int32_t)));
-    if (launch_block_intervals(L, B, T, image_block_ids, lo, hi, s) != cudaSuccess)
-      return G4ATTN_ECUDA;
+    e = bidir ? launch_chunk_intervals(L, B, T, 0, nullptr, lo, hi, s)
+              : launch_block_intervals(L, B, T, image_block_ids, lo, hi, s);
+    if (e != cudaSuccess) return G4ATTN_ECUDA;
     rows = {lo, hi};
   }
   KeyBits kb;
@@ -324,11 +329,90 @@ int g4attn_prefill_chunk(const g4attn_layer_desc* desc, int B, int T, int p0, co
   return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
 }
 
+int g4attn_qkv_prologue(const g4attn_layer_desc* desc, int B, int T, int p0, const void* x,
+                        int hidden, const void* w_qkv, const void* q_norm_w,
+                        const void* k_norm_w, void* q_hat, g4attn_cache* cache, void* stream) {
+  LayerCfg L;
+  int st = make_cfg(desc, &L);
+  if (st != G4ATTN_OK) return st;
+  if (B < 0 || T < 0 || p0 < 0) return G4ATTN_EINVAL;
+  if (!x || !w_qkv || !q_norm_w || !q_hat) return G4ATTN_EINVAL;
+  if (hidden < 8 || hidden % 8 != 0) return G4ATTN_EINVAL;  // rows of 16-byte multiples
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w_qkv) |
+       reinterpret_cast<uintptr_t>(q_hat)) & 15)
+    return G4ATTN_EINVAL;
+  if (L.dtype != G4ATTN_BF16) return G4ATTN_EUNSUPPORTED;  // the tensor-core path is bf16
+  if ((long)B * T > INT32_MAX) return G4ATTN_EINVAL;
+  KVDst kv{nullptr, nullptr, 1, 0, 0};
+  int n_heads = L.Hq;
+  if (cache) {
+    if (!k_norm_w) return G4ATTN_EINVAL;
+    if ((st = check_cache(L, cache, B)) != G4ATTN_OK) return st;
+    if (!cache->rolling && (long)p0 + T > cache->capacity) return G4ATTN_ECACHE_OVERFLOW;
+    // a rolling cache keeps the last `capacity` positions of the call
+    const long first = cache->rolling ? (long)p0 + T - cache->capacity : 0;
+    kv = {cache->k, cache->v, cache->capacity, cache->rolling, (int)std::max(0L, first)};
+    n_heads += L.k_eq_v ? L.Hkv : 2 * L.Hkv;
+  }
+  if (B == 0 || T == 0) return G4ATTN_OK;
+  cudaError_t e = launch_qkv_prologue(L, B, T, p0, x, hidden, w_qkv, n_heads, q_norm_w,
+                                      cache ? k_norm_w : nullptr, q_hat, kv,
+                                      cache ? cache->len : nullptr, status_ptr(),
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
+}
+
+size_t g4attn_attend_workspace_size(const g4attn_layer_desc* desc, int B, int T, int p0) {
+  LayerCfg L;
+  if (make_cfg(desc, &L) != G4ATTN_OK || B < 0 || T < 0 || p0 < 0) return 0;
+  return prefill_ws(L, B, T, false, true, true, p0 + T, false).total;
+}
+
+int g4attn_attend(const g4attn_layer_desc* desc, int B, int T, int p0, const void* q_hat,
+                  const int32_t* image_block_ids, const uint8_t* attention_mask,
+                  const g4attn_cache* cache, void* out, void* workspace, size_t ws_bytes,
+                  void* stream) {
+  LayerCfg L;
+  int st = make_cfg(desc, &L);
+  if (st != G4ATTN_OK) return st;
+  if (B < 0 || T < 0 || p0 < 0) return G4ATTN_EINVAL;
+  if (!q_hat || !out || !cache) return G4ATTN_EINVAL;
+  if ((st = check_cache(L, cache, B)) != G4ATTN_OK) return st;
+  if (single_tensor(cache)) return G4ATTN_EUNSUPPORTED;  // reads K from the cache
+  if ((long)p0 + T > cache->capacity) return G4ATTN_EINVAL;  // positions must be at slot = pos
+  if (B == 0 || T == 0) return G4ATTN_OK;
+  PrefillWs w = prefill_ws(L, B, T, false, true, attention_mask != nullptr, p0 + T, false);
+  if (!workspace || ws_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return G4ATTN_EWORKSPACE;
+  char* ws = static_cast<char*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* lo = reinterpret_cast<int32_t*>(ws + w.intervals);
+  int32_t* hi =
+      reinterpret_cast<int32_t*>(ws + w.intervals + align256((size_t)B * T * sizeof(int32_t)));
+  cudaError_t e = launch_chunk_intervals(
+      L, B, T, p0, L.layer_type == G4ATTN_SLIDING ? image_block_ids : nullptr, lo, hi, s);
+  if (e != cudaSuccess) return G4ATTN_ECUDA;
+  const KVSrc src{cache->k, cache->v, cache->capacity, p0 + T};
+  const RowIntervals rows{lo, hi};
+  KeyBits kb;
+  if (padding_bits(w, ws, B, p0 + T, attention_mask, &kb, s) != cudaSuccess)
+    return G4ATTN_ECUDA;
+  cudaEvent_t ev0, ev1;
+  take_timing(&ev0, &ev1);
+  if (ev0) cudaEventRecord(ev0, s);
+  e = attention_sm100_supported(L)
+          ? launch_attention_sm100(L, B, T, q_hat, src, rows, kb, out, status_ptr(), s)
+          : launch_attention_simt(L, B, T, q_hat, src, rows, kb, out, s);
+  if (ev1) cudaEventRecord(ev1, s);
+  return e == cudaSuccess ? G4ATTN_OK : G4ATTN_ECUDA;
+}
+
 int g4attn_cache_append(const g4attn_layer_desc* desc, g4attn_cache* cache, const void* k_raw,
                         const void* v_raw, const void* k_norm_w, void* stream) {
   LayerCfg L;
   int st = make_cfg(desc, &L);
   if (st != G4ATTN_OK) return st;
+  if (L.layer_type == G4ATTN_BIDIRECTIONAL) return G4ATTN_EUNSUPPORTED;  // no decode step
   if (!cache || !k_raw || !k_norm_w) return G4ATTN_EINVAL;
   if ((v_raw == nullptr) != (L.k_eq_v == 1)) return G4ATTN_EINVAL;
   if ((st = check_cache(L, cache, cache->batch)) != G4ATTN_OK) return st;
@@ -345,6 +429,7 @@ int g4attn_decode(const g4attn_layer_desc* desc, const g4attn_cache* cache, cons
   LayerCfg L;
   int st = make_cfg(desc, &L);
   if (st != G4ATTN_OK) return st;
+  if (L.layer_type == G4ATTN_BIDIRECTIONAL) return G4ATTN_EUNSUPPORTED;  // no decode step
   if (!cache || !q_raw || !q_norm_w || !out) return G4ATTN_EINVAL;
   if ((st = check_cache(L, cache, cache->batch)) != G4ATTN_OK) return st;
   if (single_tensor(cache) && !decode_mma_supported(L, cache->capacity, 0))
@@ -369,6 +454,7 @@ int g4attn_decode_noalloc(const g4attn_layer_desc* desc, const g4attn_cache* cac
   LayerCfg L;
   int st = make_cfg(desc, &L);
   if (st != G4ATTN_OK) return st;
+  if (L.layer_type == G4ATTN_BIDIRECTIONAL) return G4ATTN_EUNSUPPORTED;  // no decode step
   if (!cache || !q_raw || !q_norm_w || !out) return G4ATTN_EINVAL;
   if ((st = check_cache(L, cache, cache->batch)) != G4ATTN_OK) return st;
   if (single_tensor(cache) && !decode_mma_supported(L, cache->capacity, 0))

@@ -49,11 +49,26 @@ struct DmLayout {
   static_assert(kStages >= kConsumers, "at least one stage per consumer");
   static constexpr uint32_t kQ = kStages * kStage;         // q_hat [8][D] bf16
   static constexpr uint32_t kBars = kQ + 8 * D * 2;        // full[NS], empty[NS]
-  // single-tensor caches: per rotated pair k (< D/2) its frequency (double),
-  // cos and sin of it and the key-norm weights of dims k and k + D/2
-  static constexpr uint32_t kRot = (kBars + 2 * kStages * 8 + 15) & ~15u;
-  static constexpr uint32_t kAlloc = kRot + (D / 2) * 24 + 64;
-  static_assert(kConsumers * 8 * D * 4 + kConsumers * 8 * 8 <= kQ, "merge buffer fits");
+  static constexpr uint32_t kAlloc = kBars + 2 * kStages * 8 + 64;
+  static constexpr uint32_t kMerge = kConsumers * 8 * D * 4 + kConsumers * 8 * 8;
+  static_assert(kMerge <= kQ, "merge buffer fits");
+};
+
+constexpr int kRebuilders = 2;  // single-tensor caches: warps that rebuild K
+
+// Shared-memory plan of a single-tensor decode (set by the host: the ring's
+// stage holds the loaded V tile and one rebuilt K box per box that has
+// rotated dims).
+struct DmSingle {
+  int ns;              // stages (a multiple of 4)
+  uint32_t stage;      // bytes per stage
+  uint32_t q, bars;    // q_hat [8][D]; full, empty, ready [NS] each
+  uint32_t freq;       // [R] double: the rotated pairs' frequencies
+  uint32_t wab;        // [R] float2: (w_k[k], w_k[k + D/2])
+  uint32_t box_slot;   // 4 bits per 64-dim box: its rebuilt slot, 15 = loaded tile
+  uint32_t slot_box;   // 4 bits per rebuilt slot: its box
+  int nrb;             // rebuilt boxes
+  int nw;              // bf16 pair-words per half that the rotation covers
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
@@ -95,13 +110,14 @@ __device__ __forceinline__ uint32_t tile_off(int key, int dim) {
 
 // kSingle: a single-tensor cache of a K=V layer.  The cache holds V =
 // RMSNorm(k_raw) alone and K = RoPE(V * w_k) is rebuilt per tile: w_k folds
-// into the query on the unrotated dims (q.(V*w) = (q*w).V); the rotated pairs
-// of each 16-key tile are computed into the V half of the stage (which the
-// TMA no longer fills), and the S product reads those boxes from there.  The
-// cos/sin of a pair step from key to key by the angle addition formulas
-// (one fp64-reduced sincos per pair and tile).  V is the loaded tile itself.
+// into the query on the unrotated dims (q.(V*w) = (q*w).V), so only the
+// 64-dim boxes that hold rotated dims are rebuilt, by two extra warps, into
+// slots after the loaded tile; the S product reads those boxes from there.
+// The angle of key pos0 + j is pos0 f then j f: cos/sin of pos0 f come from
+// one fp64-reduced sincos per pair and tile, those of j f (with w_k folded
+// in) from a per-CTA table.  V is the loaded tile itself.
 template <int D, bool kSingle>
-__global__ void __launch_bounds__(kThreadsDm, 1)
+__global__ void __launch_bounds__(kThreadsDm + (kSingle ? kRebuilders * 32 : 0), 1)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __nv_bfloat16* __restrict__ q_raw, const __nv_bfloat16* __restrict__ wq,
@@ -109,17 +125,18 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
                       int layer_type, int window, float scale_log2, float cap2, KeyMask km,
                       float eps, int chunk, int nc, float* __restrict__ part_ml,
                       float* __restrict__ part_o, int* status,
-                      const __nv_bfloat16* __restrict__ wk_single, uint32_t rot_boxes,
+                      const __nv_bfloat16* __restrict__ wk_single, DmSingle sp,
                       const __grid_constant__ RopeParams rope) {
   using Ly = DmLayout<D>;
-  constexpr int NS = Ly::kStages;
+  const int NS = kSingle ? sp.ns : Ly::kStages;
+  const uint32_t kStageB = kSingle ? sp.stage : Ly::kStage;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // the swizzled boxes assume a 1024-byte aligned base
     if (threadIdx.x == 0) record_status(status, G4ATTN_EDEVICE);
     return;
   }
   const uint32_t base = smem_u32(smem);
-  const uint32_t bars = base + Ly::kBars;
+  const uint32_t bars = base + (kSingle ? sp.bars : Ly::kBars);
   __shared__ int s_abort;
   volatile int* abort = &s_abort;
 
@@ -144,12 +161,13 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(bars + 8 * s, 1);             // full: producer's expect_tx
       mbar_init(bars + 8 * (NS + s), 1);      // empty: the consuming warp
+      if (kSingle) mbar_init(bars + 8 * (2 * NS + s), 32);  // ready: a rebuilding warp
     }
     s_abort = 0;
     fence_barrier_init();
   }
   // query prologue (RMSNorm * w_q, RoPE at P) of the g heads into q_hat; rows g..7 zero
-  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem + Ly::kQ);
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem + (kSingle ? sp.q : Ly::kQ));
   if (warp < kConsumers) {
     for (int hh = warp; hh < 8; hh += kConsumers) {
       if (hh < g) {
@@ -173,18 +191,14 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
       }
     }
   }
-  if constexpr (kSingle) {  // the rotation table of this layer's pairs
+  if constexpr (kSingle) {
+    // per rotated pair k: its frequency and (w_k[k], w_k[k + D/2]), in shared
+    // memory (lane-indexed reads of the kernel's parameter space serialise)
+    double* fq = reinterpret_cast<double*>(smem + sp.freq);
+    float2* wab = reinterpret_cast<float2*>(smem + sp.wab);
     for (int k = threadIdx.x; k < rope.rotated_pairs; k += blockDim.x) {
-      uint8_t* e = smem + Ly::kRot + k * 24;
-      const double f = rope.inv_freq[k];
-      float sf, cf;
-      rope_sincos(1, f, &sf, &cf);
-      *reinterpret_cast<double*>(e) = f;
-      float* x = reinterpret_cast<float*>(e + 8);
-      x[0] = cf;
-      x[1] = sf;
-      x[2] = __bfloat162float(wk_single[k]);
-      x[3] = __bfloat162float(wk_single[k + D / 2]);
+      fq[k] = rope.inv_freq[k];
+      wab[k] = make_float2(__bfloat162float(wk_single[k]), __bfloat162float(wk_single[k + D / 2]));
     }
   }
   __syncthreads();
@@ -205,7 +219,7 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
         if (!mbar_wait(bars + 8 * (NS + s), ((i / NS) & 1) ^ 1, abort)) break;
         const int pos = (t0 + i) * kKeys;
         const int slot = rolling ? pos % cap : pos;  // rolling caches: cap % 16 == 0
-        const uint32_t st = base + s * Ly::kStage;
+        const uint32_t st = base + s * kStageB;
         mbar_arrive_expect_tx(bars + 8 * s, kSingle ? Ly::kTile : Ly::kStage);
 #pragma unroll
         for (int bx = 0; bx < Ly::kBoxes; ++bx) {
@@ -220,7 +234,123 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
         for (int i = max(0, issued - NS); i < issued; ++i)
           mbar_wait(bars + 8 * (i % NS), (i / NS) & 1, nullptr);
     }
-  } else {
+  } else if (kSingle && warp > kConsumers) {
+    // ------------------------------------------------------------ K rebuild
+    // Rebuilder rw takes tiles i = rw (mod 2); NS is even, so every stage has
+    // one rebuilder, which waits its phases in order.  The rotated dims form
+    // nch 16-byte chunks (8 pairs) per half.  When nch divides 32 (every
+    // Gemma 4 K=V shape: R = d/8) lane l keeps chunk c = l % nch and takes
+    // kpl consecutive keys from j0; the 8 pairs' angles start from one sincos
+    // each per tile and step key to key by the angle addition formulas.
+    // Other nch: any (key, chunk) per item, one sincos per pair and item.
+    const int rw = warp - kConsumers - 1;
+    const int R = rope.rotated_pairs, nch = sp.nw / 4;
+    const double* fq = reinterpret_cast<const double*>(smem + sp.freq);
+    const float2* wab = reinterpret_cast<const float2*>(smem + sp.wab);
+    const bool fixed_c = 32 % nch == 0;
+    const int c = fixed_c ? lane % nch : 0, grp = fixed_c ? 32 / nch : 1;
+    const int kpl = grp >= kKeys ? 1 : kKeys / grp, j0 = (fixed_c ? lane / nch : 0) * kpl;
+    float wa[8], wb[8], cd[8], sd[8];  // per pair of chunk c: weights, the angle of one key
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int k = 8 * c + t;
+      wa[t] = wb[t] = cd[t] = 1.f;
+      sd[t] = 0.f;
+      if (fixed_c && k < R) {
+        const float2 u = wab[k];
+        wa[t] = u.x;
+        wb[t] = u.y;
+        rope_sincos(1, fq[k], &sd[t], &cd[t]);
+      }
+    }
+    // one item: key j, chunk cc, the pairs' angles (cs, sn) at pos0 + j
+    auto item = [&](const uint8_t* sk, uint8_t* sr, int j, int cc, const float* cs,
+                    const float* sn, const float* ua, const float* ub) {
+      const int da = 8 * cc, db = D / 2 + 8 * cc;
+      const uint32_t oa = tile_off(j, da), ob = tile_off(j, db);
+      const uint4 xa = *reinterpret_cast<const uint4*>(sk + oa);
+      const uint4 xb = *reinterpret_cast<const uint4*>(sk + ob);
+      const uint32_t wa4[4] = {xa.x, xa.y, xa.z, xa.w}, wb4[4] = {xb.x, xb.y, xb.z, xb.w};
+      uint32_t ra[4], rb[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        float a[2] = {__uint_as_float(wa4[h] << 16), __uint_as_float(wa4[h] & 0xffff0000u)};
+        float bb[2] = {__uint_as_float(wb4[h] << 16), __uint_as_float(wb4[h] & 0xffff0000u)};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int t = 2 * h + e;
+          if (da + t < R) {  // unrotated pairs pass through exactly
+            const float p = a[e] * ua[t], q = bb[e] * ub[t];
+            a[e] = p * cs[t] - q * sn[t];
+            bb[e] = p * sn[t] + q * cs[t];
+          }
+        }
+        ra[h] = pack_bf16(a[0], a[1]);
+        rb[h] = pack_bf16(bb[0], bb[1]);
+      }
+      const int sa = (sp.box_slot >> (4 * (da >> 6))) & 15;
+      const int sb = (sp.box_slot >> (4 * (db >> 6))) & 15;
+      *reinterpret_cast<uint4*>(sr + sa * Ly::kBox + (oa & (Ly::kBox - 1))) =
+          make_uint4(ra[0], ra[1], ra[2], ra[3]);
+      *reinterpret_cast<uint4*>(sr + sb * Ly::kBox + (ob & (Ly::kBox - 1))) =
+          make_uint4(rb[0], rb[1], rb[2], rb[3]);
+    };
+    for (int i = rw; i < n_t; i += kRebuilders) {
+      const int s = i % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * s, (i / NS) & 1, abort))) break;
+      const long pos0 = (long)(t0 + i) * kKeys;
+      const uint8_t* sk = smem + s * kStageB;
+      uint8_t* sr = smem + s * kStageB + Ly::kTile;  // rebuilt slots
+      if (fixed_c) {
+        if (j0 < kKeys) {
+          float cs[8], sn[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            cs[t] = 1.f;
+            sn[t] = 0.f;
+            if (8 * c + t < R) rope_sincos(pos0 + j0, fq[8 * c + t], &sn[t], &cs[t]);
+          }
+          for (int m = 0; m < kpl; ++m) {
+            item(sk, sr, j0 + m, c, cs, sn, wa, wb);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {  // the angle of the next key
+              const float cn = cs[t] * cd[t] - sn[t] * sd[t];
+              sn[t] = sn[t] * cd[t] + cs[t] * sd[t];
+              cs[t] = cn;
+            }
+          }
+        }
+      } else {
+        for (int it = lane; it < kKeys * nch; it += 32) {
+          const int j = it / nch, cc = it - j * nch;
+          float cs[8], sn[8], ua[8], ub[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const int k = 8 * cc + t;
+            cs[t] = ua[t] = ub[t] = 1.f;
+            sn[t] = 0.f;
+            if (k < R) {
+              rope_sincos(pos0 + j, fq[k], &sn[t], &cs[t]);
+              ua[t] = wab[k].x;
+              ub[t] = wab[k].y;
+            }
+          }
+          item(sk, sr, j, cc, cs, sn, ua, ub);
+        }
+      }
+      // the rest of the rebuilt boxes (dims past the rotated words) is V as loaded
+      for (int it = lane; it < sp.nrb * kKeys * 8; it += 32) {
+        const int sl = it / (kKeys * 8), r = it - sl * (kKeys * 8);
+        const int j = r >> 3, bx = (sp.slot_box >> (4 * sl)) & 15;
+        const int dim = bx * 64 + (r & 7) * 8;
+        if ((dim & (D / 2 - 1)) < 8 * nch) continue;
+        const uint32_t o = tile_off(j, dim);
+        *reinterpret_cast<uint4*>(sr + sl * Ly::kBox + (o & (Ly::kBox - 1))) =
+            *reinterpret_cast<const uint4*>(sk + o);
+      }
+      mbar_arrive(bars + 8 * (2 * NS + s));
+    }
+  } else if (warp < kConsumers) {
     // ------------------------------------------------------------ consumers
     // B operand of S^T = K Q^T for every 16-dim step: q_hat[head = lane/4][dims]
     uint32_t qb[D / 16][2];
@@ -232,12 +362,14 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
     }
     for (int i = warp; i < n_t; i += kConsumers) {
       const int s = i % NS;
-      if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * s, (i / NS) & 1, abort))) break;
-      const uint32_t kb = base + s * Ly::kStage, vb = kb + Ly::kTile;
+      // two-tensor caches: the copy landed; single-tensor: K is rebuilt too
+      const uint32_t wbar = bars + 8 * ((kSingle ? 2 * NS : 0) + s);
+      if (!__all_sync(0xffffffffu, mbar_wait(wbar, (i / NS) & 1, abort))) break;
+      const uint32_t kb = base + s * kStageB, vb = kb + Ly::kTile;
       const int pos0 = (t0 + i) * kKeys;
       if (pos0 + kKeys - 1 > P) {  // last tile: zero V rows past P (never written)
         const int first = P - pos0 + 1;
-        uint8_t* vrow = smem + s * Ly::kStage + (kSingle ? 0 : Ly::kTile);
+        uint8_t* vrow = smem + s * kStageB + (kSingle ? 0 : Ly::kTile);
         for (int e = lane; e < (kKeys - first) * Ly::kBoxes * 8; e += 32) {
           const int rr = first + e / (Ly::kBoxes * 8), rest = e % (Ly::kBoxes * 8);
           *reinterpret_cast<uint4*>(vrow + (rest >> 3) * Ly::kBox + rr * 128 + (rest & 7) * 16) =
@@ -246,54 +378,24 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
         fence_proxy_async_smem();  // a later TMA refill of this stage comes after these writes
         __syncwarp();
       }
-      if constexpr (kSingle) {
-        // K of the rotated pairs of the 16 keys into the V half of the stage:
-        // (a, b) = (V[k] w_k, V[k + D/2] w_(k+D/2)) turned by pos * f_k; the
-        // unrotated dims that share a 64-dim box with rotated ones are copied
-        uint8_t* sk = smem + s * Ly::kStage;
-        uint8_t* sv = sk + Ly::kTile;
-        for (int k = lane; k < rope.rotated_pairs; k += 32) {
-          const uint8_t* e = smem + Ly::kRot + k * 24;
-          const float* x = reinterpret_cast<const float*>(e + 8);
-          const float cf = x[0], sf = x[1], wa = x[2], wb = x[3];
-          float sn, cs;
-          rope_sincos(pos0, *reinterpret_cast<const double*>(e), &sn, &cs);
-          const int da = k, db = k + D / 2;
-#pragma unroll 4
-          for (int j = 0; j < kKeys; ++j) {
-            const uint32_t oa = tile_off(j, da) + (da & 7) * 2, ob = tile_off(j, db) + (db & 7) * 2;
-            const float a = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sk + oa)) * wa;
-            const float bb = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(sk + ob)) * wb;
-            *reinterpret_cast<__nv_bfloat16*>(sv + oa) = __float2bfloat16_rn(a * cs - bb * sn);
-            *reinterpret_cast<__nv_bfloat16*>(sv + ob) = __float2bfloat16_rn(a * sn + bb * cs);
-            const float c2 = cs * cf - sn * sf;  // the angle of the next position
-            sn = sn * cf + cs * sf;
-            cs = c2;
-          }
-        }
-        for (uint32_t m = rot_boxes; m; m &= m - 1) {
-          const int bx = __ffs(m) - 1;
-          for (int e = lane; e < kKeys * 64; e += 32) {
-            const int j = e >> 6, dim = bx * 64 + (e & 63);
-            if ((dim % (D / 2)) < rope.rotated_pairs) continue;
-            const uint32_t o = tile_off(j, dim) + (dim & 7) * 2;
-            *reinterpret_cast<__nv_bfloat16*>(sv + o) = *reinterpret_cast<const __nv_bfloat16*>(sk + o);
-          }
-        }
-        __syncwarp();
-      }
       // S^T (16 keys x 8 heads)
-      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      // two accumulators over alternate 16-dim steps halve the chain of
+      // dependent MMAs (summed below)
+      float sc[4] = {0.f, 0.f, 0.f, 0.f}, sc2[4] = {0.f, 0.f, 0.f, 0.f};
       {
         const int mi = lane >> 3;
         const int key = (lane & 7) + (mi & 1) * 8;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           uint32_t a[4];
-          // single-tensor cache: the boxes with rotated dims come from the V half
-          const uint32_t src = (kSingle && ((rot_boxes >> (kk >> 2)) & 1u)) ? vb : kb;
+          // single-tensor cache: the boxes with rotated dims come from their slot
+          uint32_t src = kb;
+          if constexpr (kSingle) {
+            const uint32_t sl = (sp.box_slot >> (4 * (kk >> 2))) & 15u;
+            if (sl != 15u) src = vb + sl * Ly::kBox - (kk >> 2) * Ly::kBox;
+          }
           ldsm_x4(src + tile_off(key, kk * 16 + (mi >> 1) * 8), a);
-          mma16816(sc, a, qb[kk][0], qb[kk][1]);
+          mma16816((kk & 1) ? sc2 : sc, a, qb[kk][0], qb[kk][1]);
         }
       }
       // masked scores in log2 units: rows = keys pos0 + lane/4 (+8), cols = heads;
@@ -305,7 +407,7 @@ __global__ void __launch_bounds__(kThreadsDm, 1)
       const bool vA = kA >= lo && kA <= P && kept(kA), vB = kB >= lo && kB <= P && kept(kB);
       float r[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) r[e] = sc[e] * scale_log2;
+      for (int e = 0; e < 4; ++e) r[e] = (sc[e] + sc2[e]) * scale_log2;
       if (cap2 > 0.f) {  // soft-cap in log2 units
 #pragma unroll
         for (int e = 0; e < 4; ++e) r[e] = cap2 * tanh_fast(r[e] * (1.f / cap2));
@@ -435,20 +537,42 @@ static cudaError_t run_mma(const LayerCfg& L, int B, const void* q_raw, const vo
   if (!make_bf16_map(&tk, cache_k, 3, dims, str, box)) return cudaErrorInvalidValue;
   if (!make_bf16_map(&tv, single ? cache_k : cache_v, 3, dims, str, box))
     return cudaErrorInvalidValue;
-  // the 64-dim boxes that hold rotated dims (pairs k < R: dims k and k + D/2)
-  uint32_t rot_boxes = 0;
-  for (int k = 0; k < L.rope.rotated_pairs; ++k)
-    rot_boxes |= (1u << (k / 64)) | (1u << ((k + D / 2) / 64));
+  DmSingle sp{};
+  uint32_t smem_bytes = Ly::kAlloc;
+  if (single) {
+    // the 64-dim boxes that hold rotated dims (pairs k < R: dims k and k + D/2)
+    const int R = L.rope.rotated_pairs;
+    uint32_t rot = 0;
+    for (int k = 0; k < R; ++k) rot |= (1u << (k / 64)) | (1u << ((k + D / 2) / 64));
+    sp.box_slot = 0xffffffffu;
+    for (int bx = 0; bx < Ly::kBoxes; ++bx)
+      if ((rot >> bx) & 1u) {
+        sp.box_slot = (sp.box_slot & ~(15u << (4 * bx))) | ((uint32_t)sp.nrb << (4 * bx));
+        sp.slot_box |= (uint32_t)bx << (4 * sp.nrb);
+        ++sp.nrb;
+      }
+    sp.nw = (R + 7) / 8 * 4;  // whole 16-byte chunks of each half
+    sp.stage = Ly::kTile + sp.nrb * Ly::kBox;
+    const uint32_t fixed = 8 * D * 2 + 3 * 16 * 8 + 16 * (uint32_t)R + 64;
+    const uint32_t budget = 227 * 1024 - 1024 - fixed;  // 1 KB: static shared memory
+    sp.ns = (int)std::min<uint32_t>(16, budget / sp.stage) & ~3;
+    if (sp.ns < 4 || (uint32_t)sp.ns * sp.stage < Ly::kMerge) return cudaErrorInvalidValue;
+    sp.q = sp.ns * sp.stage;
+    sp.bars = sp.q + 8 * D * 2;
+    sp.freq = (sp.bars + 3 * sp.ns * 8 + 15) & ~15u;
+    sp.wab = sp.freq + 8 * R;
+    smem_bytes = sp.wab + 8 * R + 64;
+  }
   auto kern = single ? decode_mma_kernel<D, true> : decode_mma_kernel<D, false>;
   cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Ly::kAlloc);
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
   if (e != cudaSuccess) return e;
   dim3 grid(plan.n_chunks, L.Hkv, B);
-  kern<<<grid, kThreadsDm, Ly::kAlloc, s>>>(
+  kern<<<grid, kThreadsDm + (single ? kRebuilders * 32 : 0), smem_bytes, s>>>(
       tk, tv, static_cast<const __nv_bfloat16*>(q_raw), static_cast<const __nv_bfloat16*>(wq), len,
       cap, rolling, L.Hq, L.Hkv, L.layer_type, L.window, L.scale * 1.4426950408889634f,
       softcap_log2(L), km, L.eps, plan.chunk, plan.n_chunks, part_ml, part_o, status,
-      static_cast<const __nv_bfloat16*>(wk_single), rot_boxes, L.rope);
+      static_cast<const __nv_bfloat16*>(wk_single), sp, L.rope);
   count_launch();
   return cudaGetLastError();
 }

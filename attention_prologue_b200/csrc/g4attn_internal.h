@@ -135,6 +135,14 @@ cudaError_t launch_decode(const LayerCfg& L, int B, const void* q_raw, const voi
 // Tensor-core split kernel of g4attn_decode (bf16, <= 8 query heads per KV
 // head, rolling caches with capacity % 16 == 0); writes the same partials
 // as the CUDA-core split kernel.
+// QKV projection x W^T with the prologue in the epilogue (bf16): q_hat
+// [B, T, Hq, d]; K/V of the Hkv key (and value) heads into kv; len[b] =
+// p0 + T when len is given.  W holds n_heads * d rows.
+cudaError_t launch_qkv_prologue(const LayerCfg& L, int B, int T, int p0, const void* x,
+                                int hidden, const void* w_qkv, int n_heads, const void* wq,
+                                const void* wk, void* q_hat, KVDst kv, int32_t* len, int* status,
+                                cudaStream_t s);
+
 bool decode_mma_supported(const LayerCfg& L, int cap, int rolling);
 cudaError_t launch_decode_mma(const LayerCfg& L, int B, const void* q_raw, const void* wq,
                               const void* cache_k, const void* cache_v, const void* wk_single,

@@ -374,7 +374,8 @@ cudaError_t launch_block_intervals(const LayerCfg& L, int B, int T, const int32_
 }
 
 // lo/hi of every row of a chunk at positions p0 .. p0+T-1 of a prompt of
-// p0 + T tokens (cached prefill): a global row sees [0, pos]; a sliding row
+// p0 + T tokens (cached prefill): a global row sees [0, pos], a bidirectional
+// one [0, p0 + T - 1]; a sliding row
 // its window [max(0, pos-w+1), pos] united with the maximal run of equal
 // non-negative ids (ids [B][p0 + T], or nullptr) that contains pos, seen up
 // to the chunk's last position.
@@ -388,7 +389,9 @@ __global__ void chunk_interval_kernel(const int32_t* __restrict__ ids, int B, in
   const int Tk = p0 + T_;
   const int pos = p0 + i;
   int a = 0, e = pos;
-  if (layer_type != 1) {
+  if (layer_type == 2) {  // bidirectional: every position of the sequence
+    e = Tk - 1;
+  } else if (layer_type != 1) {
     a = pos - window + 1;
     if (a < 0) a = 0;
     if (ids) {

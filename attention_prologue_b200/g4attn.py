@@ -17,11 +17,12 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libg4attn.
 
 G4ATTN_OK, G4ATTN_EINVAL, G4ATTN_EUNSUPPORTED, G4ATTN_ECACHE_OVERFLOW = 0, 1, 2, 3
 G4ATTN_ECUDA, G4ATTN_EDEVICE, G4ATTN_EWORKSPACE, G4ATTN_ECACHE_EMPTY = 4, 5, 6, 7
-G4ATTN_SLIDING, G4ATTN_GLOBAL = 0, 1
+G4ATTN_SLIDING, G4ATTN_GLOBAL, G4ATTN_BIDIRECTIONAL = 0, 1, 2
 G4ATTN_BF16, G4ATTN_FP32 = 0, 1
 
 EXPORTED = ("g4attn_prefill_workspace_size", "g4attn_decode_workspace_size", "g4attn_prefill",
             "g4attn_prefill_chunk_workspace_size", "g4attn_prefill_chunk",
+            "g4attn_qkv_prologue", "g4attn_attend_workspace_size", "g4attn_attend",
             "g4attn_cache_append", "g4attn_decode", "g4attn_decode_noalloc",
             "g4attn_get_device_status", "g4attn_time_next_attention", "g4attn_launch_count",
             "g4attn_status_string")
@@ -74,6 +75,11 @@ def lib() -> ctypes.CDLL:
         L.g4attn_prefill_chunk_workspace_size.restype = S
         L.g4attn_prefill_chunk.argtypes = [DP, I, I, I, P, P, P, P, P, P, P, CP, P, P, S, P]
         L.g4attn_prefill_chunk.restype = I
+        L.g4attn_qkv_prologue.argtypes = [DP, I, I, I, P, I, P, P, P, P, CP, P]
+        L.g4attn_qkv_prologue.restype = I
+        L.g4attn_attend_workspace_size.argtypes = [DP, I, I, I]
+        L.g4attn_attend_workspace_size.restype = ctypes.c_size_t
+        L.g4attn_attend.argtypes = [DP, I, I, I, P, P, P, CP, P, P, S, P]
         L.g4attn_cache_append.argtypes = [DP, CP, P, P, P, P]
         L.g4attn_cache_append.restype = I
         L.g4attn_decode.argtypes = [DP, CP, P, P, P, P, S, P]
@@ -268,6 +274,57 @@ def g4attn_prefill_chunk(desc: LayerDesc, p0: int, q_raw: torch.Tensor,
         _ptr(am, "attention_mask", dev), ctypes.byref(cc), _ptr(out, "out", dev), _ptr(workspace, "workspace", dev),
         workspace.numel(), _stream(stream))
     _check(rc, "g4attn_prefill_chunk")
+    return out
+
+
+def g4attn_qkv_prologue(desc: LayerDesc, p0: int, x: torch.Tensor, w_qkv: torch.Tensor,
+                        q_norm_w: torch.Tensor, k_norm_w: torch.Tensor | None,
+                        cache: KVCache | None, q_hat: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """QKV projection of x [B, T, hidden] by w_qkv [n_heads * d, hidden] with
+    the prologue in its epilogue (see g4attn_qkv_prologue in g4attn.h):
+    returns q_hat [B, T, Hq, d]; K/V go to `cache` at positions p0 .. p0+T-1."""
+    B, T, hidden = x.shape
+    dev = x.device
+    if q_hat is None:
+        q_hat = torch.empty(B, T, desc.num_heads, desc.head_dim, dtype=x.dtype, device=dev)
+    cc = cache.c() if cache is not None else None
+    rc = lib().g4attn_qkv_prologue(
+        ctypes.byref(desc), B, T, p0, _ptr(x, "x", dev), hidden, _ptr(w_qkv, "w_qkv", dev),
+        _ptr(q_norm_w, "q_norm_w", dev), _ptr(k_norm_w, "k_norm_w", dev),
+        _ptr(q_hat, "q_hat", dev), ctypes.byref(cc) if cc is not None else None,
+        _stream(stream))
+    _check(rc, "g4attn_qkv_prologue")
+    return q_hat
+
+
+def g4attn_attend_workspace_size(desc: LayerDesc, B: int, T: int, p0: int) -> int:
+    return int(lib().g4attn_attend_workspace_size(ctypes.byref(desc), B, T, p0))
+
+
+def g4attn_attend(desc: LayerDesc, p0: int, q_hat: torch.Tensor, cache: KVCache,
+                  image_block_ids: torch.Tensor | None = None,
+                  attention_mask: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Attention of post-prologue queries q_hat [B, T, Hq, d] at positions
+    p0 .. p0+T-1 over the cache's positions 0 .. p0+T-1 (see g4attn_attend in
+    g4attn.h); image_block_ids and attention_mask [B, p0 + T]."""
+    B, T = q_hat.shape[0], q_hat.shape[1]
+    dev = q_hat.device
+    if out is None:
+        out = torch.empty_like(q_hat)
+    if workspace is None:
+        workspace = _workspace(g4attn_attend_workspace_size(desc, B, T, p0), dev)
+    if image_block_ids is not None and image_block_ids.dtype != torch.int32:
+        raise ValueError("image_block_ids must be int32")
+    am = _mask(attention_mask, (B, p0 + T), "attention_mask")
+    cc = cache.c()
+    rc = lib().g4attn_attend(
+        ctypes.byref(desc), B, T, p0, _ptr(q_hat, "q_hat", dev),
+        _ptr(image_block_ids, "image_block_ids", dev), _ptr(am, "attention_mask", dev),
+        ctypes.byref(cc), _ptr(out, "out", dev), _ptr(workspace, "workspace", dev),
+        workspace.numel(), _stream(stream))
+    _check(rc, "g4attn_attend")
     return out
 
 

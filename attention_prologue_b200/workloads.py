@@ -23,7 +23,7 @@ from dataclasses import dataclass, field, replace
 import numpy as np
 import torch
 
-SLIDING, GLOBAL = 0, 1
+SLIDING, GLOBAL, BIDIRECTIONAL = 0, 1, 2
 
 
 @dataclass(frozen=True)
@@ -68,6 +68,16 @@ def global_(num_heads, num_kv_heads, head_dim, k_eq_v=True, **kw) -> LayerShape:
                       rope_theta=1e6, k_eq_v=k_eq_v, **kw)
 
 
+def bidirectional(num_heads, num_kv_heads, head_dim, **kw) -> LayerShape:
+    """The vision tower's attention: every patch sees every patch of its image
+    ("gemma4-pt-claude" README, "Key architectural features"), softmax scale
+    1.0 ("Attention Backend Notes")."""
+    kw.setdefault("softmax_scale", 1.0)
+    kw.setdefault("rotary_fraction", 1.0)
+    kw.setdefault("rope_theta", 1e4)
+    return LayerShape(BIDIRECTIONAL, num_heads, num_kv_heads, head_dim, **kw)
+
+
 # -- the five workloads ------------------------------------------------------
 
 # tiny fp32 check: one sliding layer and one K=V global layer
@@ -82,6 +92,12 @@ G12B_SLIDING_MM = PrefillWorkload("12b-sliding-multimodal-prefill", sliding(16, 
                                   2, 16384, n_blocks=4, block_len=280)
 # 31B-shaped K=V global layer: 32 query heads on 4 KV heads, d 512
 G31B_GLOBAL = PrefillWorkload("31b-global-prefill", global_(32, 4, 512), 1, 32768)
+
+# Vision-tower-shaped bidirectional attention: images of up to 2520 patches
+# (the image processor's 280 soft tokens times its 3x3 pooling, Keras docs
+# "Gemma4ImageProcessor"), 16 heads of 64 dims (the pages give no tower
+# dimensions: a reading), scale 1.0
+VISION_BIDIR = PrefillWorkload("vision-bidirectional", bidirectional(16, 16, 64), 8, 2520)
 
 PREFILL_WORKLOADS = {w.name: w for w in
                      (TINY_SLIDING, TINY_GLOBAL, E2B_SLIDING, G12B_SLIDING_MM, G31B_GLOBAL)}
@@ -181,6 +197,47 @@ def prefill_inputs(w: PrefillWorkload, device="cpu", seed: int = 0) -> dict:
     if ids is not None:
         ids = ids.to(device)
     return dict(q_raw=q, k_raw=k, v_raw=v, q_norm_w=wq, k_norm_w=wk, image_block_ids=ids)
+
+
+# hidden size of the layer's input per variant ("gemma4-pt-claude" README,
+# "Supported Models": E2B 1536, 12B 3840, 31B 5376)
+HIDDEN = {"e2b-sliding-prefill": 1536, "12b-sliding-multimodal-prefill": 3840,
+          "31b-global-prefill": 5376}
+
+
+def projection_inputs(L: LayerShape, B: int, T: int, hidden: int, device="cpu", seed: int = 0,
+                      with_kv: bool = True) -> dict:
+    """Input of the QKV projection: x [B, T, hidden] ~ N(0, 1) and w_qkv
+    [n_heads * d, hidden] ~ N(0, 1/hidden) (raw projections of unit
+    variance; rows: the query heads, then the key heads, then the value heads
+    unless K=V), and the norm weights; drawn in that order."""
+    g = _gen(device, seed)
+    n_heads = L.num_heads + ((L.num_kv_heads if L.k_eq_v else 2 * L.num_kv_heads)
+                             if with_kv else 0)
+    x = randn((B, T, hidden), g, device, torch.bfloat16)
+    w = (randn((n_heads * L.head_dim, hidden), g, device, torch.float32) *
+         hidden ** -0.5).to(torch.bfloat16)
+    wq = norm_weight(L.head_dim, g, device, torch.bfloat16, "one_plus")
+    wk = norm_weight(L.head_dim, g, device, torch.bfloat16, "one_plus") if with_kv else None
+    return dict(x=x, w_qkv=w, q_norm_w=wq, k_norm_w=wk)
+
+
+def vision_inputs(w: PrefillWorkload, device="cpu", seed: int = 0) -> dict:
+    """Post-prologue inputs of a bidirectional layer (the tower applies its
+    own 2-D rotary before attention): q_hat [B, T, Hq, d], k_hat and v_hat
+    [B, Hkv, T, d], all N(0, 1) (unit RMS, like RMS-normalised vectors), and a
+    padding mask [B, T] (uint8): image b has n_b valid patches, n_b uniform
+    in [T/4, T] (numpy PCG64 with the seed), the rest is padding."""
+    L = w.layer
+    g = _gen(device, seed)
+    q = randn((w.B, w.T, L.num_heads, L.head_dim), g, device, w.dtype)
+    k = randn((w.B, L.num_kv_heads, w.T, L.head_dim), g, device, w.dtype)
+    v = randn((w.B, L.num_kv_heads, w.T, L.head_dim), g, device, w.dtype)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    n = rng.integers(w.T // 4, w.T, size=w.B, endpoint=True)
+    keep = (np.arange(w.T)[None, :] < n[:, None]).astype(np.uint8)
+    return dict(q_hat=q, k_hat=k, v_hat=v, attention_mask=torch.from_numpy(keep).to(device),
+                valid=n.astype(np.int64))
 
 
 def decode_lengths(w: DecodeWorkload, seed: int = 0) -> np.ndarray:

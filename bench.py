@@ -589,6 +589,198 @@ def bench_decode(args, dist: Dist, pk: dict, clk: ClockSampler):
     return res
 
 
+# ---------------------------------------------------------------------------
+# the QKV projection with the prologue in its epilogue, and the vision shape
+
+def timed(fn, K, flush, stream, ev=None):
+    """Device ms of K calls of fn (L2 flushed before each), from events on
+    `stream`; ev: events the library records around its dominant kernel."""
+    s0, s1 = made_events(K), made_events(K)
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        s0[i].record(stream)
+        if ev is not None:
+            G.g4attn_time_next_attention(ev[0][i], ev[1][i])
+        fn()
+        s1[i].record(stream)
+    torch.cuda.synchronize()
+    return [s0[i].elapsed_time(s1[i]) for i in range(K)]
+
+
+def bench_qkv(args, dist: Dist, pk: dict, clk: ClockSampler, steps: int):
+    """g4attn_qkv_prologue on the E2B-shaped layer's prompt (x [1, 8192, 1536]
+    -> 8 query heads, K and V of 256: the raw projections stay in TMEM), and
+    the same projection by cuBLAS (torch.matmul to bf16 raw, no prologue)
+    timed beside it.  Unit: the projection's FLOPs, 2 * tokens * rows of W *
+    hidden."""
+    w = W.E2B_SLIDING
+    L, hidden = w.layer, W.HIDDEN[w.name]
+    dev = torch.device("cuda", dist.local)
+    inp = W.projection_inputs(L, w.B, w.T, hidden, dev, seed=dist.rank)
+    d = desc_of(L)
+    cache = G.KVCache.allocate(w.B, L.num_kv_heads, w.T, L.head_dim, device=dev)
+    q_hat = torch.empty(w.B, w.T, L.num_heads, L.head_dim, dtype=torch.bfloat16, device=dev)
+    n_rows = inp["w_qkv"].shape[0]
+    flops = 2.0 * w.B * w.T * n_rows * hidden
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    raw = torch.empty(w.B * w.T, n_rows, dtype=torch.bfloat16, device=dev)
+    x2 = inp["x"].view(w.B * w.T, hidden)
+
+    def fused():
+        G.g4attn_qkv_prologue(d, 0, inp["x"], inp["w_qkv"], inp["q_norm_w"], inp["k_norm_w"],
+                              cache, q_hat=q_hat, stream=stream)
+
+    def cublas():
+        torch.matmul(x2, inp["w_qkv"].t(), out=raw)
+
+    for _ in range(args.warmup):
+        fused()
+        cublas()
+    dist.barrier()
+    clk.resume()
+    n0 = G.g4attn_launch_count()
+    f_ms = timed(fused, steps, flush, stream)
+    launches = G.g4attn_launch_count() - n0
+    c_ms = timed(cublas, steps, flush, stream)
+    clk.pause()
+    dist.barrier()
+    status = G.g4attn_get_device_status()
+    if status != G.G4ATTN_OK:
+        raise RuntimeError(f"device status after qkv: {G.g4attn_status_string(status)}")
+    total = dist.max(sum(f_ms))
+    avg = statistics.mean(f_ms)
+    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    achieved = flops / (avg * 1e-3) / 1e12
+    res = {"metric": "QKV projection + prologue TFLOP/s", "unit": "TFLOP/s",
+           "value": job_rate(dist.world, flops, steps, total) / 1e12,
+           "ms_per_step": total / steps, "steps": steps, "flops": flops, "launches": launches,
+           "workload": f"{w.name}: x [{w.B}, {w.T}, {hidden}] -> {n_rows} rows of W",
+           "roofline": {"bound": "tensor", "kernel": "qkv_prologue_kernel<256>",
+                        "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                        "frac": achieved / peak,
+                        "traffic": profile_field("qkv_prologue_e2b.md", "traffic_bytes_per_launch"),
+                        "algorithmic_per_launch": flops, "avg_launch_ms": avg},
+           "cublas_projection_only": {"ms": statistics.mean(c_ms),
+                                      "tflops": flops / (statistics.mean(c_ms) * 1e-3) / 1e12,
+                                      "note": "torch.matmul to bf16 raw q/k/v, no prologue"},
+           "cpu_baseline": None}
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = qkv_cpu_baseline(w, inp, hidden)
+    del raw, flush, cache, q_hat
+    return res
+
+
+def qkv_cpu_baseline(w, inp, hidden, target_s=5.0):
+    """The oracle's projection (float64 matmul) and prologue on the first
+    tokens of the prompt, sized to about target_s."""
+    import oracle
+    oracle.build()
+    ol = oracle_layer_of(w.layer)
+    cpu = {k: v.cpu() for k, v in inp.items() if v is not None}
+    n_rows = cpu["w_qkv"].shape[0]
+    n = 256
+    while True:
+        t0 = time.perf_counter()
+        oracle.qkv_prologue(ol, cpu["x"][:, :n], cpu["w_qkv"], cpu["q_norm_w"], cpu["k_norm_w"])
+        secs = time.perf_counter() - t0
+        if secs > target_s / 4 or n >= w.T:
+            break
+        n = min(w.T, n * 4)
+    flops = 2.0 * n * n_rows * hidden
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": oracle.default_threads(),
+            "kind": "oracle",
+            "sample": f"the first {n} tokens of the prompt: float64 numpy matmul (x W^T) and the "
+                      f"C prologue, {secs:.1f} s"}
+
+
+def bench_vision(args, dist: Dist, pk: dict, clk: ClockSampler, steps: int):
+    """The vision-tower attention shape through g4attn_attend (bidirectional,
+    scale 1.0, 8 images of up to 2520 patches with per-image padding, 16
+    heads of 64): unmasked TFLOP/s = 4 d Hq T sum_b n_b (every row sees the
+    n_b valid patches of its image)."""
+    w = W.VISION_BIDIR
+    L = w.layer
+    dev = torch.device("cuda", dist.local)
+    inp = W.vision_inputs(w, dev, seed=dist.rank)
+    d = desc_of(L)
+    cache = G.KVCache.allocate(w.B, L.num_kv_heads, w.T, L.head_dim, device=dev)
+    cache.k.copy_(inp["k_hat"])
+    cache.v.copy_(inp["v_hat"])
+    out = torch.empty_like(inp["q_hat"])
+    ws = torch.empty(G.g4attn_attend_workspace_size(d, w.B, w.T, 0), dtype=torch.uint8,
+                     device=dev)
+    flops = 4.0 * L.head_dim * L.num_heads * w.T * float(inp["valid"].sum())
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        G.g4attn_attend(d, 0, inp["q_hat"], cache, attention_mask=inp["attention_mask"],
+                        out=out, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    a0, a1 = made_events(steps), made_events(steps)
+    dist.barrier()
+    clk.resume()
+    n0 = G.g4attn_launch_count()
+    s_ms = timed(step, steps, flush, stream, ev=(a0, a1))
+    launches = G.g4attn_launch_count() - n0
+    clk.pause()
+    dist.barrier()
+    status = G.g4attn_get_device_status()
+    if status != G.G4ATTN_OK:
+        raise RuntimeError(f"device status after vision: {G.g4attn_status_string(status)}")
+    total = dist.max(sum(s_ms))
+    attn = statistics.mean(a0[i].elapsed_time(a1[i]) for i in range(steps))
+    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    achieved = flops / (attn * 1e-3) / 1e12
+    res = {"metric": "prefill attn TFLOP/s (unmasked)", "unit": "TFLOP/s",
+           "value": job_rate(dist.world, flops, steps, total) / 1e12,
+           "ms_per_step": total / steps, "steps": steps, "flops": flops, "launches": launches,
+           "workload": w.name,
+           "config": {"images": w.B, "patch_budget": w.T, "heads": [L.num_heads, L.num_kv_heads],
+                      "head_dim": L.head_dim, "softmax_scale": L.scale,
+                      "valid_patches": [int(n) for n in inp["valid"]],
+                      "step": "one g4attn_attend call (eager)"},
+           "roofline": {"bound": "tensor", "kernel": "attn_sm100_kernel<64> (g4attn_attend)",
+                        "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                        "frac": achieved / peak,
+                        "traffic": profile_field("attn_sm100_vision.md", "traffic_bytes_per_launch"),
+                        "algorithmic_per_launch": flops, "avg_launch_ms": attn},
+           "cpu_baseline": None}
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = vision_cpu_baseline(w, inp)
+    del cache, out, ws, flush
+    return res
+
+
+def vision_cpu_baseline(w, inp, target_s=5.0):
+    """The oracle's attention of every `stride`-th patch row of every image."""
+    import oracle
+    oracle.build()
+    threads = oracle.default_threads()
+    ol = oracle_layer_of(w.layer)
+    qh = inp["q_hat"].double().cpu().numpy()
+    kh = inp["k_hat"].double().cpu().numpy().transpose(0, 2, 1, 3)
+    vh = inp["v_hat"].double().cpu().numpy().transpose(0, 2, 1, 3)
+    keep = inp["attention_mask"].cpu().numpy()
+    stride = 256
+    while True:
+        rows = list(range(0, w.T, stride))
+        t0 = time.perf_counter()
+        oracle.attend_rows(ol, qh, kh, vh, 0, None, rows, threads, attention_mask=keep)
+        secs = time.perf_counter() - t0
+        if secs > target_s / 4 or stride == 1:
+            break
+        stride = max(1, stride // 4)
+    flops = 4.0 * w.layer.head_dim * w.layer.num_heads * len(rows) * float(inp["valid"].sum())
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{w.name}: {rows_phrase(stride)} of every image, all heads, {secs:.1f} s; "
+                      f"float64 C, {threads} threads"}
+
+
 def decode_cpu_baseline(w, lens, s_state, g_state, x_state, n_global_seqs=4):
     """The float64 oracle's decode of the same step on the host cores: the
     sliding layer for every sequence, the global and KV-shared layers for a
@@ -784,6 +976,10 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-kv-single", action="store_true",
                     help="skip the decode step over a single-tensor K=V cache")
+    ap.add_argument("--no-qkv", action="store_true",
+                    help="skip the fused QKV projection + prologue leg")
+    ap.add_argument("--no-vision", action="store_true",
+                    help="skip the vision-tower (bidirectional) attention leg")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls, not a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
@@ -848,6 +1044,15 @@ def main(argv=None):
             dargs = argparse.Namespace(**{**vars(args), "steps": extra_steps})
             dec = bench_decode(dargs, dist, pk, clk)
             dec["roofline"]["peak_source"] = f"{pk_src}: hbm_gbs"
+        qkv = vis = None
+        if not args.no_qkv and not args.seq_len:
+            torch.cuda.empty_cache()
+            qkv = bench_qkv(args, dist, pk, clk, extra_steps)
+            qkv["roofline"]["peak_source"] = f"{pk_src}: bf16_tflops (burst)"
+        if not args.no_vision and not args.seq_len:
+            torch.cuda.empty_cache()
+            vis = bench_vision(args, dist, pk, clk, extra_steps)
+            vis["roofline"]["peak_source"] = f"{pk_src}: bf16_tflops (burst)"
     roof = dict(pre["roofline"])
     roof["peak_source"] = f"{pk_src}: bf16_tflops (burst)"
     clocks = head_clocks or {}
@@ -866,7 +1071,8 @@ def main(argv=None):
                                else "one g4attn_prefill call (eager)",
                        "unmasked_gflop_per_step": pre["flops"] / 1e9},
             "roofline": roof, "cpu_baseline": cpu, "e2e": pre["e2e"],
-            "gpu_launches": pre["launches"], "clocks": clocks, "prefill": legs, "decode": dec}
+            "gpu_launches": pre["launches"], "clocks": clocks, "prefill": legs, "decode": dec,
+            "qkv_prologue": qkv, "vision": vis}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
     dist.close()

@@ -45,6 +45,11 @@
  *       logit soft-cap (attn_logits_soft_cap) exists as a layer option; the
  *       page prints no formula, the reading is the tanh cap the Keras docs'
  *       argument table names for the final logits.
+ *  [P4] "gemma4-pt-claude" README, "Key architectural features": the vision
+ *       encoder is ViT-style with bidirectional attention; "Attention
+ *       Backend Notes": the vision tower runs its attention at scale 1.0.
+ *  [V4] "Gemma 4" overview blog, "Shared KV Cache": the key and value
+ *       projections produce the K/V a layer stores (and later layers reuse).
  *
  * Definitions used throughout (readings of the pages, stated once):
  *  - RMSNorm over the d values of one head: x / sqrt(mean(x^2) + eps) * w,
@@ -62,7 +67,8 @@
  *    query inside an image block [s, e) sees the union of its window and the
  *    whole block, [min(max(0, i - window + 1), s), e - 1]  [K1][V1].
  *    An image block is a maximal run of equal non-negative ids in
- *    image_block_ids; -1 marks text.
+ *    image_block_ids; -1 marks text.  A bidirectional (vision-tower) layer:
+ *    every position of the sequence, [0, T - 1]  [P4].
  *  - o_i = sum_j softmax_j(s_ij) v_j over those keys, with the score
  *    s_ij = softmax_scale * q_i . k_j, or c * tanh(softmax_scale * q_i . k_j / c)
  *    with a logit soft-cap c > 0 [P3].  A padding key (mask entry 0) is never
@@ -90,7 +96,9 @@ typedef enum {
   G4ATTN_ECACHE_EMPTY = 7     /* decode on a sequence whose cache holds nothing */
 } g4attn_status;
 
-enum { G4ATTN_SLIDING = 0, G4ATTN_GLOBAL = 1 };
+/* G4ATTN_BIDIRECTIONAL: the vision tower's attention shape [P4]; prefill
+ * (and g4attn_attend) only: append and decode return G4ATTN_EUNSUPPORTED. */
+enum { G4ATTN_SLIDING = 0, G4ATTN_GLOBAL = 1, G4ATTN_BIDIRECTIONAL = 2 };
 enum { G4ATTN_BF16 = 0, G4ATTN_FP32 = 1 };
 
 /* One attention layer [K2].  Sliding layers: window > 0, typically
@@ -102,7 +110,8 @@ enum { G4ATTN_BF16 = 0, G4ATTN_FP32 = 1 };
  * the usual value).  dtype is the element type of every raw input, weight,
  * output and cache tensor of the call. */
 typedef struct {
-  int layer_type;        /* G4ATTN_SLIDING or G4ATTN_GLOBAL */
+  int layer_type;        /* G4ATTN_SLIDING, G4ATTN_GLOBAL or
+                            G4ATTN_BIDIRECTIONAL */
   int window;            /* keys per sliding query, itself included */
   float rotary_fraction; /* fraction of each head that is rotated */
   double rope_theta;     /* RoPE base */
@@ -181,7 +190,8 @@ size_t g4attn_decode_workspace_size(const g4attn_layer_desc *desc,
  *  k_norm_w        device [d]: QK-norm weight of the keys (ignored if k_raw
  *                  is NULL).
  *  image_block_ids device int32 [B, T] or NULL: -1 text, a block is a maximal
- *                  run of one non-negative id.  Ignored on global layers.
+ *                  run of one non-negative id.  Ignored on global and
+ *                  bidirectional layers.
  *  attention_mask  device uint8 [B, T] or NULL [K4]: a key at a position
  *                  whose entry is 0 is padding and never attended (RoPE
  *                  positions stay the token indices); a row left without any
@@ -248,13 +258,70 @@ int g4attn_prefill_chunk(const g4attn_layer_desc *desc, int B, int T, int p0,
                          void *out, void *workspace, size_t ws_bytes,
                          void *stream);
 
+/* The QKV projection with the prologue in its epilogue [V4][K1]: for every
+ * token row of x, raw = x W^T on the tensor cores, then per output head
+ * RMSNorm (* w_q / w_k) and RoPE at the token's position p0 + t for query and
+ * key heads, weightless RMSNorm for value heads (and, with k_eq_v, for the
+ * key heads' V); the raw projections are never written.  bf16 only.
+ *
+ *  x         device bf16 [B, T, hidden], hidden a multiple of 8, 16-byte
+ *            aligned.
+ *  w_qkv     device bf16 [n_heads * d, hidden], 16-byte aligned: the rows of
+ *            the num_heads query heads, then (with a cache) the num_kv_heads
+ *            key heads, then (without k_eq_v) the num_kv_heads value heads.
+ *  q_norm_w, k_norm_w  device [d]; k_norm_w is needed with a cache.
+ *  q_hat     device bf16 [B, T, num_heads, d], 16-byte aligned: the
+ *            post-prologue queries (the input of g4attn_attend).
+ *  cache     NULL: a KV-shared layer [V3] that projects its queries only.
+ *            Otherwise K/V of positions p0 .. p0+T-1 go to their slots (a
+ *            rolling cache keeps the last `capacity` of them; a single-tensor
+ *            cache V alone) and len[b] becomes p0 + T.
+ *
+ * Errors: G4ATTN_EINVAL for NULLs, hidden < 8 or not a multiple of 8,
+ * misaligned pointers, a cache shape mismatch; G4ATTN_EUNSUPPORTED for fp32;
+ * G4ATTN_ECACHE_OVERFLOW for a non-rolling cache with capacity < p0 + T;
+ * G4ATTN_ECUDA. */
+int g4attn_qkv_prologue(const g4attn_layer_desc *desc, int B, int T, int p0,
+                        const void *x, int hidden, const void *w_qkv,
+                        const void *q_norm_w, const void *k_norm_w, void *q_hat,
+                        g4attn_cache *cache, void *stream);
+
+/* Bytes of device workspace g4attn_attend needs.  Returns 0 if the
+ * arguments are invalid. */
+size_t g4attn_attend_workspace_size(const g4attn_layer_desc *desc, int B, int T,
+                                    int p0);
+
+/* The attention of a prefill from post-prologue inputs [K1][V1][P4]: the
+ * queries q_hat (RMSNorm * w_q and RoPE already applied, e.g. by
+ * g4attn_qkv_prologue or by a vision tower's own 2-D rotary) of T tokens at
+ * positions p0 .. p0+T-1 attend over the keys/values `cache` holds at
+ * positions 0 .. p0+T-1 (slots 0 .. p0+T-1), with the intervals of
+ * g4attn_prefill_chunk.  Nothing is written to the cache and len[] is not
+ * read or changed.
+ *
+ *  q_hat           device [B, T, num_heads, d] in dtype.
+ *  image_block_ids device int32 [B, p0 + T] or NULL (sliding layers only).
+ *  attention_mask  device uint8 [B, p0 + T] or NULL, as g4attn_prefill_chunk.
+ *  cache           a two-tensor cache (k and v), capacity >= p0 + T.
+ *  out             device [B, T, num_heads, d].
+ *  workspace       g4attn_attend_workspace_size bytes, 256-byte aligned.
+ *
+ * Errors: G4ATTN_EINVAL for NULLs, shape or dtype mismatch, capacity <
+ * p0 + T; G4ATTN_EUNSUPPORTED for a single-tensor cache; G4ATTN_EWORKSPACE;
+ * G4ATTN_ECUDA. */
+int g4attn_attend(const g4attn_layer_desc *desc, int B, int T, int p0,
+                  const void *q_hat, const int32_t *image_block_ids,
+                  const uint8_t *attention_mask, const g4attn_cache *cache,
+                  void *out, void *workspace, size_t ws_bytes, void *stream);
+
 /* Append one token per sequence to a layer's cache [P2][K3]: the key/value
  * prologue of k_raw/v_raw (device [B, 1, num_kv_heads, d]; v_raw NULL with
  * k_eq_v) at position p = len[b], written at slot p (rolling: p % capacity),
  * then len[b] = p + 1.  k_norm_w is device [d].
  * If p >= capacity on a non-rolling cache nothing is written for that
  * sequence, len[b] is unchanged and the device status word records
- * G4ATTN_ECACHE_OVERFLOW (read it with g4attn_get_device_status). */
+ * G4ATTN_ECACHE_OVERFLOW (read it with g4attn_get_device_status).
+ * A bidirectional layer has no cache append: G4ATTN_EUNSUPPORTED. */
 int g4attn_cache_append(const g4attn_layer_desc *desc, g4attn_cache *cache,
                         const void *k_raw, const void *v_raw,
                         const void *k_norm_w, void *stream);
@@ -274,7 +341,8 @@ int g4attn_cache_append(const g4attn_layer_desc *desc, g4attn_cache *cache,
  * The keys are split into fixed-size chunks; each chunk yields a partial
  * softmax (max, sum, weighted values) and a combine kernel merges them.
  * A sequence with len[b] == 0 gets a zero output and the device status word
- * records G4ATTN_ECACHE_EMPTY. */
+ * records G4ATTN_ECACHE_EMPTY.  A bidirectional layer has no decode step:
+ * G4ATTN_EUNSUPPORTED. */
 int g4attn_decode(const g4attn_layer_desc *desc, const g4attn_cache *cache,
                   const void *q_raw, const void *q_norm_w, void *out,
                   void *workspace, size_t ws_bytes, void *stream);

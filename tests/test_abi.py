@@ -62,7 +62,7 @@ def ccache(d, B=1, C=64, rolling=0, **kw):
     dict(num_kv_heads=0), dict(window=0),
     dict(rotary_fraction=0.3), dict(rotary_fraction=1.5), dict(rope_theta=-1.0),
     dict(rms_eps=-1.0), dict(softmax_scale=float("inf")), dict(softmax_scale=0.0),
-    dict(softmax_scale=-0.5), dict(layer_type=2), dict(logit_softcap=-1.0),
+    dict(softmax_scale=-0.5), dict(layer_type=3), dict(layer_type=-1), dict(logit_softcap=-1.0),
     dict(logit_softcap=float("inf")), dict(logit_softcap=float("nan")),
 ])
 def test_bad_descriptors_are_rejected(bad):
@@ -263,3 +263,81 @@ def test_single_tensor_cache_validation():
                 num_heads=32, num_kv_heads=2)
     assert lib.g4attn_decode_noalloc(ctypes.byref(wide), ctypes.byref(single(wide)), FAKE, FAKE,
                                      FAKE, None) == G.G4ATTN_EUNSUPPORTED
+
+
+def attend_rc(d, B=1, T=16, p0=32, q=FAKE, cache=None, out=FAKE, ws=FAKE, ws_bytes=1 << 40):
+    return G.lib().g4attn_attend(ctypes.byref(d), B, T, p0, q, None, None,
+                                 ctypes.byref(cache) if cache is not None else None, out, ws,
+                                 ws_bytes, None)
+
+
+def test_attend_validation():
+    """Attention from post-prologue queries reads a two-tensor cache that
+    holds every position up to the call's last at slot = position."""
+    lib = G.lib()
+    d = desc()
+    assert attend_rc(d) == G.G4ATTN_EINVAL  # no cache
+    assert attend_rc(d, q=None, cache=ccache(d, C=64)) == G.G4ATTN_EINVAL
+    assert attend_rc(d, out=None, cache=ccache(d, C=64)) == G.G4ATTN_EINVAL
+    assert attend_rc(d, p0=56, T=16, cache=ccache(d, C=64)) == G.G4ATTN_EINVAL
+    assert attend_rc(d, p0=-1, cache=ccache(d, C=64)) == G.G4ATTN_EINVAL
+    assert attend_rc(d, B=2, cache=ccache(d, C=64)) == G.G4ATTN_EINVAL  # batch mismatch
+    c = ccache(d, C=64)
+    c.v = None  # a single-tensor cache holds no K to read
+    assert attend_rc(d, cache=c) == G.G4ATTN_EINVAL  # ... and this layer is not K=V
+    g = desc(layer_type=G.G4ATTN_GLOBAL, head_dim=512, rotary_fraction=0.25, k_eq_v=True,
+             num_heads=8, num_kv_heads=2)
+    c = ccache(g, C=64)
+    c.v = None
+    c.k_norm_w = FAKE
+    assert attend_rc(g, cache=c) == G.G4ATTN_EUNSUPPORTED
+    assert attend_rc(d, cache=ccache(d, C=64), ws=None, ws_bytes=0) == G.G4ATTN_EWORKSPACE
+    assert attend_rc(d, T=0, cache=ccache(d, C=64)) == G.G4ATTN_OK
+    assert lib.g4attn_attend_workspace_size(ctypes.byref(d), 1, 16, -1) == 0
+    # no q_hat area: the row intervals and the padding bits only
+    n = lib.g4attn_attend_workspace_size(ctypes.byref(d), 2, 100, 900)
+    assert 2 * 2 * 100 * 4 + 2 * 16 * 8 <= n < 2 * 100 * 8 * 256 * 2
+
+
+def test_bidirectional_layer_has_prefill_but_no_decode():
+    """The vision-tower layer type: prefill and attend take it (the window is
+    ignored), append and decode have no step for it."""
+    lib = G.lib()
+    d = desc(layer_type=G.G4ATTN_BIDIRECTIONAL, window=0, softmax_scale=1.0)
+    assert prefill_rc(d, ws=None, ws_bytes=0) == G.G4ATTN_EWORKSPACE  # passes validation
+    assert lib.g4attn_prefill_workspace_size(ctypes.byref(d), 1, 16) > 0
+    assert attend_rc(d, cache=ccache(d, C=64), ws=None, ws_bytes=0) == G.G4ATTN_EWORKSPACE
+    c = ccache(d, C=64)
+    assert lib.g4attn_cache_append(ctypes.byref(d), ctypes.byref(c), FAKE, FAKE, FAKE,
+                                   None) == G.G4ATTN_EUNSUPPORTED
+    assert lib.g4attn_decode(ctypes.byref(d), ctypes.byref(c), FAKE, FAKE, FAKE, FAKE, 1 << 40,
+                             None) == G.G4ATTN_EUNSUPPORTED
+    assert lib.g4attn_decode_noalloc(ctypes.byref(d), ctypes.byref(c), FAKE, FAKE, FAKE,
+                                     None) == G.G4ATTN_EUNSUPPORTED
+    assert prefill_rc(d, cache=ccache(d, C=64, rolling=1)) == G.G4ATTN_EINVAL  # rolling: sliding only
+
+
+def qkv_rc(d, B=1, T=16, p0=0, x=FAKE, hidden=64, w=FAKE, wk=FAKE, q=FAKE, cache=None):
+    return G.lib().g4attn_qkv_prologue(ctypes.byref(d), B, T, p0, x, hidden, w, FAKE, wk, q,
+                                       ctypes.byref(cache) if cache is not None else None, None)
+
+
+def test_qkv_prologue_validation():
+    """The fused projection checks its shapes and pointers before any launch:
+    a hidden size whose rows are not 16-byte multiples, misaligned operands,
+    a non-rolling cache too small for p0 + T, fp32 (no tensor-core kernel)."""
+    d = desc()
+    assert qkv_rc(d, x=None) == G.G4ATTN_EINVAL
+    assert qkv_rc(d, w=None) == G.G4ATTN_EINVAL
+    assert qkv_rc(d, q=None) == G.G4ATTN_EINVAL
+    assert qkv_rc(d, hidden=4) == G.G4ATTN_EINVAL
+    assert qkv_rc(d, hidden=100) == G.G4ATTN_EINVAL  # 200-byte rows
+    assert qkv_rc(d, x=ctypes.c_void_p(0x10008)) == G.G4ATTN_EINVAL  # not 16-byte aligned
+    assert qkv_rc(d, B=-1) == G.G4ATTN_EINVAL
+    assert qkv_rc(d, p0=-3) == G.G4ATTN_EINVAL
+    assert qkv_rc(desc(dtype=torch.float32)) == G.G4ATTN_EUNSUPPORTED
+    assert qkv_rc(d, wk=None, cache=ccache(d, C=64)) == G.G4ATTN_EINVAL  # K needs w_k
+    assert qkv_rc(d, p0=60, T=16, cache=ccache(d, C=64)) == G.G4ATTN_ECACHE_OVERFLOW
+    assert qkv_rc(d, B=2, cache=ccache(d, C=64)) == G.G4ATTN_EINVAL  # batch mismatch
+    assert qkv_rc(d, T=0, cache=ccache(d, C=64)) == G.G4ATTN_OK
+    assert qkv_rc(d, T=0) == G.G4ATTN_OK  # queries only (a KV-shared layer)
