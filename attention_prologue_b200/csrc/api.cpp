@@ -132,7 +132,7 @@ static KeyMask cache_mask(const g4attn_cache* c) {
 
 // Workspace of one prefill call.
 struct PrefillWs {
-  size_t q_hat, kv, intervals, bits, total;  // byte offsets / sizes
+  size_t q_hat, kv, intervals, bits, span, total;  // byte offsets / sizes
   bool need_kv;                              // keys go to scratch (no usable cache)
   int words;                                 // 64-key words of the padding bits
 };
@@ -152,9 +152,22 @@ static PrefillWs prefill_ws(const LayerCfg& L, int B, int T, bool need_kv, bool 
   w.words = (Tk + 63) / 64;
   w.bits = off;
   if (mask) off += align256((size_t)B * w.words * sizeof(uint64_t));
+  w.span = off;
+  if (mask) off += align256((size_t)B * sizeof(int2));
   w.total = off;
   w.need_kv = need_kv;
   return w;
+}
+
+// The first and last kept position of every sequence (the row intervals are
+// clamped to them: key tiles of padding alone are never visited), or none.
+static cudaError_t padding_span(const PrefillWs& w, char* ws, int B, int Tk, const uint8_t* mask,
+                                const int2** span, cudaStream_t s) {
+  *span = nullptr;
+  if (!mask) return cudaSuccess;
+  int2* sp = reinterpret_cast<int2*>(ws + w.span);
+  *span = sp;
+  return launch_mask_span(B, Tk, mask, sp, s);
 }
 
 // The padding bits of a prefill call, or none.
@@ -176,7 +189,7 @@ extern "C" {
 size_t g4attn_prefill_workspace_size(const g4attn_layer_desc* desc, int B, int T) {
   LayerCfg L;
   if (make_cfg(desc, &L) != G4ATTN_OK || B < 0 || T < 0) return 0;
-  return prefill_ws(L, B, T, true, L.layer_type != G4ATTN_GLOBAL, true, T).total;
+  return prefill_ws(L, B, T, true, true, true, T).total;
 }
 
 size_t g4attn_decode_workspace_size(const g4attn_layer_desc* desc, const g4attn_cache* cache) {
@@ -215,7 +228,8 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
   // 0..T-1 at slots 0..T-1, otherwise from scratch
   const bool cache_is_src = cache && cache->capacity >= T && !single_tensor(cache);
   const bool bidir = L.layer_type == G4ATTN_BIDIRECTIONAL;
-  const bool intervals = (L.layer_type == G4ATTN_SLIDING && image_block_ids != nullptr) || bidir;
+  const bool intervals = (L.layer_type == G4ATTN_SLIDING && image_block_ids != nullptr) || bidir ||
+                         attention_mask != nullptr;
   PrefillWs w = prefill_ws(L, B, T, !cache_is_src, intervals, attention_mask != nullptr, T);
   if (!workspace || ws_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return G4ATTN_EWORKSPACE;
@@ -249,8 +263,13 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
     int32_t* lo = reinterpret_cast<int32_t*>(ws + w.intervals);
     int32_t* hi = reinterpret_cast<int32_t*>(ws + w.intervals +
                                              align256((size_t)B * T * sizeof(int32_t)));
-    e = bidir ? launch_chunk_intervals(L, B, T, 0, nullptr, lo, hi, s)
-              : launch_block_intervals(L, B, T, image_block_ids, lo, hi, s);
+    const int2* span;
+    if (padding_span(w, ws, B, T, attention_mask, &span, s) != cudaSuccess) return G4ATTN_ECUDA;
+    e = (bidir || span)
+            ? launch_chunk_intervals(
+                  L, B, T, 0, L.layer_type == G4ATTN_SLIDING ? image_block_ids : nullptr, span,
+                  lo, hi, s)
+            : launch_block_intervals(L, B, T, image_block_ids, lo, hi, s);
     if (e != cudaSuccess) return G4ATTN_ECUDA;
     rows = {lo, hi};
   }
@@ -310,9 +329,12 @@ int g4attn_prefill_chunk(const g4attn_layer_desc* desc, int B, int T, int p0, co
   int32_t* lo = reinterpret_cast<int32_t*>(ws + w.intervals);
   int32_t* hi =
       reinterpret_cast<int32_t*>(ws + w.intervals + align256((size_t)B * T * sizeof(int32_t)));
+  const int2* span;
+  if (padding_span(w, ws, B, p0 + T, attention_mask, &span, s) != cudaSuccess)
+    return G4ATTN_ECUDA;
   e = launch_chunk_intervals(L, B, T, p0,
-                             L.layer_type == G4ATTN_SLIDING ? image_block_ids : nullptr, lo, hi,
-                             s);
+                             L.layer_type == G4ATTN_SLIDING ? image_block_ids : nullptr, span, lo,
+                             hi, s);
   if (e != cudaSuccess) return G4ATTN_ECUDA;
   const KVSrc src{cache->k, cache->v, cache->capacity, p0 + T};
   const RowIntervals rows{lo, hi};
@@ -389,8 +411,11 @@ int g4attn_attend(const g4attn_layer_desc* desc, int B, int T, int p0, const voi
   int32_t* lo = reinterpret_cast<int32_t*>(ws + w.intervals);
   int32_t* hi =
       reinterpret_cast<int32_t*>(ws + w.intervals + align256((size_t)B * T * sizeof(int32_t)));
+  const int2* span;
+  if (padding_span(w, ws, B, p0 + T, attention_mask, &span, s) != cudaSuccess)
+    return G4ATTN_ECUDA;
   cudaError_t e = launch_chunk_intervals(
-      L, B, T, p0, L.layer_type == G4ATTN_SLIDING ? image_block_ids : nullptr, lo, hi, s);
+      L, B, T, p0, L.layer_type == G4ATTN_SLIDING ? image_block_ids : nullptr, span, lo, hi, s);
   if (e != cudaSuccess) return G4ATTN_ECUDA;
   const KVSrc src{cache->k, cache->v, cache->capacity, p0 + T};
   const RowIntervals rows{lo, hi};

@@ -230,16 +230,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       lo = max(0, i - window + 1);
       hi = i;
     }
-    atomicMin(&sc->klo, lo);
-    atomicMax(&sc->khi, hi);
+    if (lo <= hi) {  // a row left without keys (padding) widens nothing
+      atomicMin(&sc->klo, lo);
+      atomicMax(&sc->khi, hi);
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   cluster_sync_all();  // the peer's barriers exist before any remote access
   const uint32_t tmem = sc->tmem_base;
-  const int kt0 = sc->klo / BN;
-  const int n_tiles = sc->khi / BN - kt0 + 1;  // same in both CTAs: same rows
+  // same in both CTAs (same rows); no row with a key: one key tile, all masked
+  const bool none = sc->khi < sc->klo;
+  const int kt0 = none ? 0 : sc->klo / BN;
+  const int n_tiles = none ? 1 : sc->khi / BN - kt0 + 1;
 
   if (warp == 0 || warp == 2) {
     // ------------------------------------------------------------ producers

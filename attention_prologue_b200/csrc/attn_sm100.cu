@@ -131,11 +131,15 @@ __device__ __forceinline__ TileInfo tile_info(int t, int n_rt, int n_hg, int gp_
     lo = 0x7fffffff;
     hi = -1;
     for (int i = ti.p0 + (int)(threadIdx.x & 31); i <= p1; i += 32) {
-      lo = min(lo, rows.lo[(long)ti.b * T_ + i]);
-      hi = max(hi, rows.hi[(long)ti.b * T_ + i]);
+      const int a = rows.lo[(long)ti.b * T_ + i], e = rows.hi[(long)ti.b * T_ + i];
+      if (a <= e) {  // a row left without keys (padding) widens nothing
+        lo = min(lo, a);
+        hi = max(hi, e);
+      }
     }
     lo = __reduce_min_sync(0xffffffffu, lo);
     hi = __reduce_max_sync(0xffffffffu, hi);
+    if (hi < lo) lo = hi = 0;  // no row has a key: one key tile, all of it masked
   } else {
     lo = layer_type == 1 ? 0 : max(0, ti.p0 - window + 1);
     hi = p1;

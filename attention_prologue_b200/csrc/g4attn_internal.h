@@ -84,7 +84,9 @@ cudaError_t launch_block_intervals(const LayerCfg& L, int B, int T, const int32_
 // Per-row key intervals of a cached-prefill chunk (positions p0 .. p0+T-1);
 // ids [B][p0 + T] or nullptr.
 cudaError_t launch_chunk_intervals(const LayerCfg& L, int B, int T, int p0, const int32_t* ids,
-                                   int32_t* lo, int32_t* hi, cudaStream_t s);
+                                   const int2* span, int32_t* lo, int32_t* hi, cudaStream_t s);
+// span[b] = (first, last) kept position of sequence b's padding mask [B][Tk]
+cudaError_t launch_mask_span(int B, int Tk, const uint8_t* mask, int2* span, cudaStream_t s);
 cudaError_t launch_attention_simt(const LayerCfg& L, int B, int T, const void* q_hat, KVSrc kv,
                                   RowIntervals rows, KeyBits kb, void* out, cudaStream_t s);
 // tcgen05 prefill attention (bf16, head_dim 64/128/256/512); q_hat [B, T, Hq, d].

@@ -380,8 +380,8 @@ cudaError_t launch_block_intervals(const LayerCfg& L, int B, int T, const int32_
 // non-negative ids (ids [B][p0 + T], or nullptr) that contains pos, seen up
 // to the chunk's last position.
 __global__ void chunk_interval_kernel(const int32_t* __restrict__ ids, int B, int T_, int p0,
-                                      int layer_type, int window, int32_t* __restrict__ lo,
-                                      int32_t* __restrict__ hi) {
+                                      int layer_type, int window, const int2* __restrict__ span,
+                                      int32_t* __restrict__ lo, int32_t* __restrict__ hi) {
   const long idx = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long)B * T_) return;
   const int i = (int)(idx % T_);
@@ -405,15 +405,53 @@ __global__ void chunk_interval_kernel(const int32_t* __restrict__ ids, int B, in
       }
     }
   }
+  if (span) {  // keys outside [first kept, last kept] are padding: not visited
+    a = max(a, span[b].x);
+    e = min(e, span[b].y);  // a > e: the row has no key
+  }
   lo[idx] = a;
   hi[idx] = e;
 }
 
 cudaError_t launch_chunk_intervals(const LayerCfg& L, int B, int T, int p0, const int32_t* ids,
-                                   int32_t* lo, int32_t* hi, cudaStream_t s) {
+                                   const int2* span, int32_t* lo, int32_t* hi, cudaStream_t s) {
   const long n = (long)B * T;
   chunk_interval_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
-      ids, B, T, p0, L.layer_type, L.window, lo, hi);
+      ids, B, T, p0, L.layer_type, L.window, span, lo, hi);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// First and last kept position of each sequence's padding mask (uint8
+// [B][Tk], non-zero = keep): span[b] = (first, last), or (Tk, -1) when the
+// whole sequence is padding.  One block per sequence.
+__global__ void mask_span_kernel(const uint8_t* __restrict__ mask, int Tk,
+                                 int2* __restrict__ span) {
+  __shared__ int s_first, s_last;
+  if (threadIdx.x == 0) {
+    s_first = Tk;
+    s_last = -1;
+  }
+  __syncthreads();
+  const uint8_t* row = mask + (long)blockIdx.x * Tk;
+  int f = Tk, l = -1;
+  for (int t = threadIdx.x; t < Tk; t += blockDim.x)
+    if (row[t]) {
+      f = min(f, t);
+      l = max(l, t);
+    }
+  f = __reduce_min_sync(0xffffffffu, f);
+  l = __reduce_max_sync(0xffffffffu, l);
+  if ((threadIdx.x & 31) == 0) {
+    atomicMin(&s_first, f);
+    atomicMax(&s_last, l);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) span[blockIdx.x] = make_int2(s_first, s_last);
+}
+
+cudaError_t launch_mask_span(int B, int Tk, const uint8_t* mask, int2* span, cudaStream_t s) {
+  mask_span_kernel<<<B, 256, 0, s>>>(mask, Tk, span);
   count_launch();
   return cudaGetLastError();
 }

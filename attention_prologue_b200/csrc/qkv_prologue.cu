@@ -167,7 +167,14 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
       for (int t = blockIdx.x; ok && t < a.n_tiles; t += gridDim.x) {
         int mt, head;
         qkv_tile(a, t, &mt, &head);
-        for (int kb = 0; kb < n_k; ++kb) {
+        // the k loop starts at a tile-dependent offset: the CTAs that sweep
+        // one head (or one token tile) at the same time then read different
+        // lines of its W rows (of its x rows); many SMs reading the same
+        // lines at once serialise in L2.  The MMA side counts iterations, so
+        // only the order of the fp32 accumulation changes.
+        const int kb0 = (mt + 5 * head) % n_k;
+        for (int i = 0; i < n_k; ++i) {
+          const int kb = kb0 + i < n_k ? kb0 + i : kb0 + i - n_k;
           const int s = g % NS;
           if (!(ok = mbar_wait(empty(s), ((g / NS) & 1) ^ 1, abort))) break;
           const uint32_t st = base + s * Ly::kStage;

@@ -149,9 +149,11 @@ def test_workspace_sizes():
     B, T = 1, 8192
     ws = G.lib().g4attn_prefill_workspace_size(ctypes.byref(d), B, T)
     # q_hat + K/V scratch + two int32 interval arrays + the padding bits (one
-    # 64-bit word per 64 keys, 256-byte aligned), 256-aligned pieces
+    # 64-bit word per 64 keys) + each sequence's first and last kept position
+    # (two int32), 256-aligned pieces
     bits = -(-(B * (T // 64) * 8) // 256) * 256
-    assert ws == B * T * 8 * 256 * 2 + 2 * B * T * 1 * 256 * 2 + 2 * B * T * 4 + bits
+    span = -(-(B * 8) // 256) * 256
+    assert ws == B * T * 8 * 256 * 2 + 2 * B * T * 1 * 256 * 2 + 2 * B * T * 4 + bits + span
     c = ccache(d, B=64, C=1024, rolling=1)
     dws = G.lib().g4attn_decode_workspace_size(ctypes.byref(d), ctypes.byref(c))
     assert dws > 0 and dws % 256 == 0
