@@ -580,8 +580,10 @@ def bench_decode(args, dist: Dist, pk: dict, clk: ClockSampler):
             "roofline": {"bound": "hbm", "kernel": "decode split-KV (global layer, K rebuilt)",
                          "achieved": g1_bytes / (g1_ms * 1e-3) / 1e9, "peak": peak,
                          "unit": "GB/s", "frac": g1_bytes / (g1_ms * 1e-3) / 1e9 / peak,
-                         "traffic": None, "algorithmic_per_launch": g1_bytes,
-                         "avg_launch_ms": g1_ms}}
+                         "traffic": (profile_field("decode_mma_26b_a4b_global_single.md",
+                                                   "traffic_bytes_per_launch")
+                                     if w.batch == 64 and dist.rank == 0 else None),
+                         "algorithmic_per_launch": g1_bytes, "avg_launch_ms": g1_ms}}
         del sg
         g_cache = None
     del g_cache, s_cache
