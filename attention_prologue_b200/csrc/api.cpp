@@ -105,8 +105,11 @@ static int make_cfg(const g4attn_layer_desc* d, LayerCfg* L) {
   L->softcap = d->logit_softcap;
   std::memset(&L->rope, 0, sizeof(L->rope));
   L->rope.rotated_pairs = (int)(R2 / 2);
-  for (int k = 0; k < L->rope.rotated_pairs; ++k)
+  for (int k = 0; k < L->rope.rotated_pairs; ++k) {
     L->rope.inv_freq[k] = std::pow(d->rope_theta, -2.0 * k / (double)d->head_dim);
+    // < 1/(2 pi) turns per position (inv_freq <= 1): the fraction fits 64 bits
+    L->rope.turns[k] = (unsigned long long)std::ldexp(L->rope.inv_freq[k] / 6.283185307179586476925, 64);
+  }
   return G4ATTN_OK;
 }
 

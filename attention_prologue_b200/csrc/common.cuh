@@ -109,6 +109,21 @@ template <int N> struct Vec<__nv_bfloat16, N> {
   }
 };
 
+// sin/cos of the RoPE angle pos * f from the frequency in turns as a 64-bit
+// binary fraction, F = f / (2 pi) * 2^64: the fractional turns of pos * f
+// are bits 32..63 of the wrapping integer product pos * F (two integer
+// multiplies, no fp64), read as a signed fraction in [-1/2, 1/2) turn and
+// handed to the hardware approximation on [-pi, pi).  F carries f to 2^-53
+// relative, as the fp64 product in rope_sincos does; the 32-bit turn rounds
+// to 24 bits in the float conversion (2e-7 rad).
+__device__ __forceinline__ void rope_sincos_turns(uint32_t pos, unsigned long long F, float* s,
+                                                  float* c) {
+  const uint32_t lo = (uint32_t)F, hi = (uint32_t)(F >> 32);
+  const uint32_t top = __umulhi(lo, pos) + hi * pos;
+  const float turns = (float)(int32_t)top * 2.3283064365386963e-10f;  // 2^-32
+  __sincosf(turns * 6.283185307179586f, s, c);
+}
+
 // Angle pos * inv_freq reduced to [-pi, pi] in fp64, then sin/cos in fp32.
 // (pos * inv_freq in fp32 would err by up to ~1e-2 rad at pos ~ 1.3e5.)
 __device__ __forceinline__ void rope_sincos(long pos, double inv_freq, float* s, float* c) {

@@ -63,7 +63,7 @@ struct DmSingle {
   int ns;              // stages (a multiple of 4)
   uint32_t stage;      // bytes per stage
   uint32_t q, bars;    // q_hat [8][D]; full, empty, ready [NS] each
-  uint32_t freq;       // [R] double: the rotated pairs' frequencies
+  uint32_t freq;       // [R] the rotated pairs' frequencies in turns (64-bit fractions)
   uint32_t wab;        // [R] float2: (w_k[k], w_k[k + D/2])
   uint32_t box_slot;   // 4 bits per 64-dim box: its rebuilt slot, 15 = loaded tile
   uint32_t slot_box;   // 4 bits per rebuilt slot: its box
@@ -194,10 +194,10 @@ __global__ void __launch_bounds__(kThreadsDm + (kSingle ? kRebuilders * 32 : 0),
   if constexpr (kSingle) {
     // per rotated pair k: its frequency and (w_k[k], w_k[k + D/2]), in shared
     // memory (lane-indexed reads of the kernel's parameter space serialise)
-    double* fq = reinterpret_cast<double*>(smem + sp.freq);
+    unsigned long long* fq = reinterpret_cast<unsigned long long*>(smem + sp.freq);
     float2* wab = reinterpret_cast<float2*>(smem + sp.wab);
     for (int k = threadIdx.x; k < rope.rotated_pairs; k += blockDim.x) {
-      fq[k] = rope.inv_freq[k];
+      fq[k] = rope.turns[k];
       wab[k] = make_float2(__bfloat162float(wk_single[k]), __bfloat162float(wk_single[k + D / 2]));
     }
   }
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kThreadsDm + (kSingle ? kRebuilders * 32 : 0),
     // Other nch: any (key, chunk) per item, one sincos per pair and item.
     const int rw = warp - kConsumers - 1;
     const int R = rope.rotated_pairs, nch = sp.nw / 4;
-    const double* fq = reinterpret_cast<const double*>(smem + sp.freq);
+    const unsigned long long* fq = reinterpret_cast<const unsigned long long*>(smem + sp.freq);
     const float2* wab = reinterpret_cast<const float2*>(smem + sp.wab);
     const bool fixed_c = 32 % nch == 0;
     const int c = fixed_c ? lane % nch : 0, grp = fixed_c ? 32 / nch : 1;
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kThreadsDm + (kSingle ? kRebuilders * 32 : 0),
         const float2 u = wab[k];
         wa[t] = u.x;
         wb[t] = u.y;
-        rope_sincos(1, fq[k], &sd[t], &cd[t]);
+        rope_sincos_turns(1, fq[k], &sd[t], &cd[t]);
       }
     }
     // one item: key j, chunk cc, the pairs' angles (cs, sn) at pos0 + j
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kThreadsDm + (kSingle ? kRebuilders * 32 : 0),
           for (int t = 0; t < 8; ++t) {
             cs[t] = 1.f;
             sn[t] = 0.f;
-            if (8 * c + t < R) rope_sincos(pos0 + j0, fq[8 * c + t], &sn[t], &cs[t]);
+            if (8 * c + t < R) rope_sincos_turns((uint32_t)(pos0 + j0), fq[8 * c + t], &sn[t], &cs[t]);
           }
           for (int m = 0; m < kpl; ++m) {
             item(sk, sr, j0 + m, c, cs, sn, wa, wb);
@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kThreadsDm + (kSingle ? kRebuilders * 32 : 0),
             cs[t] = ua[t] = ub[t] = 1.f;
             sn[t] = 0.f;
             if (k < R) {
-              rope_sincos(pos0 + j, fq[k], &sn[t], &cs[t]);
+              rope_sincos_turns((uint32_t)(pos0 + j), fq[k], &sn[t], &cs[t]);
               ua[t] = wab[k].x;
               ub[t] = wab[k].y;
             }

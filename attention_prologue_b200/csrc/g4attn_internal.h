@@ -13,6 +13,9 @@ constexpr int kMaxHalf = 256;  // head_dim <= 512
 // inv_freq[k] = theta^(-2k/d) computed on the host in fp64.
 struct RopeParams {
   double inv_freq[kMaxHalf];
+  // the same frequencies in turns per position as 64-bit binary fractions,
+  // F = inv_freq / (2 pi) * 2^64 (rope_sincos_turns)
+  unsigned long long turns[kMaxHalf];
   int rotated_pairs;
 };
 

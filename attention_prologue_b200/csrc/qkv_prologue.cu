@@ -55,7 +55,7 @@ struct QkvLayout {
   static constexpr int kStages = kFit > 8 ? 8 : kFit;  // 8, 6, 4, 2
   static constexpr uint32_t kBars = kStages * kStage;
   static constexpr uint32_t kW = kBars + 256;          // float w_q [D], w_k [D]
-  static constexpr uint32_t kFreq = kW + 2 * D * 4;    // double inv_freq [D / 2]
+  static constexpr uint32_t kFreq = kW + 2 * D * 4;    // the pairs' frequencies in turns [D / 2]
   static constexpr uint32_t kAlloc = kFreq + (D / 2) * 8;
   static_assert(kAlloc + 1024 <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
   static_assert(2 * kStages + 5 <= 32, "barriers fit their 256 bytes");
@@ -176,8 +176,8 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
 // or the weightless vectors.  Warp-collective (the TMEM loads).
 template <int D>
 __device__ __forceinline__ void qkv_epilogue_tile(const QkvArgs& a, uint32_t tacc, int m,
-                                                  int head, const float* wsm, const double* fq,
-                                                  int R) {
+                                                  int head, const float* wsm,
+                                                  const unsigned long long* fq, int R) {
   // pass 1: the head's mean square, from the fp32 accumulator
   float ss = 0.f;
 #pragma unroll 1
@@ -238,7 +238,7 @@ __device__ __forceinline__ void qkv_epilogue_tile(const QkvArgs& a, uint32_t tac
           y1[u] *= w[kp + D / 2];
           if (kp < R) {
             float sn, cs;
-            rope_sincos(pos, fq[kp], &sn, &cs);
+            rope_sincos_turns((uint32_t)pos, fq[kp], &sn, &cs);
             const float t0 = y0[u] * cs - y1[u] * sn;
             y1[u] = y0[u] * sn + y1[u] * cs;
             y0[u] = t0;
@@ -289,14 +289,14 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
   const uint32_t drain = bars + 8u * (uint32_t)(2 * NS + 4);
 
   float* wsm = reinterpret_cast<float*>(smem + Ly::kW);  // w_q [D], w_k [D]
-  double* fq = reinterpret_cast<double*>(smem + Ly::kFreq);
+  unsigned long long* fq = reinterpret_cast<unsigned long long*>(smem + Ly::kFreq);
   for (int k = threadIdx.x; k < D; k += blockDim.x) {
     wsm[k] = __bfloat162float(a.wq[k]);
     wsm[D + k] = a.wk ? __bfloat162float(a.wk[k]) : 1.f;
   }
   // the frequencies in shared memory: lane-indexed reads of the parameter
   // space would serialise
-  for (int k = threadIdx.x; k < rope.rotated_pairs; k += blockDim.x) fq[k] = rope.inv_freq[k];
+  for (int k = threadIdx.x; k < rope.rotated_pairs; k += blockDim.x) fq[k] = rope.turns[k];
   if (blockIdx.x == 0 && a.len)
     for (int b = threadIdx.x; b < a.B; b += blockDim.x) a.len[b] = a.p0 + a.T;
   if (threadIdx.x == 0) {
@@ -461,12 +461,12 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
   const int pair = (int)blockIdx.x >> 1, n_pairs = (int)gridDim.x >> 1;
 
   float* wsm = reinterpret_cast<float*>(smem + Ly::kW);
-  double* fq = reinterpret_cast<double*>(smem + Ly::kFreq);
+  unsigned long long* fq = reinterpret_cast<unsigned long long*>(smem + Ly::kFreq);
   for (int k = threadIdx.x; k < D; k += blockDim.x) {
     wsm[k] = __bfloat162float(a.wq[k]);
     wsm[D + k] = a.wk ? __bfloat162float(a.wk[k]) : 1.f;
   }
-  for (int k = threadIdx.x; k < rope.rotated_pairs; k += blockDim.x) fq[k] = rope.inv_freq[k];
+  for (int k = threadIdx.x; k < rope.rotated_pairs; k += blockDim.x) fq[k] = rope.turns[k];
   if (blockIdx.x == 0 && a.len)
     for (int b = threadIdx.x; b < a.B; b += blockDim.x) a.len[b] = a.p0 + a.T;
   if (threadIdx.x == 0) {

@@ -659,7 +659,7 @@ def bench_qkv(args, dist: Dist, pk: dict, clk: ClockSampler, steps: int):
            "value": job_rate(dist.world, flops, steps, total) / 1e12,
            "ms_per_step": total / steps, "steps": steps, "flops": flops, "launches": launches,
            "workload": f"{w.name}: x [{w.B}, {w.T}, {hidden}] -> {n_rows} rows of W",
-           "roofline": {"bound": "tensor", "kernel": "qkv_prologue_kernel<256>",
+           "roofline": {"bound": "tensor", "kernel": "qkv_pair_kernel<256> (CTA pairs)",
                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                         "frac": achieved / peak,
                         "traffic": profile_field("qkv_prologue_e2b.md", "traffic_bytes_per_launch"),
