@@ -662,7 +662,7 @@ def bench_qkv(args, dist: Dist, pk: dict, clk: ClockSampler, steps: int):
            "roofline": {"bound": "tensor", "kernel": "qkv_pair_kernel<256> (CTA pairs)",
                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                         "frac": achieved / peak,
-                        "traffic": profile_field("qkv_prologue_e2b.md", "traffic_bytes_per_launch"),
+                        "traffic": profile_field("qkv_pair_e2b.md", "traffic_bytes_per_launch"),
                         "algorithmic_per_launch": flops, "avg_launch_ms": avg},
            "cublas_projection_only": {"ms": statistics.mean(c_ms),
                                       "tflops": flops / (statistics.mean(c_ms) * 1e-3) / 1e12,
