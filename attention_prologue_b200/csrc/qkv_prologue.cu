@@ -148,14 +148,19 @@ __device__ __forceinline__ void mma_pair_ss(uint32_t d_tmem, uint64_t a_desc, ui
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
-// One arrival on the mbarrier at offset `bar` of each CTA in `mask` once the
-// issuing thread's earlier pair MMAs are complete.
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t mask) {
+// One arrival on the mbarrier at `bar_cluster` (a shared::cluster address:
+// this CTA's own barrier or the peer's) once the issuing thread's earlier
+// pair MMAs are complete.
+__device__ __forceinline__ void mma_commit_pair_to(uint32_t bar_cluster) {
   asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(bar),
-      "h"(mask)
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          bar_cluster)
       : "memory");
+}
+// ... on the barrier at the same offset in both CTAs of the pair (two commits)
+__device__ __forceinline__ void mma_commit_pair_both(uint32_t bar) {
+  mma_commit_pair_to(bar);
+  mma_commit_pair_to(map_peer(bar, 1));
 }
 // A tile into this CTA's shared memory whose bytes are counted on an
 // mbarrier of the pair's even CTA (a shared::cluster address).
@@ -426,6 +431,8 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
 // x one head; the even CTA issues M256 MMAs (cta_group::2) that read each
 // CTA's 128 x rows and the two halves of the head's W rows from the two
 // CTAs' shared memory and accumulate each CTA's 128 rows in its own TMEM.
+// No load or commit uses cluster multicast: each CTA loads its own tiles and
+// the even CTA commits once to each CTA's barrier.
 //   warp 0      (both) TMA of this CTA's x rows and W half; the bytes of both
 //               CTAs are counted on the even CTA's full barrier
 //   warp 1      (both) TMEM allocation; (even) the MMA issuer, whose commits
@@ -557,13 +564,13 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
                           desc_add(db0, off + h * Ly::kBHalf), idesc,
                           (i > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit_pair(empty(s), 3);  // frees the stage in both CTAs
+          mma_commit_pair_both(empty(s));  // frees the stage in both CTAs
           ++g;
         }
-        if (ok) mma_commit_pair(acc_full(ai), 3);
+        if (ok) mma_commit_pair_both(acc_full(ai));
       }
       if (*abort) {  // every pair MMA issued so far completes before TMEM is freed
-        mma_commit_pair(drain, 1);
+        mma_commit_pair_to(drain);
         mbar_wait(drain, 0, nullptr);
       }
     }

@@ -2,7 +2,8 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--no-extra-prefill] [--no-decode] [--decode-only]
-                    [--decode-batch B] [--no-e2e] [--no-cpu-baseline]
+                    [--decode-batch B] [--no-kv-single] [--no-qkv] [--no-vision]
+                    [--no-e2e] [--no-cpu-baseline]
 
 Headline: prefill attention TFLOP/s counting unmasked FLOPs only
 (4 * d * sum_i |I_i| * Hq * B; 2d for QK^T and 2d for PV per allowed pair) on
@@ -14,7 +15,11 @@ head_dim 512, each with its own roofline and CPU baseline), and the second
 half of the metric, decode KV-cache GB/s on the 26B-A4B-shaped step (64
 sequences, cache lengths uniform in [4096, 131072]; a sliding layer on a
 1024-slot rolling cache, a K=V global layer and a KV-shared layer reading it),
-under "decode".
+under "decode" (with the same step over a single-tensor K=V cache under
+"kv_single").  Two more legs: "qkv_prologue", the QKV projection with the
+prologue in its epilogue on the E2B-shaped prompt (TFLOP/s of the
+projection, cuBLAS's projection alone timed beside it), and "vision", the
+vision tower's bidirectional attention shape through g4attn_attend.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream; L2 is flushed (a 256 MiB write) before every timed
