@@ -154,3 +154,32 @@ def test_attend_matches_the_oracle(case):
     ref = _oracle_attend(L, q, k, v, p0, ids, keep)
     check_beyond_output_rounding(out, ref, f"attend {case}", p_bound=_p_bound(v))
     record(out, ref, f"attend {case} (plain bar)")
+
+
+def test_bidirectional_cached_prefill_chunks():
+    """A bidirectional layer through g4attn_prefill then g4attn_prefill_chunk:
+    the chunk's rows see every key up to the chunk's last position (the first
+    chunk's rows saw only their own chunk); both against the oracle."""
+    L = W.bidirectional(8, 2, 128, softmax_scale=128 ** -0.5)
+    B, T, p0 = 2, 520, 300
+    w = W.PrefillWorkload("bidir-chunks", L, B, T)
+    inp = W.prefill_inputs(w, DEV, 56)
+    d = desc_of(L, torch.bfloat16)
+    cache = G.KVCache.allocate(B, 2, T, 128, device=DEV)
+    sl = lambda t, a, b: t[:, a:b].contiguous()
+    o0 = G.g4attn_prefill(d, sl(inp["q_raw"], 0, p0), sl(inp["k_raw"], 0, p0),
+                          sl(inp["v_raw"], 0, p0), inp["q_norm_w"], inp["k_norm_w"], cache=cache)
+    o1 = G.g4attn_prefill_chunk(d, p0, sl(inp["q_raw"], p0, T), sl(inp["k_raw"], p0, T),
+                                sl(inp["v_raw"], p0, T), inp["q_norm_w"], inp["k_norm_w"], None,
+                                cache)
+    torch.cuda.synchronize()
+    assert G.g4attn_get_device_status() == G.G4ATTN_OK
+    cpu = {k: (v.cpu() if v is not None else None) for k, v in inp.items()}
+    OL = oracle_layer(L)
+    ref0 = oracle.prefill(OL, cpu["q_raw"][:, :p0], cpu["k_raw"][:, :p0], cpu["v_raw"][:, :p0],
+                          cpu["q_norm_w"], cpu["k_norm_w"])
+    kh, vh = oracle.prefill_kv(OL, cpu["k_raw"][:, :p0], cpu["v_raw"][:, :p0], cpu["k_norm_w"])
+    ref1, _, _ = oracle.prefill_chunk(OL, cpu["q_raw"][:, p0:], cpu["k_raw"][:, p0:],
+                                      cpu["v_raw"][:, p0:], cpu["q_norm_w"], cpu["k_norm_w"], kh, vh)
+    check(o0, ref0, torch.bfloat16, "bidirectional first chunk")
+    check(o1, ref1, torch.bfloat16, "bidirectional cached chunk")
