@@ -57,7 +57,7 @@ namespace {
 
 constexpr int BM = 128;  // query rows per work tile
 constexpr int BN = 64;   // keys per key tile
-constexpr int kStagesV = 2;
+constexpr int kMaxStages = 8;  // K or V ring slots (barrier area)
 constexpr int kNS = 4;   // S buffers in TMEM
 constexpr int kThreads = 384;
 constexpr int kSoftmaxWarp0 = 4;
@@ -66,8 +66,14 @@ constexpr int kEpiWarp0 = 8;
 template <int D>
 struct Layout {
   // Q lives in shared memory (TMEM holds NS = 4 S buffers and O: 512
-  // columns at d = 256); d = 256 then leaves room for three K stages.
-  static constexpr int kStagesK = D == 256 ? 3 : 4;
+  // columns at d = 256); d = 256 then leaves room for three K stages and two
+  // V stages.  Smaller heads take deeper rings: a tile's copy takes a few
+  // thousand cycles to land, and with two V slots the PV of key tile j waited
+  // for the copy that the PV of tile j - 2 released (the period was half
+  // that latency at d = 64).
+  static constexpr int kStagesK = D == 256 ? 3 : (D == 128 ? 6 : 8);
+  static constexpr int kStagesV = D == 256 ? 2 : (D == 128 ? 6 : 8);
+  static_assert(kStagesK <= kMaxStages && kStagesV <= kMaxStages, "ring barriers");
   static constexpr int kChunks = D / 64;                  // 64-element (128-byte) columns
   static constexpr uint32_t kQChunk = BM * 128;           // bytes of one 128-row chunk
   static constexpr uint32_t kKVChunk = BN * 128;          // bytes of one K or V chunk
@@ -92,14 +98,14 @@ struct Bars {  // offsets (in 8-byte words) of the mbarriers from Layout::kBars
     l_free = 6,    // [2] the epilogue warps have read those row sums (128 arrivals)
     drain = 8,     // (S issuer)
     drain2 = 9,    // (PV issuer)
-    k_full = 10,   // [4]
-    k_empty = 14,  // [4]
-    v_full = 18,   // [2]
-    v_empty = 20,  // [2]
-    s_full = 22,   // [NS]
-    p_full = 26,   // [NS]
-    o_done = 30,   // [NS] PV_j done (one per S buffer: rescale waits stay in one phase)
-    count = 34
+    k_full = 10,                   // [kStagesK]
+    k_empty = k_full + kMaxStages,  // [kStagesK]
+    v_full = k_empty + kMaxStages,  // [kStagesV]
+    v_empty = v_full + kMaxStages,  // [kStagesV]
+    s_full = v_empty + kMaxStages,  // [NS]
+    p_full = s_full + kNS,          // [NS]
+    o_done = p_full + kNS,  // [NS] PV_j done (one per S buffer: rescale waits stay in one phase)
+    count = o_done + kNS
   };
 };
 
@@ -109,11 +115,18 @@ struct Scalars {  // after the barriers
 };
 
 // Work tile t: sequence b, first query head h0, first position p0 (row
-// tiles latest first) and key-tile range [kt0, kt0 + n).  Warp-collective:
-// with image blocks the range is a min/max over the tile's positions.
+// tiles latest first) and key-tile range [kt0, kt0 + n), walked from
+// kt0 + rot and wrapping around.  Warp-collective: with image blocks the
+// range is a min/max over the tile's positions.
 struct TileInfo {
-  int b, h0, p0, kt0, n;
+  int b, h0, p0, kt0, n, rot;
 };
+
+// Key tile of step j of a work tile.
+__device__ __forceinline__ int key_tile(const TileInfo& ti, int j) {
+  const int jj = j + ti.rot;
+  return ti.kt0 + (jj < ti.n ? jj : jj - ti.n);
+}
 
 __device__ __forceinline__ TileInfo tile_info(int t, int n_rt, int n_hg, int gp_log2, int T_,
                                               const RowIntervals& rows, int layer_type,
@@ -146,6 +159,15 @@ __device__ __forceinline__ TileInfo tile_info(int t, int n_rt, int n_hg, int gp_
   }
   ti.kt0 = lo / BN;
   ti.n = hi < lo ? 0 : hi / BN - ti.kt0 + 1;
+  // The row tiles of one (sequence, head group) run side by side on the SMs
+  // (consecutive tiles).  Where they share a key range that starts at the
+  // same tile (global and bidirectional layers), each starts its walk at its
+  // own offset: otherwise all of them ask for the same K and V tiles at
+  // once, and the copies of those tiles were several times slower than
+  // those of staggered readers.  Sliding windows are staggered already.
+  // The order of the key tiles changes only the rounding of the online
+  // softmax.
+  ti.rot = layer_type == 0 || ti.n <= 1 ? 0 : (int)(((long)rt * ti.n) / n_rt) % ti.n;
   return ti;
 }
 
@@ -163,6 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       float cap2, int gp_log2, int n_work, int* status) {
   using Ly = Layout<D>;
   constexpr int kStagesK = Ly::kStagesK;
+  constexpr int kStagesV = Ly::kStagesV;
   static_assert(8 * Bars::count + (int)sizeof(Scalars) <= 512, "barrier area");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte-swizzle atoms assume a 1024-byte aligned base
@@ -256,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(bar(full + s), BN * D * 2);
           for (int c = 0; c < Ly::kChunks; ++c)
             tma_load_3d(ring + (s * Ly::kChunks + c) * Ly::kKVChunk, tm, bar(full + s), c * 64,
-                        (ti.kt0 + j) * BN, kv_row);
+                        key_tile(ti, j) * BN, kv_row);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -370,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the padding bits of this key tile (all kept without a mask), read
         // before the wait so the load overlaps it
         const uint64_t keep =
-            (kExtras && kb.bits) ? kb.bits[(long)ti.b * kb.words + ti.kt0 + j] : ~0ull;
+            (kExtras && kb.bits) ? kb.bits[(long)ti.b * kb.words + key_tile(ti, j)] : ~0ull;
         ok = __all_sync(0xffffffffu, mbar_wait(bar(Bars::s_full + sb), (g / kNS) & 1, abort));
         if (!ok) break;
         tc_fence_after();
@@ -378,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_off + sb * BN, sr);
         tmem_ld32(tmem + lane_off + sb * BN + 32, sr + 32);
         tmem_wait_ld();
-        const int key0 = (ti.kt0 + j) * BN;
+        const int key0 = key_tile(ti, j) * BN;
         float x[BN];
 #pragma unroll
         for (int c = 0; c < BN; ++c) x[c] = __uint_as_float(sr[c]);
