@@ -54,15 +54,20 @@ struct DmLayout {
   static_assert(kMerge <= kQ, "merge buffer fits");
 };
 
-constexpr int kRebuilders = 2;  // single-tensor caches: warps that rebuild K
+// single-tensor caches: warps that rebuild K (with the 5 others, two warps
+// per sub-partition, so the consumers keep their 252 registers)
+constexpr int kRebuilders = 3;
 
-// Shared-memory plan of a single-tensor decode (set by the host: the ring's
-// stage holds the loaded V tile and one rebuilt K box per box that has
-// rotated dims).
+// Shared-memory plan of a single-tensor decode (set by the host): a ring of
+// loaded V tiles, and a smaller ring of rebuilt K boxes (one per 64-dim box
+// that has rotated dims) whose slots are free again once the S product of
+// their tile is done, so the load ring keeps more tiles in flight.
 struct DmSingle {
-  int ns;              // stages (a multiple of 4)
-  uint32_t stage;      // bytes per stage
-  uint32_t q, bars;    // q_hat [8][D]; full, empty, ready [NS] each
+  int ns;              // load stages (a multiple of 4)
+  uint32_t stage;      // bytes per load stage (one V tile)
+  int nrs;             // rebuilt slots (a multiple of the rebuilders)
+  uint32_t rb;         // the rebuilt ring: [nrs][nrb] boxes
+  uint32_t q, bars;    // q_hat [8][D]; full, empty, ready [NS] each, rebuilt-slot free [nrs]
   uint32_t freq;       // [R] the rotated pairs' frequencies in turns (64-bit fractions)
   uint32_t wab;        // [R] float2: (w_k[k], w_k[k + D/2])
   uint32_t box_slot;   // 4 bits per 64-dim box: its rebuilt slot, 15 = loaded tile
@@ -111,8 +116,9 @@ __device__ __forceinline__ uint32_t tile_off(int key, int dim) {
 // kSingle: a single-tensor cache of a K=V layer.  The cache holds V =
 // RMSNorm(k_raw) alone and K = RoPE(V * w_k) is rebuilt per tile: w_k folds
 // into the query on the unrotated dims (q.(V*w) = (q*w).V), so only the
-// 64-dim boxes that hold rotated dims are rebuilt, by two extra warps, into
-// slots after the loaded tile; the S product reads those boxes from there.
+// 64-dim boxes that hold rotated dims are rebuilt, by three extra warps
+// taking tiles in turn, into a slot of the rebuilt ring; the S product reads
+// those boxes from there.
 // The angle of key pos0 + j is pos0 f then j f: cos/sin of pos0 f come from
 // one fp64-reduced sincos per pair and tile, those of j f (with w_k folded
 // in) from a per-CTA table.  V is the loaded tile itself.
@@ -163,6 +169,8 @@ __global__ void __launch_bounds__(kThreadsDm + (kSingle ? kRebuilders * 32 : 0),
       mbar_init(bars + 8 * (NS + s), 1);      // empty: the consuming warp
       if (kSingle) mbar_init(bars + 8 * (2 * NS + s), 32);  // ready: a rebuilding warp
     }
+    if (kSingle)
+      for (int r = 0; r < sp.nrs; ++r) mbar_init(bars + 8 * (3 * NS + r), 1);  // slot r free
     s_abort = 0;
     fence_barrier_init();
   }
@@ -236,13 +244,14 @@ __global__ void __launch_bounds__(kThreadsDm + (kSingle ? kRebuilders * 32 : 0),
     }
   } else if (kSingle && warp > kConsumers) {
     // ------------------------------------------------------------ K rebuild
-    // Rebuilder rw takes tiles i = rw (mod 2); NS is even, so every stage has
-    // one rebuilder, which waits its phases in order.  The rotated dims form
-    // nch 16-byte chunks (8 pairs) per half.  When nch divides 32 (every
-    // Gemma 4 K=V shape: R = d/8) lane l keeps chunk c = l % nch and takes
-    // kpl consecutive keys from j0; the 8 pairs' angles start from one sincos
-    // each per tile and step key to key by the angle addition formulas.
-    // Other nch: any (key, chunk) per item, one sincos per pair and item.
+    // Rebuilder rw takes tiles i = rw (mod 3); NS and nrs are multiples of
+    // 3, so every stage and every rebuilt slot has one rebuilder, which waits
+    // its phases in order.  The rotated dims form nch 16-byte chunks (8
+    // pairs) per half.  When nch divides 32 (every Gemma 4 K=V shape:
+    // R = d/8) lane l keeps chunk c = l % nch and takes kpl consecutive keys
+    // from j0; the 8 pairs' angles start from one sincos each per tile and
+    // step key to key by the angle addition formulas.  Other nch: any (key,
+    // chunk) per item, one sincos per pair and item.
     const int rw = warp - kConsumers - 1;
     const int R = rope.rotated_pairs, nch = sp.nw / 4;
     const unsigned long long* fq = reinterpret_cast<const unsigned long long*>(smem + sp.freq);
@@ -296,11 +305,15 @@ __global__ void __launch_bounds__(kThreadsDm + (kSingle ? kRebuilders * 32 : 0),
           make_uint4(rb[0], rb[1], rb[2], rb[3]);
     };
     for (int i = rw; i < n_t; i += kRebuilders) {
-      const int s = i % NS;
+      const int s = i % NS, rs = i % sp.nrs;
       if (!__all_sync(0xffffffffu, mbar_wait(bars + 8 * s, (i / NS) & 1, abort))) break;
+      // the slot's previous tile has been read by its S product
+      if (i >= sp.nrs && !__all_sync(0xffffffffu, mbar_wait(bars + 8 * (3 * NS + rs),
+                                                             ((i / sp.nrs) - 1) & 1, abort)))
+        break;
       const long pos0 = (long)(t0 + i) * kKeys;
       const uint8_t* sk = smem + s * kStageB;
-      uint8_t* sr = smem + s * kStageB + Ly::kTile;  // rebuilt slots
+      uint8_t* sr = smem + sp.rb + rs * (sp.nrb * Ly::kBox);  // this tile's rebuilt boxes
       if (fixed_c) {
         if (j0 < kKeys) {
           float cs[8], sn[8];
@@ -366,6 +379,8 @@ __global__ void __launch_bounds__(kThreadsDm + (kSingle ? kRebuilders * 32 : 0),
       const uint32_t wbar = bars + 8 * ((kSingle ? 2 * NS : 0) + s);
       if (!__all_sync(0xffffffffu, mbar_wait(wbar, (i / NS) & 1, abort))) break;
       const uint32_t kb = base + s * kStageB, vb = kb + Ly::kTile;
+      // single-tensor: this tile's rebuilt boxes
+      const uint32_t rbb = kSingle ? base + sp.rb + (i % sp.nrs) * (sp.nrb * Ly::kBox) : 0u;
       const int pos0 = (t0 + i) * kKeys;
       if (pos0 + kKeys - 1 > P) {  // last tile: zero V rows past P (never written)
         const int first = P - pos0 + 1;
@@ -392,11 +407,15 @@ __global__ void __launch_bounds__(kThreadsDm + (kSingle ? kRebuilders * 32 : 0),
           uint32_t src = kb;
           if constexpr (kSingle) {
             const uint32_t sl = (sp.box_slot >> (4 * (kk >> 2))) & 15u;
-            if (sl != 15u) src = vb + sl * Ly::kBox - (kk >> 2) * Ly::kBox;
+            if (sl != 15u) src = rbb + sl * Ly::kBox - (kk >> 2) * Ly::kBox;
           }
           ldsm_x4(src + tile_off(key, kk * 16 + (mi >> 1) * 8), a);
           mma16816((kk & 1) ? sc2 : sc, a, qb[kk][0], qb[kk][1]);
         }
+      }
+      if constexpr (kSingle) {  // the rebuilt slot is free for the tile nrs later
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars + 8 * (3 * NS + i % sp.nrs));
       }
       // masked scores in log2 units: rows = keys pos0 + lane/4 (+8), cols = heads;
       // a padding key of the prompt (km) is masked like one outside [lo, P]
@@ -552,14 +571,21 @@ static cudaError_t run_mma(const LayerCfg& L, int B, const void* q_raw, const vo
         ++sp.nrb;
       }
     sp.nw = (R + 7) / 8 * 4;  // whole 16-byte chunks of each half
-    sp.stage = Ly::kTile + sp.nrb * Ly::kBox;
-    const uint32_t fixed = 8 * D * 2 + 3 * 16 * 8 + 16 * (uint32_t)R + 64;
+    sp.stage = Ly::kTile;
+    const uint32_t rbytes = sp.nrb * Ly::kBox;  // one rebuilt slot
+    const uint32_t fixed = 8 * D * 2 + (3 * 12 + 6) * 8 + 16 * (uint32_t)R + 64;
     const uint32_t budget = 227 * 1024 - 1024 - fixed;  // 1 KB: static shared memory
-    sp.ns = (int)std::min<uint32_t>(16, budget / sp.stage) & ~3;
-    if (sp.ns < 4 || (uint32_t)sp.ns * sp.stage < Ly::kMerge) return cudaErrorInvalidValue;
-    sp.q = sp.ns * sp.stage;
+    // 12 load stages (a multiple of the 4 consumers and the 3 rebuilders)
+    // and 6 rebuilt slots (a multiple of the rebuilders); the largest head
+    // (d 512: 16 KB tiles, two rebuilt boxes) fills the 227 KB with them
+    sp.ns = 4 * kRebuilders;
+    sp.nrs = 2 * kRebuilders;
+    if (sp.ns * sp.stage + sp.nrs * rbytes > budget || (uint32_t)sp.ns * sp.stage < Ly::kMerge)
+      return cudaErrorInvalidValue;
+    sp.rb = sp.ns * sp.stage;
+    sp.q = sp.rb + sp.nrs * rbytes;
     sp.bars = sp.q + 8 * D * 2;
-    sp.freq = (sp.bars + 3 * sp.ns * 8 + 15) & ~15u;
+    sp.freq = (sp.bars + (3 * sp.ns + sp.nrs) * 8 + 15) & ~15u;
     sp.wab = sp.freq + 8 * R;
     smem_bytes = sp.wab + 8 * R + 64;
   }

@@ -21,7 +21,12 @@
 // next.
 //   warp 0      TMA producer: x (128 x 64) and W (d x 64) per stage
 //   warp 1      owns TMEM; one thread issues raw (+)= x W^T, M 128, N <= 256, K 16
-//   warps 2..5  epilogue: TMEM lane quarter warp % 4
+//   warps 2..9  epilogue: TMEM lane quarter warp % 4, two warps per quarter;
+//               each of the two threads of a row sums the squares of the
+//               whole head and rotates, weights and stores half of its pairs
+//               (one warp per quarter left the epilogue slower than the MMAs
+//               of a tile at the E2B shape: the RoPE factors of 128 pairs a
+//               row are a long dependent chain per thread)
 // Every wait is bounded; on a timeout the CTA records G4ATTN_EDEVICE, lets
 // its copies and MMAs finish, frees TMEM and exits.
 #include <cuda.h>
@@ -41,7 +46,8 @@ namespace {
 
 constexpr int kQM = 128;  // tokens per tile (TMEM lanes)
 constexpr int kQK = 64;   // hidden dims per stage (one 128-byte swizzled row)
-constexpr int kQkvThreads = 192;
+constexpr int kQkvThreads = 320;
+constexpr int kEpiWarps = 8;  // warps 2 .. 9
 constexpr int kMaxGroupM = 32;
 
 template <int D>
@@ -179,10 +185,13 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
 // address tacc): RMSNorm over the head from the fp32 accumulator, the
 // weight and RoPE for query and key heads, bf16 stores of the rotated and /
 // or the weightless vectors.  Warp-collective (the TMEM loads).
+// half: which half of the rotation pairs (k, k + D/2) this thread takes
+// (the two threads of a row each read the whole head for the mean square).
 template <int D>
 __device__ __forceinline__ void qkv_epilogue_tile(const QkvArgs& a, uint32_t tacc, int m,
                                                   int head, const float* wsm,
-                                                  const unsigned long long* fq, int R) {
+                                                  const unsigned long long* fq, int R,
+                                                  int half) {
   // pass 1: the head's mean square, from the fp32 accumulator
   float ss = 0.f;
 #pragma unroll 1
@@ -220,9 +229,12 @@ __device__ __forceinline__ void qkv_epilogue_tile(const QkvArgs& a, uint32_t tac
     }
   }
   const bool rotate = is_q || is_k;  // warp-uniform: one head per tile
-  // pass 2: pairs (k, k + D/2), 32 at a time
+  // pass 2: pairs (k, k + D/2), 32 at a time; head_dim 64 has one chunk of
+  // 32 pairs, which the first thread of the row takes alone
+  constexpr int kPer = D / 2 >= 64 ? D / 4 : D / 2;  // pairs a thread takes
+  if (kPer * half >= D / 2) return;
 #pragma unroll 1
-  for (int c = 0; c < D / 2; c += 32) {
+  for (int c = kPer * half; c < kPer * (half + 1); c += 32) {
     uint32_t lo[32], hi[32];
     tmem_ld32(tacc + c, lo);
     tmem_ld32(tacc + D / 2 + c, hi);
@@ -311,7 +323,7 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(acc_full(i), 1);
-      mbar_init(acc_empty(i), 4);  // one arrival per epilogue warp
+      mbar_init(acc_empty(i), kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(drain, 1);
     s_abort = 0;
@@ -411,7 +423,7 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
       int mt, head;
       qkv_tile(a, t, &mt, &head);
       qkv_epilogue_tile<D>(a, tmem + lane_off + ai * D, mt * kQM + r, head, wsm, fq,
-                           rope.rotated_pairs);
+                           rope.rotated_pairs, (warp - 2) >> 2);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty(ai));  // the accumulator may take a new tile
@@ -437,7 +449,7 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
 //               CTAs are counted on the even CTA's full barrier
 //   warp 1      (both) TMEM allocation; (even) the MMA issuer, whose commits
 //               arrive on the barriers of both CTAs
-//   warps 2..5  (both) epilogue of this CTA's 128 rows; the odd CTA's warps
+//   warps 2..9  (both) epilogue of this CTA's 128 rows; the odd CTA's warps
 //               free an accumulator on the even CTA's barrier
 template <int D>
 __global__ void __launch_bounds__(kQkvThreads, 1)
@@ -483,7 +495,7 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(acc_full(i), 1);
-      mbar_init(acc_empty(i), 8);  // one arrival per epilogue warp of both CTAs
+      mbar_init(acc_empty(i), 2 * kEpiWarps);  // one arrival per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
     s_abort = 0;
@@ -589,7 +601,7 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
       int pt, head;
       qkv_tile(a, t, &pt, &head);
       qkv_epilogue_tile<D>(a, tmem + lane_off + ai * D, pt * (2 * kQM) + (int)rank * kQM + r,
-                           head, wsm, fq, rope.rotated_pairs);
+                           head, wsm, fq, rope.rotated_pairs, (warp - 2) >> 2);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(ae + 8u * (uint32_t)ai);

@@ -44,6 +44,10 @@ CASES = {
     "d64_bidirectional_queries_only": (W.bidirectional(4, 4, 64), 3, 130, 96, 0, None),
     "d512_single_tensor": (W.global_(8, 2, 512), 2, 140, 256, 7, "single"),
     "d256_global_separate_v": (W.global_(8, 2, 256, k_eq_v=False), 1, 390, 512, 0, "two"),
+    # at most 128 tokens: the single-CTA kernel (M 128 MMAs) instead of CTA pairs
+    "single_cta_d128_p0": (W.sliding(4, 2, 128, 64), 2, 50, 256, 10, "two"),
+    "single_cta_d512_k_eq_v_128_tokens": (W.global_(8, 1, 512), 1, 128, 192, 0, "two"),
+    "single_cta_d64_rolling": (W.sliding(2, 2, 64, 32), 1, 77, 64, 40, "rolling"),
 }
 
 
