@@ -10,6 +10,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "g4attn.h"
 #include "g4attn_internal.h"
@@ -18,6 +19,15 @@ namespace g4 {
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// An NVTX range over one entry point, so a profiler's timeline shows the
+// library's calls around their kernels (a no-op unless a tool is attached).
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 // The unique id of the calling thread's current CUDA context (cuCtxGetId:
 // never reused within a process, unlike the context handle).  Device
@@ -207,6 +217,7 @@ int g4attn_prefill(const g4attn_layer_desc* desc, int B, int T, const void* q_ra
                    const void* k_norm_w, const int32_t* image_block_ids,
                    const uint8_t* attention_mask, g4attn_cache* cache, void* out,
                    void* workspace, size_t ws_bytes, void* stream) {
+  g4::CallRange range("g4attn_prefill");
   LayerCfg L;
   int st = make_cfg(desc, &L);
   if (st != G4ATTN_OK) return st;
@@ -299,6 +310,7 @@ int g4attn_prefill_chunk(const g4attn_layer_desc* desc, int B, int T, int p0, co
                          const void* k_norm_w, const int32_t* image_block_ids,
                          const uint8_t* attention_mask, g4attn_cache* cache, void* out,
                          void* workspace, size_t ws_bytes, void* stream) {
+  g4::CallRange range("g4attn_prefill_chunk");
   LayerCfg L;
   int st = make_cfg(desc, &L);
   if (st != G4ATTN_OK) return st;
@@ -357,6 +369,7 @@ int g4attn_prefill_chunk(const g4attn_layer_desc* desc, int B, int T, int p0, co
 int g4attn_qkv_prologue(const g4attn_layer_desc* desc, int B, int T, int p0, const void* x,
                         int hidden, const void* w_qkv, const void* q_norm_w,
                         const void* k_norm_w, void* q_hat, g4attn_cache* cache, void* stream) {
+  g4::CallRange range("g4attn_qkv_prologue");
   LayerCfg L;
   int st = make_cfg(desc, &L);
   if (st != G4ATTN_OK) return st;
@@ -397,6 +410,7 @@ int g4attn_attend(const g4attn_layer_desc* desc, int B, int T, int p0, const voi
                   const int32_t* image_block_ids, const uint8_t* attention_mask,
                   const g4attn_cache* cache, void* out, void* workspace, size_t ws_bytes,
                   void* stream) {
+  g4::CallRange range("g4attn_attend");
   LayerCfg L;
   int st = make_cfg(desc, &L);
   if (st != G4ATTN_OK) return st;
@@ -437,6 +451,7 @@ int g4attn_attend(const g4attn_layer_desc* desc, int B, int T, int p0, const voi
 
 int g4attn_cache_append(const g4attn_layer_desc* desc, g4attn_cache* cache, const void* k_raw,
                         const void* v_raw, const void* k_norm_w, void* stream) {
+  g4::CallRange range("g4attn_cache_append");
   LayerCfg L;
   int st = make_cfg(desc, &L);
   if (st != G4ATTN_OK) return st;
@@ -454,6 +469,7 @@ int g4attn_cache_append(const g4attn_layer_desc* desc, g4attn_cache* cache, cons
 int g4attn_decode(const g4attn_layer_desc* desc, const g4attn_cache* cache, const void* q_raw,
                   const void* q_norm_w, void* out, void* workspace, size_t ws_bytes,
                   void* stream) {
+  g4::CallRange range("g4attn_decode");
   LayerCfg L;
   int st = make_cfg(desc, &L);
   if (st != G4ATTN_OK) return st;
@@ -479,6 +495,7 @@ int g4attn_decode(const g4attn_layer_desc* desc, const g4attn_cache* cache, cons
 
 int g4attn_decode_noalloc(const g4attn_layer_desc* desc, const g4attn_cache* cache,
                           const void* q_raw, const void* q_norm_w, void* out, void* stream) {
+  g4::CallRange range("g4attn_decode_noalloc");
   LayerCfg L;
   int st = make_cfg(desc, &L);
   if (st != G4ATTN_OK) return st;
